@@ -1,0 +1,248 @@
+"""Banded log-domain Sinkhorn attention on B200 (sm_100a).
+
+A thin ctypes binding over ``libsinkhorn_attn.so`` (C ABI declared in
+``include/sinkhorn_attn.h``).  The functions here carry the C entry points'
+names and only marshal arguments: they allocate the output, state and
+workspace tensors with PyTorch on the inputs' device, pass raw pointers and the
+current CUDA stream, and raise on a non-OK status.  Every step of the method
+runs in the library's CUDA kernels; there is no fallback of any kind, so a
+missing or unloadable library raises on first use.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libsinkhorn_attn.so")
+
+SA_OK = 0
+SA_F32, SA_BF16 = 0, 1
+SA_BWD_ONE_REFERENCE, SA_BWD_DIRECT = 0, 1
+_STATUS = {0: "SA_OK", -1: "SA_ERR_INVALID_ARG", -2: "SA_ERR_UNSUPPORTED",
+           -3: "SA_ERR_WORKSPACE", -4: "SA_ERR_CUDA", -5: "SA_ERR_NONFINITE",
+           -6: "SA_ERR_TIMEOUT"}
+SCHEDULES = {"one_reference": SA_BWD_ONE_REFERENCE, "direct": SA_BWD_DIRECT}
+
+
+class SinkhornAttnError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {_STATUS.get(status, status)} ({strerror(status)})")
+
+
+class sa_params(ctypes.Structure):
+    _fields_ = [
+        ("B", ctypes.c_int), ("H", ctypes.c_int), ("L", ctypes.c_int), ("d", ctypes.c_int),
+        ("W", ctypes.c_int), ("eps", ctypes.c_float), ("T", ctypes.c_int), ("R", ctypes.c_int),
+        ("dtype", ctypes.c_int), ("dustbin", ctypes.c_int), ("dustbin_score", ctypes.c_float),
+        ("bwd", ctypes.c_int), ("check_finite", ctypes.c_int),
+        ("trace_events", ctypes.c_void_p), ("trace_kinds", ctypes.c_void_p),
+        ("trace_count", ctypes.c_void_p), ("trace_cap", ctypes.c_int),
+    ]
+
+
+KERNEL_KINDS = {1: "lse_sweep", 2: "pv", 3: "wsum", 4: "ds", 5: "aux", 6: "fused_sweep"}
+
+
+class LaunchTrace:
+    """CUDA events recorded by the library around each of its kernel launches
+    (the ``trace_*`` fields of ``sa_params``).  Pass as ``trace=`` to the
+    forward/backward; after synchronising, ``durations()`` lists
+    ``(kind, milliseconds)`` per launch."""
+
+    def __init__(self, cap: int = 512):
+        self.cap = cap
+        self.events = [torch.cuda.Event(enable_timing=True) for _ in range(2 * cap)]
+        for e in self.events:
+            e.record()  # materialise the handle
+        self.handles = (ctypes.c_void_p * (2 * cap))(*[e.cuda_event for e in self.events])
+        self.kinds = (ctypes.c_int * cap)()
+        self.count = ctypes.c_int(0)
+
+    def attach(self, p: "sa_params"):
+        p.trace_events = ctypes.cast(self.handles, ctypes.c_void_p)
+        p.trace_kinds = ctypes.cast(self.kinds, ctypes.c_void_p)
+        p.trace_count = ctypes.cast(ctypes.pointer(self.count), ctypes.c_void_p)
+        p.trace_cap = self.cap
+
+    def durations(self):
+        n = min(self.count.value, self.cap)
+        return [(KERNEL_KINDS.get(self.kinds[i], str(self.kinds[i])),
+                 self.events[2 * i].elapsed_time(self.events[2 * i + 1])) for i in range(n)]
+
+
+_lib = None
+
+
+def _L():
+    """The loaded library; raises if it is missing (there is no fallback)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is missing: build it with `python -m banded_log_domain_b200.build` "
+            "(nvcc, sm_100a); there is no non-CUDA implementation")
+    lib = ctypes.CDLL(LIB_PATH)
+    P = ctypes.POINTER(sa_params)
+    vp, sz = ctypes.c_void_p, ctypes.c_size_t
+    lib.sinkhorn_attn_state_size.argtypes = [P, ctypes.POINTER(sz)]
+    lib.sinkhorn_attn_workspace_size.argtypes = [P, ctypes.POINTER(sz), ctypes.POINTER(sz)]
+    lib.sinkhorn_attn_fwd.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.sinkhorn_attn_bwd.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz,
+                                      vp]
+    lib.sinkhorn_attn_debug_plan.argtypes = [P, ctypes.c_int, ctypes.c_int, vp, vp, vp, vp, vp,
+                                             vp, vp, vp]
+    lib.sinkhorn_attn_poll.argtypes = [vp, vp]
+    lib.sinkhorn_attn_strerror.argtypes = [ctypes.c_int]
+    lib.sinkhorn_attn_strerror.restype = ctypes.c_char_p
+    for f in ("sinkhorn_attn_state_size", "sinkhorn_attn_workspace_size", "sinkhorn_attn_fwd",
+              "sinkhorn_attn_bwd", "sinkhorn_attn_debug_plan", "sinkhorn_attn_poll"):
+        getattr(lib, f).restype = ctypes.c_int
+    _lib = lib
+    return lib
+
+
+def load():
+    """Loads the CUDA library now (raises ImportError if it was not built)."""
+    return _L()
+
+
+EXPORTS = ("sinkhorn_attn_state_size", "sinkhorn_attn_workspace_size", "sinkhorn_attn_fwd",
+           "sinkhorn_attn_bwd", "sinkhorn_attn_debug_plan", "sinkhorn_attn_poll",
+           "sinkhorn_attn_strerror")
+
+
+def strerror(status: int) -> str:
+    return _L().sinkhorn_attn_strerror(int(status)).decode()
+
+
+def _check(rc: int, what: str):
+    if rc != SA_OK:
+        raise SinkhornAttnError(rc, what)
+
+
+def make_params(B, H, L, d, *, W, eps, T, R=2, dtype=torch.float32, dustbin=False,
+                dustbin_score=-2.0, schedule="one_reference", check_finite=False) -> sa_params:
+    dt = {torch.float32: SA_F32, torch.bfloat16: SA_BF16}[dtype]
+    return sa_params(int(B), int(H), int(L), int(d), int(W), float(eps), int(T), int(R), dt,
+                     int(bool(dustbin)), float(dustbin_score), SCHEDULES[schedule],
+                     int(bool(check_finite)))
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(device):
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def sinkhorn_attn_state_size(p: sa_params) -> int:
+    n = ctypes.c_size_t(0)
+    _check(_L().sinkhorn_attn_state_size(ctypes.byref(p), ctypes.byref(n)), "state_size")
+    return n.value
+
+
+def sinkhorn_attn_workspace_size(p: sa_params):
+    f, b = ctypes.c_size_t(0), ctypes.c_size_t(0)
+    _check(_L().sinkhorn_attn_workspace_size(ctypes.byref(p), ctypes.byref(f), ctypes.byref(b)),
+           "workspace_size")
+    return f.value, b.value
+
+
+def _params_for(q, W, eps, T, R, dustbin, dustbin_score, schedule, check_finite):
+    B, H, L, d = q.shape
+    return make_params(B, H, L, d, W=W, eps=eps, T=T, R=R, dtype=q.dtype, dustbin=dustbin,
+                       dustbin_score=dustbin_score, schedule=schedule,
+                       check_finite=check_finite)
+
+
+def _contig(*ts):
+    for t in ts:
+        if t is not None and not t.is_contiguous():
+            raise ValueError("tensors must be contiguous")
+
+
+def sinkhorn_attn_fwd(q, k, v, *, W, eps, T, R=2, mask=None, dustbin=False, dustbin_score=-2.0,
+                      v_dust=None, o=None, state=None, ws=None, check_finite=False, trace=None):
+    """Forward.  ``q, k, v``: ``[B,H,L,64]`` float32 or bfloat16 CUDA tensors;
+    ``mask``: ``[B,L]`` uint8 (1 = valid) or None; ``v_dust``: ``[H,64]`` float32.
+    Returns ``(o, state)``; ``state`` is ``[B,H,2R+2,L+dustbin]`` float32."""
+    _contig(q, k, v, mask, v_dust, o, state, ws)
+    p = _params_for(q, W, eps, T, R, dustbin, dustbin_score, "one_reference", check_finite)
+    if trace is not None:
+        trace.attach(p)
+    dev = q.device
+    if o is None:
+        o = torch.empty_like(q)
+    if state is None:
+        state = torch.empty(sinkhorn_attn_state_size(p), dtype=torch.float32, device=dev)
+    if ws is None:
+        ws = torch.zeros(sinkhorn_attn_workspace_size(p)[0], dtype=torch.uint8, device=dev)
+    rc = _L().sinkhorn_attn_fwd(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(mask),
+                                _ptr(v_dust), _ptr(o), _ptr(state), _ptr(ws), ws.numel(),
+                                _stream(dev))
+    _check(rc, "sinkhorn_attn_fwd")
+    B, H, L, _ = q.shape
+    return o, state.view(B, H, 2 * R + 2, L + int(bool(dustbin)))
+
+
+def sinkhorn_attn_bwd(q, k, v, o, dO, state, *, W, eps, R=2, mask=None, dustbin=False,
+                      dustbin_score=-2.0, v_dust=None, schedule="one_reference", dq=None, dk=None,
+                      dv=None, dv_dust=None, ws=None, check_finite=False, trace=None):
+    """Backward of <dO, O> through the tail.  Returns ``(dq, dk, dv, dv_dust)``
+    (``dv_dust`` is ``[H,64]`` float32 when ``dustbin``, else None)."""
+    _contig(q, k, v, o, dO, state, mask, v_dust, dq, dk, dv, dv_dust, ws)
+    p = _params_for(q, W, eps, 0, R, dustbin, dustbin_score, schedule, check_finite)
+    if trace is not None:
+        trace.attach(p)
+    dev = q.device
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(q) if dk is None else dk
+    dv = torch.empty_like(q) if dv is None else dv
+    if dustbin and dv_dust is None:
+        dv_dust = torch.empty(q.shape[1], q.shape[3], dtype=torch.float32, device=dev)
+    if ws is None:
+        ws = torch.zeros(sinkhorn_attn_workspace_size(p)[1], dtype=torch.uint8, device=dev)
+    rc = _L().sinkhorn_attn_bwd(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(mask),
+                                _ptr(v_dust), _ptr(o), _ptr(dO), _ptr(state), _ptr(dq), _ptr(dk),
+                                _ptr(dv), _ptr(dv_dust if dustbin else None), _ptr(ws),
+                                ws.numel(), _stream(dev))
+    _check(rc, "sinkhorn_attn_bwd")
+    return dq, dk, dv, (dv_dust if dustbin else None)
+
+
+def sinkhorn_attn_debug_plan(q, k, state, a, b, *, W, eps, R=2, mask=None, dustbin=False,
+                             dustbin_score=-2.0):
+    """``P^(a,b)``: ``band [B,H,L,2W+1]``, ``dcol [B,H,L]``, ``drow [B,H,L+1]``
+    (the last two only with ``dustbin``)."""
+    _contig(q, k, state, mask)
+    p = _params_for(q, W, eps, 0, R, dustbin, dustbin_score, "one_reference", False)
+    B, H, L, _ = q.shape
+    dev = q.device
+    band = torch.empty(B, H, L, 2 * W + 1, dtype=torch.float32, device=dev)
+    dcol = torch.empty(B, H, L, dtype=torch.float32, device=dev) if dustbin else None
+    drow = torch.empty(B, H, L + 1, dtype=torch.float32, device=dev) if dustbin else None
+    rc = _L().sinkhorn_attn_debug_plan(ctypes.byref(p), int(a), int(b), _ptr(q), _ptr(k),
+                                       _ptr(mask), _ptr(state), _ptr(band), _ptr(dcol),
+                                       _ptr(drow), _stream(dev))
+    _check(rc, "sinkhorn_attn_debug_plan")
+    return band, dcol, drow
+
+
+def sinkhorn_attn_poll(ws) -> int:
+    """Status word recorded in ``ws`` (after synchronising the current stream)."""
+    return int(_L().sinkhorn_attn_poll(_ptr(ws), _stream(ws.device)))
+
+
+def sinkhorn_attn_strerror(status: int) -> str:
+    return strerror(status)
+
+
+def score_scale(d: int, eps: float) -> float:
+    return 1.0 / (math.sqrt(d) * eps)

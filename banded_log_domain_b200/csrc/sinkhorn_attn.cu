@@ -1,0 +1,693 @@
+// C ABI of the banded log-domain Sinkhorn attention library: argument
+// validation, workspace layout and the launch sequence of each entry point.
+//
+// Forward (Block-Wise Differentiable Sinkhorn Attention, technical summary
+// section 2.1): v0 = 0; T base iterations and R tail iterations, each a row
+// sweep (u from v) followed by a column sweep (v from u); then O = P^(R,R) V.
+//
+// Backward (section 2.2), the one-reference schedule for general R:
+//   a      = rowdot(dO, O)
+//   dV     = P^T dO,                      vbar^R = rowdot(V, dV)      [key sweep]
+//   ubar^R = a - P vbar^R                                             [query sweep]
+//   for r = R..2:
+//     vbar^(r-1) = -ev^(r-1) . P^T (eu^r . ubar^r)                    [key sweep]
+//     ubar^(r-1) = -eu^(r-1) . P (ev^(r-1) . vbar^(r-1))              [query sweep]
+//   dS = P . M,  M = G - vbar^R_j - sum_r eu^r_i ev^(r-1)_j ubar^r_i
+//                               - sum_{r<R} eu^r_i ev^r_j vbar^r_j
+//   dQ = c dS K [query sweep],  dK = c dS^T Q [key sweep]
+// where P = P^(R,R), G_ij = <dO_i, V_j>, eu^a = exp(u^(a) - u^(R)) and
+// ev^b = exp(v^(b) - v^(R)) (the transport-orbit factors).  The direct
+// schedule runs the same sweeps with every staircase plan P^(r,r-1),
+// P^(r,r) formed by its own exponential.
+#include <cmath>
+#include <cstring>
+
+#include "../../include/sinkhorn_attn.h"
+#include "simt_sweep.cuh"
+
+namespace sa {
+namespace {
+
+constexpr size_t kHeader = 256;   // status word + padding at the start of every workspace
+constexpr int kD = simt::D;
+
+size_t align_up(size_t x) { return (x + 255) & ~size_t(255); }
+
+struct Dims {
+    int B, H, L, R, ld, BH;
+    bool ok;
+};
+
+sa_status check_params(const sa_params* p, Dims* dd) {
+    if (!p) return SA_ERR_INVALID_ARG;
+    if (p->B < 0 || p->H < 0 || p->L < 0 || p->d <= 0 || p->W < 0 || p->T < 0 || p->R < 1)
+        return SA_ERR_INVALID_ARG;
+    if (!(p->eps > 0.f) || !std::isfinite(p->eps)) return SA_ERR_INVALID_ARG;
+    if (p->dtype != SA_F32 && p->dtype != SA_BF16) return SA_ERR_INVALID_ARG;
+    if (p->dustbin != 0 && p->dustbin != 1) return SA_ERR_INVALID_ARG;
+    if (p->dustbin && !std::isfinite(p->dustbin_score)) return SA_ERR_INVALID_ARG;
+    if (p->bwd != SA_BWD_ONE_REFERENCE && p->bwd != SA_BWD_DIRECT) return SA_ERR_INVALID_ARG;
+    if (p->check_finite != 0 && p->check_finite != 1) return SA_ERR_INVALID_ARG;
+    if (p->d != kD) return SA_ERR_UNSUPPORTED;
+    if (p->R > 4) return SA_ERR_UNSUPPORTED;
+    const long long BH = (long long)p->B * p->H;
+    if (BH > 65535) return SA_ERR_UNSUPPORTED;
+    if ((long long)p->L * kD > (1LL << 40)) return SA_ERR_UNSUPPORTED;
+    dd->B = p->B;
+    dd->H = p->H;
+    dd->L = p->L;
+    dd->R = p->R;
+    dd->ld = p->L + p->dustbin;
+    dd->BH = (int)BH;
+    dd->ok = true;
+    return SA_OK;
+}
+
+bool aligned16(const void* x) { return ((uintptr_t)x & 15u) == 0; }
+
+// Rejects pointers the device cannot dereference (plain pageable host memory).
+bool device_ok(const void* x) {
+    if (!x || !aligned16(x)) return false;
+    cudaPointerAttributes at;
+    if (cudaPointerGetAttributes(&at, x) != cudaSuccess) {
+        cudaGetLastError();
+        return false;
+    }
+    return at.type == cudaMemoryTypeDevice || at.type == cudaMemoryTypeManaged ||
+           at.type == cudaMemoryTypeHost;
+}
+bool mask_ok(const void* x) {
+    if (!x) return true;
+    cudaPointerAttributes at;
+    if (cudaPointerGetAttributes(&at, x) != cudaSuccess) {
+        cudaGetLastError();
+        return false;
+    }
+    return at.type != cudaMemoryTypeUnregistered;
+}
+
+// Backward workspace layout (float32 vectors of BH * ld elements each).
+struct BwdLayout {
+    size_t a, ubar, vbar, eu, ev, w, rv, cv, dvd, total;
+    size_t vec;  // bytes of one [BH][ld] vector, 256-aligned
+};
+BwdLayout bwd_layout(const Dims& d) {
+    BwdLayout l;
+    l.vec = align_up((size_t)d.BH * d.ld * sizeof(float));
+    size_t o = kHeader;
+    l.a = o;    o += l.vec;
+    l.ubar = o; o += l.vec * (d.R + 1);   // index r = 0..R (0 unused)
+    l.vbar = o; o += l.vec * (d.R + 1);
+    l.eu = o;   o += l.vec * (d.R + 1);
+    l.ev = o;   o += l.vec * (d.R + 1);
+    l.w = o;    o += l.vec;
+    l.rv = o;   o += l.vec * 2 * d.R;
+    l.cv = o;   o += l.vec * 2 * d.R;
+    l.dvd = o;  o += align_up((size_t)d.BH * kD * sizeof(float));
+    l.total = o;
+    return l;
+}
+
+// ---------------------------------------------------------------------------
+// small elementwise kernels
+// ---------------------------------------------------------------------------
+
+// out[bh][t] = <X_t, Y_t> over d for valid tokens, 0 for masked ones and for
+// the dustbin slot t = L.  One warp per token.
+template <typename T>
+__global__ void k_rowdot(const T* X, const T* Y, const uint8_t* mask, int L, int H, int ld,
+                         int BH, float* out) {
+    const long long gw = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    if (gw >= (long long)BH * ld) return;
+    const int bh = (int)(gw / ld), t = (int)(gw % ld);
+    float s = 0.f;
+    const bool ok = t < L && (mask == nullptr || mask[(size_t)(bh / H) * L + t]);
+    if (ok) {
+        const size_t o = ((size_t)bh * L + t) * kD;
+        for (int e = lane; e < kD; e += 32) s = fmaf(to_f32(X[o + e]), to_f32(Y[o + e]), s);
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+    if (lane == 0) out[(size_t)bh * ld + t] = s;
+}
+
+// eu[a][bh][t] = exp(u^(a) - u^(R)), ev[a][bh][t] = exp(v^(a) - v^(R)), a = 0..R;
+// zero on masked tokens.  state: [BH][2R+2][ld].
+__global__ void k_orbit(const float* state, int R, int L, int H, int ld, int BH,
+                        const uint8_t* mask, float* eu, float* ev, size_t vstride) {
+    const long long g = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (g >= (long long)BH * ld) return;
+    const int bh = (int)(g / ld), t = (int)(g % ld);
+    const bool ok = t >= L || mask == nullptr || mask[(size_t)(bh / H) * L + t];
+    const float* st = state + (size_t)bh * (2 * R + 2) * ld;
+    const float uR = st[(size_t)(2 * R) * ld + t], vR = st[(size_t)(2 * R + 1) * ld + t];
+    for (int a = 0; a <= R; ++a) {
+        const float ua = st[(size_t)(2 * a) * ld + t], va = st[(size_t)(2 * a + 1) * ld + t];
+        eu[a * vstride + g] = ok ? ex2((ua - uR) * kLog2e) : 0.f;
+        ev[a * vstride + g] = ok ? ex2((va - vR) * kLog2e) : 0.f;
+    }
+}
+
+// out = s * x * y elementwise over BH*ld (x or y null means 1).
+__global__ void k_vmul(const float* x, const float* y, float s, float* out, long long n) {
+    const long long g = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (g >= n) return;
+    float v = s;
+    if (x) v *= x[g];
+    if (y) v *= y[g];
+    out[g] = v;
+}
+
+// dv_dust[h][e] = sum_b part[(b*H + h)][e]
+__global__ void k_dvd_reduce(const float* part, int B, int H, float* out) {
+    const int g = blockIdx.x * blockDim.x + threadIdx.x;
+    if (g >= H * kD) return;
+    const int h = g / kD, e = g % kD;
+    float s = 0.f;
+    for (int b = 0; b < B; ++b) s += part[((size_t)b * H + h) * kD + e];
+    out[g] = s;
+}
+
+// Sets the status word when any element is NaN or Inf.
+template <typename T>
+__global__ void k_finite(const T* x, long long n, int* status) {
+    const long long g = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    bool bad = false;
+    for (long long i = g; i < n; i += (long long)gridDim.x * blockDim.x)
+        if (!isfinite(to_f32(x[i]))) bad = true;
+    if (__any_sync(0xffffffffu, bad) && (threadIdx.x & 31) == 0)
+        atomicCAS(status, (int)SA_OK, (int)SA_ERR_NONFINITE);
+}
+
+// P^(a,b) in band layout; scores with the same fp32 FMA order as the sweeps.
+template <typename T>
+__global__ void k_debug_plan(const T* q, const T* k, const uint8_t* mask, const float* state,
+                             int a, int b, int R, int L, int H, int W, int ld, float c2,
+                             int dustbin, float sd2, float* band, float* dcol, float* drow) {
+    const int bh = blockIdx.y;
+    const int i = blockIdx.x;
+    const int bw = 2 * W + 1;
+    const uint8_t* mk = mask ? mask + (size_t)(bh / H) * L : nullptr;
+    const float* st = state + (size_t)bh * (2 * R + 2) * ld;
+    const float* ua = st + (size_t)(2 * a) * ld;
+    const float* vb = st + (size_t)(2 * b + 1) * ld;
+    if (i == L) {  // dustbin row
+        if (!dustbin || !drow) return;
+        for (int j = threadIdx.x; j <= L; j += blockDim.x) {
+            float v = 0.f;
+            if (j == L || !mk || mk[j]) v = ex2(sd2 + (ua[L] + vb[j]) * kLog2e);
+            drow[(size_t)bh * (L + 1) + j] = v;
+        }
+        return;
+    }
+    const bool vi = !mk || mk[i];
+    const T* qi = q + ((size_t)bh * L + i) * kD;
+    for (int t = threadIdx.x; t < bw; t += blockDim.x) {
+        const int j = i - W + t;
+        float v = 0.f;
+        if (vi && j >= 0 && j < L && (!mk || mk[j])) {
+            const T* kj = k + ((size_t)bh * L + j) * kD;
+            float acc = 0.f;
+            for (int e = 0; e < kD; ++e) acc = fmaf(to_f32(qi[e]), to_f32(kj[e]), acc);
+            v = ex2(fmaf(c2, acc, (ua[i] + vb[j]) * kLog2e));
+        }
+        band[((size_t)bh * L + i) * bw + t] = v;
+    }
+    if (dustbin && dcol && threadIdx.x == 0)
+        dcol[(size_t)bh * L + i] = vi ? ex2(sd2 + (ua[i] + vb[L]) * kLog2e) : 0.f;
+}
+
+// ---------------------------------------------------------------------------
+// launch helpers
+// ---------------------------------------------------------------------------
+
+// Optional launch trace (sa_params.trace_*): caller-owned CUDA events recorded
+// on the call's stream around each kernel launch.
+struct Tracer {
+    const sa_params* p = nullptr;
+    cudaStream_t st = nullptr;
+    int n = 0;
+    bool on() const { return p->trace_events && p->trace_cap > 0 && n < p->trace_cap; }
+    void begin(int kind) {
+        if (!on()) return;
+        cudaEventRecord((cudaEvent_t)p->trace_events[2 * n], st);
+        if (p->trace_kinds) p->trace_kinds[n] = kind;
+    }
+    void end() {
+        if (on()) cudaEventRecord((cudaEvent_t)p->trace_events[2 * n + 1], st);
+        ++n;
+        if (p->trace_count) *p->trace_count = n;
+    }
+};
+
+constexpr int kind_of(int mode) {
+    return mode == simt::LSE ? SA_KERNEL_LSE_SWEEP
+         : mode == simt::PV ? SA_KERNEL_PV
+         : mode == simt::WSUM ? SA_KERNEL_WSUM : SA_KERNEL_DS;
+}
+
+template <typename T, int MODE>
+cudaError_t launch_sweep(const simt::SweepArgs& a, int BH, cudaStream_t st, Tracer& tr) {
+    const int nblk = (a.L + simt::BM - 1) / simt::BM;
+    const dim3 grid(nblk + (a.dust_cta ? 1 : 0), BH);
+    const size_t smem = (size_t)simt::smem_floats(MODE) * sizeof(float);
+    cudaError_t e = cudaFuncSetAttribute(simt::band_sweep<T, MODE>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    tr.begin(kind_of(MODE));
+    simt::band_sweep<T, MODE><<<grid, simt::NT, smem, st>>>(a);
+    tr.end();
+    return cudaGetLastError();
+}
+
+#define SA_AUX(tr, ...)                        \
+    do {                                       \
+        (tr).begin(SA_KERNEL_AUX);             \
+        __VA_ARGS__;                           \
+        (tr).end();                            \
+        SA_CUDA(cudaGetLastError());           \
+    } while (0)
+
+Vec vec(const float* p, long long s) { return Vec{p, s}; }
+MVec mvec(float* p, long long s) { return MVec{p, s}; }
+
+struct Ctx {
+    const sa_params* p;
+    Dims d;
+    cudaStream_t st;
+    float c;     // natural score scale 1/(sqrt(d) eps)
+    long long sst;  // per-bh stride of a state row: (2R+2)*ld
+    const float* state;
+    mutable Tracer tr;
+    // state row r (0..2R+1) as a Vec
+    Vec srow(int r) const { return vec(state + (size_t)r * d.ld, sst); }
+};
+
+simt::SweepArgs base_args(const Ctx& x) {
+    simt::SweepArgs a;
+    std::memset(&a, 0, sizeof(a));
+    a.L = x.d.L;
+    a.W = x.p->W;
+    a.H = x.d.H;
+    a.ld = x.d.ld;
+    a.c2 = x.c * kLog2e;
+    a.dustbin = x.p->dustbin;
+    a.dust_cta = x.p->dustbin;
+    a.sd2 = x.p->dustbin ? x.p->dustbin_score * kLog2e : 0.f;
+    a.sgn = 1.f;
+    a.out_scale = x.c;
+    return a;
+}
+
+#define SA_CUDA(call)                              \
+    do {                                           \
+        cudaError_t e_ = (call);                   \
+        if (e_ != cudaSuccess) return SA_ERR_CUDA; \
+    } while (0)
+
+template <typename T>
+sa_status fwd_impl(const Ctx& x, const T* q, const T* k, const T* v, const uint8_t* mask,
+                   const float* v_dust, T* o, float* state) {
+    const Dims& d = x.d;
+    // v0 = 0 and u0 = 0 (u0 stays 0 when T == 0)
+    SA_CUDA(cudaMemsetAsync(state, 0, (size_t)d.BH * (2 * d.R + 2) * d.ld * sizeof(float), x.st));
+    simt::SweepArgs a = base_args(x);
+    a.mask = mask;
+    const int iters = x.p->T + d.R;
+    for (int it = 0; it < iters; ++it) {
+        const int rin = it < x.p->T ? 0 : it - x.p->T;       // v index read
+        const int rout = it < x.p->T ? 0 : it - x.p->T + 1;  // u, v index written
+        // rows: u^(rout) = -LSE_j(S + v^(rin))
+        a.A = q; a.Bo = k;
+        a.cd = x.srow(2 * rin + 1);
+        a.out_vec = mvec(state + (size_t)(2 * rout) * d.ld, x.sst);
+        SA_CUDA((launch_sweep<T, simt::LSE>(a, d.BH, x.st, x.tr)));
+        // columns: v^(rout) = -LSE_i(S + u^(rout))
+        a.A = k; a.Bo = q;
+        a.cd = x.srow(2 * rout);
+        a.out_vec = mvec(state + (size_t)(2 * rout + 1) * d.ld, x.sst);
+        SA_CUDA((launch_sweep<T, simt::LSE>(a, d.BH, x.st, x.tr)));
+    }
+    // O = P^(R,R) V (+ dustbin column times v_dust)
+    simt::SweepArgs b = base_args(x);
+    b.mask = mask;
+    b.dust_cta = 0;
+    b.A = q; b.Bo = k; b.X = v;
+    b.Xd = v_dust;
+    b.rd = x.srow(2 * d.R);
+    b.cd = x.srow(2 * d.R + 1);
+    b.out_mat = o;
+    SA_CUDA((launch_sweep<T, simt::PV>(b, d.BH, x.st, x.tr)));
+    return SA_OK;
+}
+
+template <typename T>
+sa_status bwd_impl(const Ctx& x, const T* q, const T* k, const T* v, const uint8_t* mask,
+                   const float* v_dust, const T* o, const T* dO, T* dq, T* dk, T* dv,
+                   float* dv_dust, char* ws) {
+    const Dims& d = x.d;
+    const int R = d.R;
+    const BwdLayout l = bwd_layout(d);
+    const long long vs = d.ld;  // per-bh stride of a workspace vector
+    const size_t vstride = l.vec / sizeof(float);
+    auto W_ = [&](size_t off, int idx) { return (float*)(ws + off + (size_t)idx * l.vec); };
+    float* A_ = W_(l.a, 0);
+    float* dvd = (float*)(ws + l.dvd);
+    const long long nvec = (long long)d.BH * d.ld;
+    const int eb = 256;
+    const unsigned egrid = (unsigned)((nvec + eb - 1) / eb);
+    const bool direct = x.p->bwd == SA_BWD_DIRECT;
+
+    // a = rowdot(dO, O); orbit factors
+    {
+        const long long thr = nvec * 32;
+        SA_AUX(x.tr, k_rowdot<T><<<(unsigned)((thr + 255) / 256), 256, 0, x.st>>>(
+                         dO, o, mask, d.L, d.H, d.ld, d.BH, A_));
+        SA_AUX(x.tr, k_orbit<<<egrid, eb, 0, x.st>>>(x.state, R, d.L, d.H, d.ld, d.BH, mask,
+                                                     W_(l.eu, 0), W_(l.ev, 0), vstride));
+    }
+    const Vec uR = x.srow(2 * R), vR = x.srow(2 * R + 1);
+    auto U = [&](int r) { return x.srow(2 * r); };
+    auto V = [&](int r) { return x.srow(2 * r + 1); };
+    auto ub = [&](int r) { return W_(l.ubar, r); };
+    auto vb = [&](int r) { return W_(l.vbar, r); };
+    auto eu = [&](int r) { return W_(l.eu, r); };
+    auto ev = [&](int r) { return W_(l.ev, r); };
+
+    // dV = P^T dO, vbar^R = rowdot(V, dV)  (key sweep; dustbin row: dv_dust partials)
+    {
+        simt::SweepArgs a = base_args(x);
+        a.mask = mask;
+        a.A = k; a.Bo = q; a.X = dO; a.Y = v;
+        a.Yd = v_dust;
+        a.rd = vR; a.cd = uR;
+        a.out_mat = dv;
+        a.out_vec = mvec(vb(R), vs);
+        a.dvd_part = dvd;
+        SA_CUDA((launch_sweep<T, simt::PV>(a, d.BH, x.st, x.tr)));
+    }
+    // ubar^R = a - P vbar^R  (query sweep)
+    {
+        simt::SweepArgs a = base_args(x);
+        a.mask = mask;
+        a.A = q; a.Bo = k;
+        a.rd = uR; a.cd = vR;
+        a.w = vec(vb(R), vs);
+        a.base = vec(A_, vs);
+        a.sgn = -1.f;
+        a.out_vec = mvec(ub(R), vs);
+        SA_CUDA((launch_sweep<T, simt::WSUM>(a, d.BH, x.st, x.tr)));
+    }
+    for (int r = R; r >= 2; --r) {
+        // vbar^(r-1) = -P^(r,r-1)^T ubar^r
+        simt::SweepArgs a = base_args(x);
+        a.mask = mask;
+        a.A = k; a.Bo = q;
+        a.sgn = -1.f;
+        a.out_vec = mvec(vb(r - 1), vs);
+        if (direct) {
+            a.rd = V(r - 1); a.cd = U(r);
+            a.w = vec(ub(r), vs);
+        } else {
+            SA_AUX(x.tr, k_vmul<<<egrid, eb, 0, x.st>>>(eu(r), ub(r), 1.f, W_(l.w, 0), nvec));
+            a.rd = vR; a.cd = uR;
+            a.w = vec(W_(l.w, 0), vs);
+            a.mult = vec(ev(r - 1), vs);
+        }
+        SA_CUDA((launch_sweep<T, simt::WSUM>(a, d.BH, x.st, x.tr)));
+        // ubar^(r-1) = -P^(r-1,r-1) vbar^(r-1)
+        simt::SweepArgs b = base_args(x);
+        b.mask = mask;
+        b.A = q; b.Bo = k;
+        b.sgn = -1.f;
+        b.out_vec = mvec(ub(r - 1), vs);
+        if (direct) {
+            b.rd = U(r - 1); b.cd = V(r - 1);
+            b.w = vec(vb(r - 1), vs);
+        } else {
+            SA_AUX(x.tr, k_vmul<<<egrid, eb, 0, x.st>>>(ev(r - 1), vb(r - 1), 1.f, W_(l.w, 0), nvec));
+            b.rd = uR; b.cd = vR;
+            b.w = vec(W_(l.w, 0), vs);
+            b.mult = vec(eu(r - 1), vs);
+        }
+        SA_CUDA((launch_sweep<T, simt::WSUM>(b, d.BH, x.st, x.tr)));
+    }
+
+    // modifier / staircase terms, query side (rq) and key side (rk)
+    //   one reference:  M = G + sum_k rq_k[i] rk_k[j]
+    //     k=0: (1, -vbar^R);  r=1..R: (-eu^r ubar^r, ev^(r-1));  r=1..R-1: (-eu^r, ev^r vbar^r)
+    //   direct: dS = sum_k exp(S + eq_k[i] + ek_k[j]) (g_k G + cq_k[i] + ck_k[j])
+    //     k=0: (u^R, v^R; G - vbar^R);  r: (u^r, v^(r-1); -ubar^r);  r<R: (u^r, v^r; -vbar^r)
+    int nt = 0;
+    Vec rq[simt::MAXT], rk[simt::MAXT];
+    Vec eq[simt::MAXT], ek[simt::MAXT], cq[simt::MAXT], ck[simt::MAXT];
+    float gk[simt::MAXT];
+    const Vec none{nullptr, 0};
+    auto slot_q = [&](int i) { return (float*)(ws + l.rv + (size_t)i * l.vec); };
+    auto slot_k = [&](int i) { return (float*)(ws + l.cv + (size_t)i * l.vec); };
+    {
+        // k = 0
+        SA_AUX(x.tr, k_vmul<<<egrid, eb, 0, x.st>>>(vb(R), nullptr, -1.f, slot_k(0), nvec));
+        rq[nt] = none; rk[nt] = vec(slot_k(0), vs);
+        eq[nt] = uR; ek[nt] = vR; cq[nt] = none; ck[nt] = vec(slot_k(0), vs); gk[nt] = 1.f;
+        ++nt;
+        for (int r = 1; r <= R; ++r) {
+            if (direct) {
+                SA_AUX(x.tr, k_vmul<<<egrid, eb, 0, x.st>>>(ub(r), nullptr, -1.f, slot_q(nt), nvec));
+            } else {
+                SA_AUX(x.tr, k_vmul<<<egrid, eb, 0, x.st>>>(eu(r), ub(r), -1.f, slot_q(nt), nvec));
+            }
+            rq[nt] = vec(slot_q(nt), vs); rk[nt] = vec(ev(r - 1), vs);
+            eq[nt] = U(r); ek[nt] = V(r - 1); cq[nt] = vec(slot_q(nt), vs); ck[nt] = none;
+            gk[nt] = 0.f;
+            ++nt;
+        }
+        for (int r = 1; r < R; ++r) {
+            if (direct) {
+                SA_AUX(x.tr, k_vmul<<<egrid, eb, 0, x.st>>>(vb(r), nullptr, -1.f, slot_k(nt), nvec));
+                eq[nt] = U(r); ek[nt] = V(r); cq[nt] = none; ck[nt] = vec(slot_k(nt), vs);
+                gk[nt] = 0.f;
+            } else {
+                SA_AUX(x.tr, k_vmul<<<egrid, eb, 0, x.st>>>(eu(r), nullptr, -1.f, slot_q(nt), nvec));
+                SA_AUX(x.tr, k_vmul<<<egrid, eb, 0, x.st>>>(ev(r), vb(r), 1.f, slot_k(nt), nvec));
+                rq[nt] = vec(slot_q(nt), vs); rk[nt] = vec(slot_k(nt), vs);
+            }
+            ++nt;
+        }
+    }
+    // dQ (query sweep) and dK (key sweep)
+    for (int side = 0; side < 2; ++side) {
+        simt::SweepArgs a = base_args(x);
+        a.mask = mask;
+        a.dust_cta = 0;
+        a.nterms = nt;
+        if (side == 0) {
+            a.A = q; a.Bo = k; a.A2 = dO; a.B2 = v; a.X = k;
+            a.rd = uR; a.cd = vR;
+            a.out_mat = dq;
+            for (int t = 0; t < nt; ++t) {
+                a.rv[t] = rq[t]; a.cv[t] = rk[t];
+                a.er[t] = eq[t]; a.ec[t] = ek[t]; a.cr[t] = cq[t]; a.cc[t] = ck[t];
+                a.gk[t] = gk[t];
+            }
+        } else {
+            a.A = k; a.Bo = q; a.A2 = v; a.B2 = dO; a.X = q;
+            a.rd = vR; a.cd = uR;
+            a.out_mat = dk;
+            for (int t = 0; t < nt; ++t) {
+                a.rv[t] = rk[t]; a.cv[t] = rq[t];
+                a.er[t] = ek[t]; a.ec[t] = eq[t]; a.cr[t] = ck[t]; a.cc[t] = cq[t];
+                a.gk[t] = gk[t];
+            }
+        }
+        if (direct) SA_CUDA((launch_sweep<T, simt::DSD>(a, d.BH, x.st, x.tr)));
+        else SA_CUDA((launch_sweep<T, simt::DS1>(a, d.BH, x.st, x.tr)));
+    }
+    if (x.p->dustbin && dv_dust) {
+        SA_AUX(x.tr, k_dvd_reduce<<<(d.H * kD + 255) / 256, 256, 0, x.st>>>(dvd, d.B, d.H,
+                                                                            dv_dust));
+    }
+    return SA_OK;
+}
+
+template <typename T>
+cudaError_t scan_finite(const T* x, long long n, int* status, cudaStream_t st) {
+    if (n <= 0) return cudaSuccess;
+    long long blocks = (n + 255) / 256;
+    if (blocks > 4096) blocks = 4096;
+    k_finite<T><<<(unsigned)blocks, 256, 0, st>>>(x, n, status);
+    return cudaGetLastError();
+}
+
+}  // namespace
+}  // namespace sa
+
+using namespace sa;
+
+extern "C" {
+
+sa_status sinkhorn_attn_state_size(const sa_params* p, size_t* n_floats) {
+    Dims d;
+    sa_status s = check_params(p, &d);
+    if (s != SA_OK) return s;
+    if (!n_floats) return SA_ERR_INVALID_ARG;
+    *n_floats = (size_t)d.BH * (2 * d.R + 2) * d.ld;
+    return SA_OK;
+}
+
+sa_status sinkhorn_attn_workspace_size(const sa_params* p, size_t* fwd_bytes, size_t* bwd_bytes) {
+    Dims d;
+    sa_status s = check_params(p, &d);
+    if (s != SA_OK) return s;
+    if (fwd_bytes) *fwd_bytes = kHeader;
+    if (bwd_bytes) *bwd_bytes = bwd_layout(d).total;
+    return SA_OK;
+}
+
+sa_status sinkhorn_attn_fwd(const sa_params* p, const void* q, const void* k, const void* v,
+                            const uint8_t* mask, const float* v_dust, void* o, float* state,
+                            void* ws, size_t ws_bytes, void* stream) {
+    Dims d;
+    sa_status s = check_params(p, &d);
+    if (s != SA_OK) return s;
+    if (ws_bytes < kHeader) return SA_ERR_WORKSPACE;
+    if (d.BH == 0 || d.L == 0) return SA_OK;
+    if (!device_ok(q) || !device_ok(k) || !device_ok(v) || !device_ok(o) || !device_ok(state) ||
+        !device_ok(ws) || !mask_ok(mask))
+        return SA_ERR_INVALID_ARG;
+    if (p->dustbin && v_dust && !device_ok(v_dust)) return SA_ERR_INVALID_ARG;
+    Ctx x;
+    x.p = p;
+    x.d = d;
+    x.st = (cudaStream_t)stream;
+    x.c = 1.0f / (std::sqrt((float)p->d) * p->eps);
+    x.sst = (long long)(2 * d.R + 2) * d.ld;
+    x.state = state;
+    x.tr.p = p;
+    x.tr.st = x.st;
+    const float* vd = p->dustbin ? v_dust : nullptr;
+    if (p->dtype == SA_F32)
+        s = fwd_impl<float>(x, (const float*)q, (const float*)k, (const float*)v, mask, vd,
+                            (float*)o, state);
+    else
+        s = fwd_impl<__nv_bfloat16>(x, (const __nv_bfloat16*)q, (const __nv_bfloat16*)k,
+                                    (const __nv_bfloat16*)v, mask, vd, (__nv_bfloat16*)o, state);
+    if (s != SA_OK) return s;
+    if (p->check_finite) {
+        int* status = (int*)ws;
+        const long long n = (long long)d.BH * d.L * kD;
+        if (scan_finite<float>(state, (long long)d.BH * (2 * d.R + 2) * d.ld, status, x.st) !=
+            cudaSuccess)
+            return SA_ERR_CUDA;
+        cudaError_t e = p->dtype == SA_F32
+                            ? scan_finite<float>((const float*)o, n, status, x.st)
+                            : scan_finite<__nv_bfloat16>((const __nv_bfloat16*)o, n, status, x.st);
+        if (e != cudaSuccess) return SA_ERR_CUDA;
+    }
+    return SA_OK;
+}
+
+sa_status sinkhorn_attn_bwd(const sa_params* p, const void* q, const void* k, const void* v,
+                            const uint8_t* mask, const float* v_dust, const void* o,
+                            const void* dO, const float* state, void* dq, void* dk, void* dv,
+                            float* dv_dust, void* ws, size_t ws_bytes, void* stream) {
+    Dims d;
+    sa_status s = check_params(p, &d);
+    if (s != SA_OK) return s;
+    if (ws_bytes < bwd_layout(d).total) return SA_ERR_WORKSPACE;
+    if (d.BH == 0 || d.L == 0) return SA_OK;
+    if (!device_ok(q) || !device_ok(k) || !device_ok(v) || !device_ok(o) || !device_ok(dO) ||
+        !device_ok(state) || !device_ok(dq) || !device_ok(dk) || !device_ok(dv) ||
+        !device_ok(ws) || !mask_ok(mask))
+        return SA_ERR_INVALID_ARG;
+    if (p->dustbin && v_dust && !device_ok(v_dust)) return SA_ERR_INVALID_ARG;
+    if (p->dustbin && dv_dust && !device_ok(dv_dust)) return SA_ERR_INVALID_ARG;
+    Ctx x;
+    x.p = p;
+    x.d = d;
+    x.st = (cudaStream_t)stream;
+    x.c = 1.0f / (std::sqrt((float)p->d) * p->eps);
+    x.sst = (long long)(2 * d.R + 2) * d.ld;
+    x.state = state;
+    x.tr.p = p;
+    x.tr.st = x.st;
+    const float* vd = p->dustbin ? v_dust : nullptr;
+    float* dvd = p->dustbin ? dv_dust : nullptr;
+    if (p->dtype == SA_F32)
+        s = bwd_impl<float>(x, (const float*)q, (const float*)k, (const float*)v, mask, vd,
+                            (const float*)o, (const float*)dO, (float*)dq, (float*)dk, (float*)dv,
+                            dvd, (char*)ws);
+    else
+        s = bwd_impl<__nv_bfloat16>(
+            x, (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v, mask, vd,
+            (const __nv_bfloat16*)o, (const __nv_bfloat16*)dO, (__nv_bfloat16*)dq,
+            (__nv_bfloat16*)dk, (__nv_bfloat16*)dv, dvd, (char*)ws);
+    if (s != SA_OK) return s;
+    if (p->check_finite) {
+        int* status = (int*)ws;
+        const long long n = (long long)d.BH * d.L * kD;
+        for (const void* t : {(const void*)dq, (const void*)dk, (const void*)dv}) {
+            cudaError_t e =
+                p->dtype == SA_F32
+                    ? scan_finite<float>((const float*)t, n, status, x.st)
+                    : scan_finite<__nv_bfloat16>((const __nv_bfloat16*)t, n, status, x.st);
+            if (e != cudaSuccess) return SA_ERR_CUDA;
+        }
+    }
+    return SA_OK;
+}
+
+sa_status sinkhorn_attn_debug_plan(const sa_params* p, int a, int b, const void* q,
+                                   const void* k, const uint8_t* mask, const float* state,
+                                   float* band, float* dcol, float* drow, void* stream) {
+    Dims d;
+    sa_status s = check_params(p, &d);
+    if (s != SA_OK) return s;
+    if (a < 0 || b < 0 || a > d.R || b > d.R) return SA_ERR_INVALID_ARG;
+    if (d.BH == 0 || d.L == 0) return SA_OK;
+    if (!device_ok(q) || !device_ok(k) || !device_ok(state) || !device_ok(band) ||
+        !mask_ok(mask))
+        return SA_ERR_INVALID_ARG;
+    if (p->dustbin && ((dcol && !device_ok(dcol)) || (drow && !device_ok(drow))))
+        return SA_ERR_INVALID_ARG;
+    const float c = 1.0f / (std::sqrt((float)p->d) * p->eps);
+    const dim3 grid(d.L + (p->dustbin ? 1 : 0), d.BH);
+    cudaStream_t st = (cudaStream_t)stream;
+    const float sd2 = p->dustbin ? p->dustbin_score * kLog2e : 0.f;
+    if (p->dtype == SA_F32)
+        k_debug_plan<float><<<grid, 256, 0, st>>>((const float*)q, (const float*)k, mask, state, a,
+                                                  b, d.R, d.L, d.H, p->W, d.ld, c * kLog2e,
+                                                  p->dustbin, sd2, band, dcol, drow);
+    else
+        k_debug_plan<__nv_bfloat16><<<grid, 256, 0, st>>>(
+            (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, mask, state, a, b, d.R, d.L, d.H,
+            p->W, d.ld, c * kLog2e, p->dustbin, sd2, band, dcol, drow);
+    return cudaGetLastError() == cudaSuccess ? SA_OK : SA_ERR_CUDA;
+}
+
+sa_status sinkhorn_attn_poll(void* ws, void* stream) {
+    if (!ws) return SA_ERR_INVALID_ARG;
+    if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return SA_ERR_CUDA;
+    int h = 0;
+    if (cudaMemcpy(&h, ws, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return SA_ERR_CUDA;
+    const int zero = 0;
+    if (cudaMemcpy(ws, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess)
+        return SA_ERR_CUDA;
+    return (sa_status)h;
+}
+
+const char* sinkhorn_attn_strerror(sa_status s) {
+    switch (s) {
+        case SA_OK: return "success";
+        case SA_ERR_INVALID_ARG: return "invalid argument (null/misaligned pointer, bad size or parameter)";
+        case SA_ERR_UNSUPPORTED: return "unsupported configuration for this build";
+        case SA_ERR_WORKSPACE: return "workspace too small";
+        case SA_ERR_CUDA: return "CUDA runtime or launch error";
+        case SA_ERR_NONFINITE: return "non-finite value in duals or outputs";
+        case SA_ERR_TIMEOUT: return "bounded device wait gave up";
+    }
+    return "unknown status";
+}
+
+}  // extern "C"

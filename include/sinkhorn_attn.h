@@ -1,0 +1,166 @@
+/*
+ * sinkhorn_attn.h -- C ABI of the B200 (sm_100a) banded log-domain Sinkhorn
+ * attention library (libsinkhorn_attn.so).
+ *
+ * The operation (Block-Wise Differentiable Sinkhorn Attention; gist.science/de
+ * and gist.science/fr technical summaries, sections 2.1-2.3; abstracts on
+ * dzcademia.com and searcharxiv.com):
+ *
+ *   S_ij = <q_i, k_j> / (sqrt(d) * eps) on the band
+ *   Omega = {(i, j) : |i - j| <= W, mask_i = mask_j = 1}.
+ *   Stopped base: v = 0, then T iterations of
+ *       u_i <- -log sum_{j in Omega_i} exp(S_ij + v_j)      (rows first)
+ *       v_j <- -log sum_{i in Omega_j} exp(S_ij + u_i)      (then columns)
+ *   giving (u0, v0), held constant under differentiation.
+ *   Tail: R more iterations of the same update from v0, giving u1, v1, ..., uR, vR.
+ *   O = P^(R,R) V with P^(a,b)_ij = exp(S_ij + u^(a)_i + v^(b)_j) on Omega.
+ *   Backward: the exact vector-Jacobian product of the tail with respect to
+ *   Q, K, V for an arbitrary cotangent dO (section 2.2; R = 2 has the four
+ *   staircase plans P^(2,2), P^(2,1), P^(1,1), P^(1,0)).
+ *   Dustbin (section 2.3): the same surrogate on a support enlarged by one
+ *   dustbin row and one dustbin column (plus their corner) carrying the
+ *   constant score dustbin_score, with unit mass like every other row/column.
+ *
+ * Conventions shared by every entry point
+ *   - The caller owns every buffer.  The library allocates no device or host
+ *     memory in any call and keeps no mutable global state, so concurrent
+ *     calls on different buffers are safe.
+ *   - Device pointers must be 16-byte aligned and the tensors contiguous in
+ *     the stated layout; otherwise the call returns SA_ERR_INVALID_ARG before
+ *     launching anything.
+ *   - Work is enqueued asynchronously on `stream` (a cudaStream_t; NULL means
+ *     the legacy default stream).  Argument and launch errors are returned at
+ *     once.  Conditions found on the device (a non-finite dual or output when
+ *     check_finite is set) are recorded in a status word at the start of the
+ *     workspace and returned by sinkhorn_attn_poll().
+ *   - Masked tokens (mask_i == 0) have exactly zero duals, O, dQ, dK and dV.
+ *   - Tensors Q, K, V, O, dO, dQ, dK, dV are [B][H][L][d] row-major with d
+ *     contiguous, of element type `dtype`.  Duals are float32.
+ */
+#ifndef SINKHORN_ATTN_H
+#define SINKHORN_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    SA_OK = 0,
+    SA_ERR_INVALID_ARG = -1,  /* null/misaligned pointer, bad size or parameter */
+    SA_ERR_UNSUPPORTED = -2,  /* valid request outside what this build implements */
+    SA_ERR_WORKSPACE = -3,    /* workspace smaller than sinkhorn_attn_workspace_size() */
+    SA_ERR_CUDA = -4,         /* a CUDA runtime call or kernel launch failed */
+    SA_ERR_NONFINITE = -5,    /* device found a NaN/Inf (only with check_finite) */
+    SA_ERR_TIMEOUT = -6       /* a bounded device-side wait gave up */
+} sa_status;
+
+typedef enum { SA_F32 = 0, SA_BF16 = 1 } sa_dtype;
+
+/* Backward schedule (section 2.2).  ONE_REFERENCE forms only P^(R,R) and
+ * rescales it with exp(u^(a)-u^(R)) exp(v^(b)-v^(R)); DIRECT forms every
+ * staircase plan with its own exponential (the direct-four adjoint for R=2). */
+typedef enum { SA_BWD_ONE_REFERENCE = 0, SA_BWD_DIRECT = 1 } sa_bwd_schedule;
+
+typedef struct {
+    int B, H, L, d;        /* batch, heads, sequence length, head dim (d == 64) */
+    int W;                 /* band half-width, W >= 0 (W >= L-1 is dense) */
+    float eps;             /* entropic temperature, > 0 */
+    int T;                 /* stopped base iterations, T >= 0 */
+    int R;                 /* tail iterations, 1 <= R <= 4 (2 in the pages) */
+    sa_dtype dtype;        /* element type of Q, K, V, O, dO, dQ, dK, dV */
+    int dustbin;           /* 0 or 1: add the dustbin row and column */
+    float dustbin_score;   /* score on every dustbin entry, used as given */
+    sa_bwd_schedule bwd;   /* backward schedule */
+    int check_finite;      /* 0 or 1: scan duals/outputs, set SA_ERR_NONFINITE */
+    /* Optional launch trace for profiling (all NULL/0 to disable).  When
+     * trace_cap > 0 the call records trace_events[2i] before and
+     * trace_events[2i+1] after its i-th kernel launch on `stream` (cudaEvent_t
+     * handles created by the caller), stores that launch's sa_kernel_kind in
+     * trace_kinds[i] (host memory) for i < trace_cap, and writes the number
+     * of launches it made to *trace_count (host memory, may be NULL). */
+    void* const* trace_events;
+    int* trace_kinds;
+    int* trace_count;
+    int trace_cap;
+} sa_params;
+
+/* Kernel kinds reported by the launch trace. */
+typedef enum {
+    SA_KERNEL_LSE_SWEEP = 1,   /* dual update: u <- -LSE_j(S+v) or v <- -LSE_i(S+u) */
+    SA_KERNEL_PV = 2,          /* O = P V, or dV = P^T dO with vbar = rowdot(V, dV) */
+    SA_KERNEL_WSUM = 3,        /* vector cotangent sweep: weighted plan row sums */
+    SA_KERNEL_DS = 4,          /* dQ = c dS K or dK = c dS^T Q */
+    SA_KERNEL_AUX = 5,         /* O(L) elementwise helpers */
+    SA_KERNEL_FUSED_SWEEP = 6  /* tensor-core fused iteration (row LSE + column partials) */
+} sa_kernel_kind;
+
+/* Number of float32 elements of the dual state: B*H*(2R+2)*(L+dustbin).
+ * Layout [B][H][2R+2][L+dustbin]: row 2r is u^(r), row 2r+1 is v^(r),
+ * r = 0..R; with a dustbin, index L of each row is the dustbin's dual.
+ * Returns SA_ERR_INVALID_ARG for invalid params. */
+sa_status sinkhorn_attn_state_size(const sa_params* p, size_t* n_floats);
+
+/* Workspace bytes needed by sinkhorn_attn_fwd and sinkhorn_attn_bwd (either
+ * pointer may be NULL).  Both are O(B*H*L) and include a 256-byte status
+ * header at offset 0. */
+sa_status sinkhorn_attn_workspace_size(const sa_params* p, size_t* fwd_bytes, size_t* bwd_bytes);
+
+/*
+ * Forward (sections 2.1 and 2.3).
+ *   q, k, v : [B][H][L][d] dtype, device.
+ *   mask    : [B][L] uint8 (1 = valid, 0 = padding), device, or NULL (all valid).
+ *   v_dust  : [H][d] float32 dustbin value vectors, device, or NULL (zero);
+ *             read only when p->dustbin.
+ *   o       : [B][H][L][d] dtype, device, written (masked rows = 0).
+ *   state   : sinkhorn_attn_state_size() float32, device, written.
+ *   ws      : workspace of ws_bytes >= fwd_bytes, device.
+ * Score tiles are recomputed in every sweep; nothing of size L*W is stored.
+ */
+sa_status sinkhorn_attn_fwd(const sa_params* p, const void* q, const void* k, const void* v,
+                            const uint8_t* mask, const float* v_dust, void* o, float* state,
+                            void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Backward: dQ, dK, dV (and the dustbin value gradient) of <dO, O> through the
+ * R-step tail, the stopped base held constant (section 2.2).
+ *   q, k, v, mask, v_dust : as given to the forward.
+ *   o, state              : the forward's outputs.
+ *   dO                    : [B][H][L][d] dtype, device.
+ *   dq, dk, dv            : [B][H][L][d] dtype, device, written.
+ *   dv_dust               : [H][d] float32, device, written (summed over the
+ *                           batch), or NULL; used only when p->dustbin.
+ *   ws                    : workspace of ws_bytes >= bwd_bytes, device.
+ * The schedule is p->bwd.
+ */
+sa_status sinkhorn_attn_bwd(const sa_params* p, const void* q, const void* k, const void* v,
+                            const uint8_t* mask, const float* v_dust, const void* o,
+                            const void* dO, const float* state, void* dq, void* dk, void* dv,
+                            float* dv_dust, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Test hook: the plan P^(a,b) (0 <= a, b <= R) from a finished forward state.
+ *   band : [B][H][L][2W+1] float32, entry t of row i is column i-W+t (0 off Omega).
+ *   dcol : [B][H][L] float32 entries (i, dustbin), or NULL.
+ *   drow : [B][H][L+1] float32 entries (dustbin, j), corner last, or NULL.
+ * dcol/drow are written only when p->dustbin.
+ */
+sa_status sinkhorn_attn_debug_plan(const sa_params* p, int a, int b, const void* q,
+                                   const void* k, const uint8_t* mask, const float* state,
+                                   float* band, float* dcol, float* drow, void* stream);
+
+/* Synchronises `stream`, then returns the status word recorded in `ws` by the
+ * last forward/backward that used it (SA_OK, SA_ERR_NONFINITE or
+ * SA_ERR_TIMEOUT) and resets it to SA_OK. */
+sa_status sinkhorn_attn_poll(void* ws, void* stream);
+
+/* Static English description of a status code. */
+const char* sinkhorn_attn_strerror(sa_status s);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SINKHORN_ATTN_H */

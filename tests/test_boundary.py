@@ -1,0 +1,113 @@
+"""The C ABI without a GPU: the library loads, exports every entry point that
+include/sinkhorn_attn.h declares, and validates its arguments on the host
+before touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+import banded_log_domain_b200 as sa
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "sinkhorn_attn.h")
+
+
+def declared():
+    txt = open(HEADER).read()
+    return sorted(set(re.findall(r"\b(sinkhorn_attn_\w+)\s*\(", txt)))
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ctypes.CDLL(sa.LIB_PATH)
+    names = declared()
+    assert len(names) >= 7
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(sa.EXPORTS) <= set(names)
+
+
+def P(**kw):
+    base = dict(B=2, H=3, L=100, d=64, W=5, eps=0.5, T=4, R=2, dtype=torch.float32)
+    base.update(kw)
+    B, H, L, d = base.pop("B"), base.pop("H"), base.pop("L"), base.pop("d")
+    return sa.make_params(B, H, L, d, **base)
+
+
+def test_state_and_workspace_sizes():
+    assert sa.sinkhorn_attn_state_size(P()) == 2 * 3 * 6 * 100
+    assert sa.sinkhorn_attn_state_size(P(R=3, dustbin=True)) == 2 * 3 * 8 * 101
+    f, b = sa.sinkhorn_attn_workspace_size(P())
+    assert f >= 256 and b >= 256 + 10 * 2 * 3 * 100 * 4
+    # O(L): the backward workspace grows linearly in L and not with W
+    _, b1 = sa.sinkhorn_attn_workspace_size(P(L=10000, W=5))
+    _, b2 = sa.sinkhorn_attn_workspace_size(P(L=10000, W=500))
+    _, b3 = sa.sinkhorn_attn_workspace_size(P(L=20000, W=5))
+    assert b1 == b2 and 1.9 < b3 / b1 < 2.1
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(W=-1), -1), (dict(eps=0.0), -1), (dict(eps=float("nan")), -1), (dict(T=-1), -1),
+    (dict(R=0), -1), (dict(L=-5), -1), (dict(d=32), -2), (dict(R=5), -2),
+    (dict(dustbin=True, dustbin_score=float("inf")), -1),
+])
+def test_invalid_params_rejected(kw, status):
+    with pytest.raises(sa.SinkhornAttnError) as e:
+        sa.sinkhorn_attn_state_size(P(**kw))
+    assert e.value.status == status
+
+
+def test_bad_enum_and_flags_rejected():
+    p = P()
+    p.dtype = 7
+    assert sa._L().sinkhorn_attn_state_size(ctypes.byref(p), ctypes.byref(ctypes.c_size_t())) == -1
+    p = P()
+    p.dustbin = 2
+    assert sa._L().sinkhorn_attn_state_size(ctypes.byref(p), ctypes.byref(ctypes.c_size_t())) == -1
+    p = P()
+    p.bwd = 3
+    assert sa._L().sinkhorn_attn_state_size(ctypes.byref(p), ctypes.byref(ctypes.c_size_t())) == -1
+
+
+def test_null_and_host_pointers_rejected_before_launch():
+    lib = sa._L()
+    p = P()
+    ws = ctypes.create_string_buffer(4096)
+    buf = ctypes.create_string_buffer(2 * 3 * 100 * 64 * 4 + 64)
+    addr = (ctypes.addressof(buf) + 15) & ~15
+    # null tensors
+    rc = lib.sinkhorn_attn_fwd(ctypes.byref(p), None, None, None, None, None, None, None,
+                               ctypes.addressof(ws), 4096, None)
+    assert rc == -1
+    # plain host memory is not a device pointer
+    rc = lib.sinkhorn_attn_fwd(ctypes.byref(p), addr, addr, addr, None, None, addr, addr,
+                               ctypes.addressof(ws), 4096, None)
+    assert rc == -1
+    # misaligned
+    rc = lib.sinkhorn_attn_fwd(ctypes.byref(p), addr + 4, addr, addr, None, None, addr, addr,
+                               ctypes.addressof(ws), 4096, None)
+    assert rc == -1
+
+
+def test_workspace_too_small():
+    lib = sa._L()
+    p = P()
+    _, b = sa.sinkhorn_attn_workspace_size(p)
+    rc = lib.sinkhorn_attn_bwd(ctypes.byref(p), *([None] * 13), b - 1, None)
+    assert rc == -3
+    rc = lib.sinkhorn_attn_fwd(ctypes.byref(p), *([None] * 8), 16, None)
+    assert rc == -3
+
+
+def test_empty_problem_is_a_noop():
+    lib = sa._L()
+    p = P(L=0)
+    rc = lib.sinkhorn_attn_fwd(ctypes.byref(p), *([None] * 8), 256, None)
+    assert rc == 0
+
+
+def test_strerror_covers_every_status():
+    for s in range(0, -7, -1):
+        assert sa.strerror(s) and "unknown" not in sa.strerror(s)
+    assert "unknown" in sa.strerror(42)
