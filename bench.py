@@ -166,18 +166,28 @@ def barrier(ws):
 # CPU oracle timing (cpu_baseline leg and --impl reference)
 # ---------------------------------------------------------------------------
 
-def oracle_sample_rate(w, L_s, schedule):
-    """tokens*heads/s of the oracle's forward + backward on one head of the
-    workload truncated to its first L_s tokens."""
+def oracle_sample_rate(w, L_s, schedule, heads=1):
+    """tokens*heads/s of the oracle's forward + backward on ``heads`` heads of
+    the workload truncated to their first L_s tokens."""
     import oracle
 
-    x = workloads.draw(1, 1, L_s, w.d, dtype=w.dtype, seed=0)
+    x = workloads.draw(1, heads, L_s, w.d, dtype=w.dtype, seed=0)
     t0 = time.perf_counter()
     o, st = oracle.forward(x["q"], x["k"], x["v"], W=w.W, eps=w.eps, T=w.T, R=w.R)
     oracle.backward(x["q"], x["k"], x["v"], st, x["dO"], W=w.W, eps=w.eps, R=w.R,
                     schedule=schedule)
     dt = time.perf_counter() - t0
-    return L_s / dt, dt
+    return heads * L_s / dt, dt
+
+
+def size_sample(w, schedule, target_s):
+    """(heads, tokens) of a sample of about target_s seconds of oracle work."""
+    L1 = min(w.L, max(2 * w.W + 2, 2048))
+    _, dt1 = oracle_sample_rate(w, L1, schedule)
+    per_tok = max(dt1, 1e-4) / L1
+    L_s = int(min(w.L, max(L1, target_s / per_tok)))
+    heads = int(min(w.B * w.H, max(1, round(target_s / (per_tok * L_s)))))
+    return heads, L_s
 
 
 def oracle_cores():
@@ -190,14 +200,12 @@ def oracle_cores():
         return os.cpu_count() or 1
 
 
-def cpu_baseline(w, schedule, target_s=15.0):
-    L1 = min(w.L, max(2 * w.W + 2, 2048))
-    _, dt1 = oracle_sample_rate(w, L1, schedule)
-    L_s = int(min(w.L, max(L1, L1 * target_s / max(dt1, 1e-3))))
-    rate, dt = oracle_sample_rate(w, L_s, schedule)
+def cpu_baseline(w, schedule, target_s=12.0):
+    heads, L_s = size_sample(w, schedule, target_s)
+    rate, dt = oracle_sample_rate(w, L_s, schedule, heads)
     return {"value": rate, "unit": UNIT, "cores": oracle_cores(), "kind": "oracle",
-            "sample": f"1 head x first {L_s} tokens of {w.name} (W={w.W}, T={w.T}, R={w.R}, "
-                      f"d={w.d}), forward + {schedule} backward, float64, {dt:.1f} s"}
+            "sample": f"{heads} head(s) x first {L_s} tokens of {w.name} (W={w.W}, T={w.T}, "
+                      f"R={w.R}, d={w.d}), forward + {schedule} backward, float64, {dt:.1f} s"}
 
 
 def run_reference(args, w):
@@ -205,19 +213,17 @@ def run_reference(args, w):
     if rank != 0:
         return
     # size each step's sample to a few seconds
-    L1 = min(w.L, max(2 * w.W + 2, 1024))
-    _, dt1 = oracle_sample_rate(w, L1, args.schedule)
-    L_s = int(min(w.L, max(L1, L1 * 3.0 / max(dt1, 1e-3))))
+    heads, L_s = size_sample(w, args.schedule, 3.0)
     for _ in range(args.warmup):
-        oracle_sample_rate(w, L_s, args.schedule)
+        oracle_sample_rate(w, L_s, args.schedule, heads)
     times = []
     for _ in range(args.steps):
-        _, dt = oracle_sample_rate(w, L_s, args.schedule)
+        _, dt = oracle_sample_rate(w, L_s, args.schedule, heads)
         times.append(dt)
     total = sum(times)
-    value = args.steps * L_s / total
-    sample = (f"1 head x first {L_s} tokens of {w.name} per step, forward + {args.schedule} "
-              f"backward, float64")
+    value = args.steps * heads * L_s / total
+    sample = (f"{heads} head(s) x first {L_s} tokens of {w.name} per step, forward + "
+              f"{args.schedule} backward, float64")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
