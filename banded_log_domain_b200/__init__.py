@@ -95,6 +95,9 @@ def _L():
     lib.sinkhorn_attn_fwd.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
     lib.sinkhorn_attn_bwd.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz,
                                       vp]
+    lib.sinkhorn_attn_bwd_static_ws.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp,
+                                                vp, vp]
+    lib.sinkhorn_attn_bwd_static_ws.restype = ctypes.c_int
     lib.sinkhorn_attn_debug_plan.argtypes = [P, ctypes.c_int, ctypes.c_int, vp, vp, vp, vp, vp,
                                              vp, vp, vp]
     lib.sinkhorn_attn_poll.argtypes = [vp, vp]
@@ -113,8 +116,8 @@ def load():
 
 
 EXPORTS = ("sinkhorn_attn_state_size", "sinkhorn_attn_workspace_size", "sinkhorn_attn_fwd",
-           "sinkhorn_attn_bwd", "sinkhorn_attn_debug_plan", "sinkhorn_attn_poll",
-           "sinkhorn_attn_strerror")
+           "sinkhorn_attn_bwd", "sinkhorn_attn_bwd_static_ws", "sinkhorn_attn_debug_plan",
+           "sinkhorn_attn_poll", "sinkhorn_attn_strerror")
 
 
 def strerror(status: int) -> str:
@@ -214,6 +217,37 @@ def sinkhorn_attn_bwd(q, k, v, o, dO, state, *, W, eps, R=2, mask=None, dustbin=
                                 _ptr(dv), _ptr(dv_dust if dustbin else None), _ptr(ws),
                                 ws.numel(), _stream(dev))
     _check(rc, "sinkhorn_attn_bwd")
+    return dq, dk, dv, (dv_dust if dustbin else None)
+
+
+STATIC_SCRATCH_BYTES = 32 << 20
+
+
+def sinkhorn_attn_bwd_static_ws(q, k, v, o, dO, state, *, W, eps, R=2, mask=None,
+                                dustbin=False, dustbin_score=-2.0, v_dust=None,
+                                schedule="one_reference", dq=None, dk=None, dv=None,
+                                dv_dust=None, trace=None):
+    """Backward that takes no workspace: for callers that cannot allocate
+    device memory where they run it (see ``sinkhorn_attn_bwd_static_ws`` in
+    the C header).  The library's fixed scratch array (``STATIC_SCRATCH_BYTES``
+    per GPU) is used instead; calls that overlap on the GPU race.  Pass
+    preallocated ``dq, dk, dv`` (and ``dv_dust``) to keep the call free of
+    allocations on the Python side too."""
+    _contig(q, k, v, o, dO, state, mask, v_dust, dq, dk, dv, dv_dust)
+    p = _params_for(q, W, eps, 0, R, dustbin, dustbin_score, schedule, False)
+    if trace is not None:
+        trace.attach(p)
+    dev = q.device
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(q) if dk is None else dk
+    dv = torch.empty_like(q) if dv is None else dv
+    if dustbin and dv_dust is None:
+        dv_dust = torch.empty(q.shape[1], q.shape[3], dtype=torch.float32, device=dev)
+    rc = _L().sinkhorn_attn_bwd_static_ws(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(mask),
+                                          _ptr(v_dust), _ptr(o), _ptr(dO), _ptr(state), _ptr(dq),
+                                          _ptr(dk), _ptr(dv), _ptr(dv_dust if dustbin else None),
+                                          _stream(dev))
+    _check(rc, "sinkhorn_attn_bwd_static_ws")
     return dq, dk, dv, (dv_dust if dustbin else None)
 
 

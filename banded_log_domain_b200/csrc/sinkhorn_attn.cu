@@ -21,6 +21,7 @@
 // P^(r,r) formed by its own exponential.
 #include <cmath>
 #include <cstring>
+#include <mutex>
 
 #include "../../include/sinkhorn_attn.h"
 #include "simt_sweep.cuh"
@@ -636,6 +637,85 @@ sa_status sinkhorn_attn_bwd(const sa_params* p, const void* q, const void* k, co
         }
     }
     return SA_OK;
+}
+
+}  // extern "C"
+
+// Fixed scratch for sinkhorn_attn_bwd_static_ws: one array per device that
+// loads the library, alive until the process exits.  Host code must not use
+// this name as a pointer (it is a host-side stand-in); the device address is
+// looked up once per device below.
+static __device__ __align__(256) unsigned char g_bwd_scratch[SA_STATIC_SCRATCH_BYTES];
+
+namespace {
+constexpr int kMaxDevices = 64;
+void* g_bwd_scratch_addr[kMaxDevices];   // device address of g_bwd_scratch, per device
+std::mutex g_bwd_scratch_mu;
+
+// Address of the scratch array on the current device (looked up on first use).
+sa_status bwd_scratch_current_device(void** out) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) return SA_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return SA_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_bwd_scratch_mu);
+    if (!g_bwd_scratch_addr[dev]) {
+        void* ptr = nullptr;
+        if (cudaGetSymbolAddress(&ptr, g_bwd_scratch) != cudaSuccess || !ptr) {
+            cudaGetLastError();
+            return SA_ERR_CUDA;
+        }
+        g_bwd_scratch_addr[dev] = ptr;
+    }
+    *out = g_bwd_scratch_addr[dev];
+    return SA_OK;
+}
+}  // namespace
+
+extern "C" {
+
+sa_status sinkhorn_attn_bwd_static_ws(const sa_params* p, const void* q, const void* k,
+                                      const void* v, const uint8_t* mask, const float* v_dust,
+                                      const void* o, const void* dO, const float* state,
+                                      void* dq, void* dk, void* dv, float* dv_dust,
+                                      void* stream) {
+    Dims d;
+    sa_status s = check_params(p, &d);
+    if (s != SA_OK) return s;
+    if (p->check_finite) return SA_ERR_UNSUPPORTED;
+    const size_t need = bwd_layout(d).total;
+    if (need > (size_t)SA_STATIC_SCRATCH_BYTES) return SA_ERR_WORKSPACE;
+    if (d.BH == 0 || d.L == 0) return SA_OK;
+    if (!device_ok(q) || !device_ok(k) || !device_ok(v) || !device_ok(o) || !device_ok(dO) ||
+        !device_ok(state) || !device_ok(dq) || !device_ok(dk) || !device_ok(dv) ||
+        !mask_ok(mask))
+        return SA_ERR_INVALID_ARG;
+    if (p->dustbin && v_dust && !device_ok(v_dust)) return SA_ERR_INVALID_ARG;
+    if (p->dustbin && dv_dust && !device_ok(dv_dust)) return SA_ERR_INVALID_ARG;
+    void* ws = nullptr;
+    s = bwd_scratch_current_device(&ws);
+    if (s != SA_OK) return s;
+    cudaStream_t st = (cudaStream_t)stream;
+    // the status header is the only part of the workspace read before it is written
+    if (cudaMemsetAsync(ws, 0, kHeader, st) != cudaSuccess) return SA_ERR_CUDA;
+    Ctx x;
+    x.p = p;
+    x.d = d;
+    x.st = st;
+    x.c = 1.0f / (std::sqrt((float)p->d) * p->eps);
+    x.sst = (long long)(2 * d.R + 2) * d.ld;
+    x.state = state;
+    x.tr.p = p;
+    x.tr.st = st;
+    const float* vd = p->dustbin ? v_dust : nullptr;
+    float* dvd = p->dustbin ? dv_dust : nullptr;
+    if (p->dtype == SA_F32)
+        return bwd_impl<float>(x, (const float*)q, (const float*)k, (const float*)v, mask, vd,
+                               (const float*)o, (const float*)dO, (float*)dq, (float*)dk,
+                               (float*)dv, dvd, (char*)ws);
+    return bwd_impl<__nv_bfloat16>(
+        x, (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v, mask, vd,
+        (const __nv_bfloat16*)o, (const __nv_bfloat16*)dO, (__nv_bfloat16*)dq,
+        (__nv_bfloat16*)dk, (__nv_bfloat16*)dv, dvd, (char*)ws);
 }
 
 sa_status sinkhorn_attn_debug_plan(const sa_params* p, int a, int b, const void* q,

@@ -24,7 +24,8 @@
  * Conventions shared by every entry point
  *   - The caller owns every buffer.  The library allocates no device or host
  *     memory in any call and keeps no mutable global state, so concurrent
- *     calls on different buffers are safe.
+ *     calls on different buffers are safe (sinkhorn_attn_bwd_static_ws is the
+ *     one exception: it uses a fixed scratch array inside the library).
  *   - Device pointers must be 16-byte aligned and the tensors contiguous in
  *     the stated layout; otherwise the call returns SA_ERR_INVALID_ARG before
  *     launching anything.
@@ -150,6 +151,37 @@ sa_status sinkhorn_attn_bwd(const sa_params* p, const void* q, const void* k, co
 sa_status sinkhorn_attn_debug_plan(const sa_params* p, int a, int b, const void* q,
                                    const void* k, const uint8_t* mask, const float* state,
                                    float* band, float* dcol, float* drow, void* stream);
+
+/*
+ * Backward without caller-provided workspace.  No counterpart in the paper:
+ * this exists for callers that cannot allocate device memory at the point
+ * where they run the backward -- for example a host framework that owns all
+ * device memory and forbids allocations inside its step, or latency-critical
+ * code that cannot afford cudaMalloc's implicit device-wide synchronisation --
+ * and that have no spare buffer to lend as workspace.
+ *
+ * Same arguments, layouts and results as sinkhorn_attn_bwd, minus ws and
+ * ws_bytes.  The scratch comes from one fixed array of
+ * SA_STATIC_SCRATCH_BYTES bytes compiled into the library; every GPU that
+ * loads the library holds it until the process exits.  Problems whose
+ * backward workspace (sinkhorn_attn_workspace_size) exceeds that size are
+ * rejected with SA_ERR_WORKSPACE before anything is launched.
+ *   - The call allocates nothing: no cudaMalloc/cudaFree or allocating
+ *     library routine.
+ *   - The first call on a device looks up the array's device address (with
+ *     that device current); make that first call before any stream capture.
+ *   - All calls share the one array and it keeps the last call's contents, so
+ *     calls whose work overlaps on the GPU (different streams, or different
+ *     host threads on one device) race: serialise them.
+ *   - check_finite is not supported here (there is no workspace to poll):
+ *     SA_ERR_UNSUPPORTED.
+ */
+#define SA_STATIC_SCRATCH_BYTES (32u << 20)
+sa_status sinkhorn_attn_bwd_static_ws(const sa_params* p, const void* q, const void* k,
+                                      const void* v, const uint8_t* mask, const float* v_dust,
+                                      const void* o, const void* dO, const float* state,
+                                      void* dq, void* dk, void* dv, float* dv_dust,
+                                      void* stream);
 
 /* Synchronises `stream`, then returns the status word recorded in `ws` by the
  * last forward/backward that used it (SA_OK, SA_ERR_NONFINITE or
