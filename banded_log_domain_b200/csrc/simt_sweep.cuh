@@ -68,6 +68,7 @@ struct SweepArgs {
     Vec er[MAXT], ec[MAXT], cr[MAXT], cc[MAXT];  // DSD (cr/cc p null = 0)
     float gk[MAXT];                          // DSD: weight of G in term k
     float* dvd_part;        // PV dustbin row: [BH][D] sum_c P_(dust,c) X_c (or null)
+    int online;             // LSE on tensor cores: 1 = no previous dual, use a running max
 };
 
 // ---------------------------------------------------------------------------

@@ -23,8 +23,13 @@
 #include <cstring>
 #include <mutex>
 
+#include <cudaTypedefs.h>
+
+#include <type_traits>
+
 #include "../../include/sinkhorn_attn.h"
 #include "simt_sweep.cuh"
+#include "tc_sweep.cuh"
 
 namespace sa {
 namespace {
@@ -248,8 +253,65 @@ constexpr int kind_of(int mode) {
          : mode == simt::WSUM ? SA_KERNEL_WSUM : SA_KERNEL_DS;
 }
 
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no libcuda link).
+PFN_cuTensorMapEncodeTiled_v12000 encode_tiled() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) !=
+                cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            p = nullptr;
+        return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }();
+    return fn;
+}
+
+// [BH][L][64] bf16 viewed as a 3-D tensor; 64 x 128 x 1 boxes, 128-byte swizzle,
+// zero fill outside the tensor (rows < 0 or >= L).
+bool make_map(CUtensorMap* m, const void* ptr, int L, int BH) {
+    auto fn = encode_tiled();
+    if (!fn || !ptr) return false;
+    cuuint64_t dims[3] = {64, (cuuint64_t)L, (cuuint64_t)BH};
+    cuuint64_t strides[2] = {64 * 2, (cuuint64_t)L * 64 * 2};
+    cuuint32_t box[3] = {64, 128, 1};
+    cuuint32_t es[3] = {1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box,
+              es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+           CUDA_SUCCESS;
+}
+
+template <int MODE, bool ONLINE>
+cudaError_t launch_tc(const simt::SweepArgs& a, int BH, cudaStream_t st, Tracer& tr,
+                      int* status) {
+    tcs::Maps maps;
+    std::memset(&maps, 0, sizeof(maps));
+    bool ok = make_map(&maps.A, a.A, a.L, BH) && make_map(&maps.B, a.Bo, a.L, BH);
+    if (tcs::is_ds(MODE)) ok = ok && make_map(&maps.A2, a.A2, a.L, BH) && make_map(&maps.B2, a.B2, a.L, BH);
+    if (MODE == simt::PV) ok = ok && make_map(&maps.X, a.X, a.L, BH);
+    if (!ok) return cudaErrorInvalidValue;
+    const dim3 grid((a.L + 127) / 128, BH);
+    const int smem = tcs::smem_bytes(MODE);
+    cudaError_t e = cudaFuncSetAttribute(tcs::tc_band_sweep<MODE, ONLINE>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    tr.begin(kind_of(MODE));
+    tcs::tc_band_sweep<MODE, ONLINE><<<grid, tcs::NTHREADS, smem, st>>>(a, maps, status);
+    tr.end();
+    return cudaGetLastError();
+}
+
 template <typename T, int MODE>
-cudaError_t launch_sweep(const simt::SweepArgs& a, int BH, cudaStream_t st, Tracer& tr) {
+cudaError_t launch_sweep(const simt::SweepArgs& a, int BH, cudaStream_t st, Tracer& tr,
+                         int* status) {
+    // bf16 storage without a dustbin runs on the tensor cores
+    if constexpr (std::is_same<T, __nv_bfloat16>::value) {
+        if (!a.dustbin) {
+            if (MODE == simt::LSE && a.online) return launch_tc<MODE, true>(a, BH, st, tr, status);
+            return launch_tc<MODE, false>(a, BH, st, tr, status);
+        }
+    }
     const int nblk = (a.L + simt::BM - 1) / simt::BM;
     const dim3 grid(nblk + (a.dust_cta ? 1 : 0), BH);
     const size_t smem = (size_t)simt::smem_floats(MODE) * sizeof(float);
@@ -280,6 +342,7 @@ struct Ctx {
     float c;     // natural score scale 1/(sqrt(d) eps)
     long long sst;  // per-bh stride of a state row: (2R+2)*ld
     const float* state;
+    int* status;   // device status word (workspace header)
     mutable Tracer tr;
     // state row r (0..2R+1) as a Vec
     Vec srow(int r) const { return vec(state + (size_t)r * d.ld, sst); }
@@ -319,16 +382,21 @@ sa_status fwd_impl(const Ctx& x, const T* q, const T* k, const T* v, const uint8
     for (int it = 0; it < iters; ++it) {
         const int rin = it < x.p->T ? 0 : it - x.p->T;       // v index read
         const int rout = it < x.p->T ? 0 : it - x.p->T + 1;  // u, v index written
-        // rows: u^(rout) = -LSE_j(S + v^(rin))
+        // rows: u^(rout) = -LSE_j(S + v^(rin)); the previous u (u^(rin), or u0 in
+        // place during the base) is the exponent shift, except on the first update
         a.A = q; a.Bo = k;
         a.cd = x.srow(2 * rin + 1);
+        a.rd = x.srow(2 * rin);
+        a.online = (it == 0);
         a.out_vec = mvec(state + (size_t)(2 * rout) * d.ld, x.sst);
-        SA_CUDA((launch_sweep<T, simt::LSE>(a, d.BH, x.st, x.tr)));
-        // columns: v^(rout) = -LSE_i(S + u^(rout))
+        SA_CUDA((launch_sweep<T, simt::LSE>(a, d.BH, x.st, x.tr, x.status)));
+        // columns: v^(rout) = -LSE_i(S + u^(rout)), shifted by the previous v
         a.A = k; a.Bo = q;
         a.cd = x.srow(2 * rout);
+        a.rd = x.srow(2 * rin + 1);
+        a.online = 0;
         a.out_vec = mvec(state + (size_t)(2 * rout + 1) * d.ld, x.sst);
-        SA_CUDA((launch_sweep<T, simt::LSE>(a, d.BH, x.st, x.tr)));
+        SA_CUDA((launch_sweep<T, simt::LSE>(a, d.BH, x.st, x.tr, x.status)));
     }
     // O = P^(R,R) V (+ dustbin column times v_dust)
     simt::SweepArgs b = base_args(x);
@@ -339,7 +407,7 @@ sa_status fwd_impl(const Ctx& x, const T* q, const T* k, const T* v, const uint8
     b.rd = x.srow(2 * d.R);
     b.cd = x.srow(2 * d.R + 1);
     b.out_mat = o;
-    SA_CUDA((launch_sweep<T, simt::PV>(b, d.BH, x.st, x.tr)));
+    SA_CUDA((launch_sweep<T, simt::PV>(b, d.BH, x.st, x.tr, x.status)));
     return SA_OK;
 }
 
@@ -386,7 +454,7 @@ sa_status bwd_impl(const Ctx& x, const T* q, const T* k, const T* v, const uint8
         a.out_mat = dv;
         a.out_vec = mvec(vb(R), vs);
         a.dvd_part = dvd;
-        SA_CUDA((launch_sweep<T, simt::PV>(a, d.BH, x.st, x.tr)));
+        SA_CUDA((launch_sweep<T, simt::PV>(a, d.BH, x.st, x.tr, x.status)));
     }
     // ubar^R = a - P vbar^R  (query sweep)
     {
@@ -398,7 +466,7 @@ sa_status bwd_impl(const Ctx& x, const T* q, const T* k, const T* v, const uint8
         a.base = vec(A_, vs);
         a.sgn = -1.f;
         a.out_vec = mvec(ub(R), vs);
-        SA_CUDA((launch_sweep<T, simt::WSUM>(a, d.BH, x.st, x.tr)));
+        SA_CUDA((launch_sweep<T, simt::WSUM>(a, d.BH, x.st, x.tr, x.status)));
     }
     for (int r = R; r >= 2; --r) {
         // vbar^(r-1) = -P^(r,r-1)^T ubar^r
@@ -416,7 +484,7 @@ sa_status bwd_impl(const Ctx& x, const T* q, const T* k, const T* v, const uint8
             a.w = vec(W_(l.w, 0), vs);
             a.mult = vec(ev(r - 1), vs);
         }
-        SA_CUDA((launch_sweep<T, simt::WSUM>(a, d.BH, x.st, x.tr)));
+        SA_CUDA((launch_sweep<T, simt::WSUM>(a, d.BH, x.st, x.tr, x.status)));
         // ubar^(r-1) = -P^(r-1,r-1) vbar^(r-1)
         simt::SweepArgs b = base_args(x);
         b.mask = mask;
@@ -432,7 +500,7 @@ sa_status bwd_impl(const Ctx& x, const T* q, const T* k, const T* v, const uint8
             b.w = vec(W_(l.w, 0), vs);
             b.mult = vec(eu(r - 1), vs);
         }
-        SA_CUDA((launch_sweep<T, simt::WSUM>(b, d.BH, x.st, x.tr)));
+        SA_CUDA((launch_sweep<T, simt::WSUM>(b, d.BH, x.st, x.tr, x.status)));
     }
 
     // modifier / staircase terms, query side (rq) and key side (rk)
@@ -502,8 +570,8 @@ sa_status bwd_impl(const Ctx& x, const T* q, const T* k, const T* v, const uint8
                 a.gk[t] = gk[t];
             }
         }
-        if (direct) SA_CUDA((launch_sweep<T, simt::DSD>(a, d.BH, x.st, x.tr)));
-        else SA_CUDA((launch_sweep<T, simt::DS1>(a, d.BH, x.st, x.tr)));
+        if (direct) SA_CUDA((launch_sweep<T, simt::DSD>(a, d.BH, x.st, x.tr, x.status)));
+        else SA_CUDA((launch_sweep<T, simt::DS1>(a, d.BH, x.st, x.tr, x.status)));
     }
     if (x.p->dustbin && dv_dust) {
         SA_AUX(x.tr, k_dvd_reduce<<<(d.H * kD + 255) / 256, 256, 0, x.st>>>(dvd, d.B, d.H,
@@ -565,6 +633,7 @@ sa_status sinkhorn_attn_fwd(const sa_params* p, const void* q, const void* k, co
     x.c = 1.0f / (std::sqrt((float)p->d) * p->eps);
     x.sst = (long long)(2 * d.R + 2) * d.ld;
     x.state = state;
+    x.status = (int*)ws;
     x.tr.p = p;
     x.tr.st = x.st;
     const float* vd = p->dustbin ? v_dust : nullptr;
@@ -611,6 +680,7 @@ sa_status sinkhorn_attn_bwd(const sa_params* p, const void* q, const void* k, co
     x.c = 1.0f / (std::sqrt((float)p->d) * p->eps);
     x.sst = (long long)(2 * d.R + 2) * d.ld;
     x.state = state;
+    x.status = (int*)ws;
     x.tr.p = p;
     x.tr.st = x.st;
     const float* vd = p->dustbin ? v_dust : nullptr;
@@ -704,6 +774,7 @@ sa_status sinkhorn_attn_bwd_static_ws(const sa_params* p, const void* q, const v
     x.c = 1.0f / (std::sqrt((float)p->d) * p->eps);
     x.sst = (long long)(2 * d.R + 2) * d.ld;
     x.state = state;
+    x.status = (int*)ws;
     x.tr.p = p;
     x.tr.st = st;
     const float* vd = p->dustbin ? v_dust : nullptr;

@@ -1,0 +1,540 @@
+// Tensor-core band sweeps for bf16 storage (sm_100a: TMA + tcgen05 + TMEM).
+//
+// Same sweeps and epilogues as the SIMT kernels (see simt_sweep.cuh), with
+// the band contractions on the 5th-generation tensor cores:
+//   S  = A_blk B_chunk^T   128 x 128 x 64, bf16 in, fp32 accumulation in TMEM
+//   G  = A2_blk B2_chunk^T (dS sweeps only)
+//   O += P X_chunk         128 x 64 x 128, P (or dS) rounded to bf16 and staged
+//                          in shared memory in the 128-byte-swizzled K-major
+//                          layout, X read MN-major straight from its TMA tile.
+// One CTA owns a block of 128 rows (TMEM lanes) of one (batch, head) problem
+// and walks the band's column chunks [r0 - W, r0 + 127 + W] in steps of 128.
+//
+// Warp roles (320 threads):
+//   warps 0-7  epilogue: warp w reads TMEM lanes 32*(w%4)..+31 (its rows) and
+//              columns 64*(w/4)..+63 of each chunk;
+//   warp 8     loader: TMA tiles (lane 0) and the chunk's column vectors
+//              (all lanes) into a ring of NST stages;
+//   warp 9     MMA issuer (lane 0).
+// Pipelines are mbarriers; every wait is bounded and a timeout records
+// SA_ERR_TIMEOUT in the status word and unwinds.
+//
+// Dual updates use the previous value of the updated dual as the exponent
+// shift (u_new = u_old - log sum_j exp(S + u_old + v)): every term is then a
+// plan entry of a plan with unit columns (or rows) and is at most 1.  The
+// first row update of a solve (no previous u) uses an online max instead.
+#pragma once
+
+#include "common.cuh"
+#include "simt_sweep.cuh"
+#include "tc_ptx.cuh"
+
+namespace sa {
+namespace tcs {
+
+using simt::SweepArgs;
+using simt::MAXT;
+constexpr int LSE = simt::LSE, WSUM = simt::WSUM, PV = simt::PV, DS1 = simt::DS1,
+              DSD = simt::DSD;
+constexpr int NTHREADS = 320;
+constexpr int TILE = 16384;  // one 128 x 64 bf16 tile
+constexpr long long kWaitBudget = 4000000000LL;  // clock cycles (about 2 s)
+
+struct Maps {
+    CUtensorMap A, B, A2, B2, X;
+};
+
+__host__ __device__ constexpr bool is_ds(int m) { return m == DS1 || m == DSD; }
+__host__ __device__ constexpr bool has_x(int m) { return m == PV || is_ds(m); }
+__host__ __device__ constexpr int nst(int m) { return is_ds(m) ? 2 : (m == PV ? 3 : 4); }
+__host__ __device__ constexpr int nsb(int m) { return is_ds(m) ? 1 : 2; }
+__host__ __device__ constexpr int ncv(int m) {
+    return m == WSUM ? 2 : (m == DS1 ? 1 + MAXT : (m == DSD ? 2 * MAXT : 1));
+}
+__host__ __device__ constexpr int stage_bytes(int m) {
+    return TILE * (1 + (is_ds(m) ? 1 : 0) + (m == PV ? 1 : 0));
+}
+__host__ __device__ constexpr int tmem_cols(int m) { return has_x(m) ? 512 : 256; }
+
+// shared-memory carve-up (offsets from a 1024-aligned base)
+__host__ __device__ constexpr int off_a2(int m) { return TILE; }
+__host__ __device__ constexpr int off_stage(int m) { return TILE * (is_ds(m) ? 2 : 1); }
+__host__ __device__ constexpr int off_p(int m) { return off_stage(m) + nst(m) * stage_bytes(m); }
+__host__ __device__ constexpr int off_cv(int m) { return off_p(m) + (has_x(m) ? 2 * 2 * TILE : 0); }
+__host__ __device__ constexpr int off_red(int m) { return off_cv(m) + nst(m) * ncv(m) * 128 * 4; }
+__host__ __device__ constexpr int off_bar(int m) { return off_red(m) + 4 * 128 * 4; }
+__host__ __device__ constexpr int smem_bytes(int m) { return off_bar(m) + 64 * 8 + 64 + 1024; }
+
+// barrier slots
+enum { B_A = 0, B_FULL = 1, B_EMPTY = 5, B_SFULL = 9, B_SEMPTY = 11, B_PFULL = 13, B_PEMPTY = 15,
+       B_OFULL = 17, B_DRAIN = 18, NBAR = 19 };
+
+struct Ctl {
+    uint64_t* bar;
+    volatile int* abort;
+    int* status;
+    __device__ bool wait(int slot, uint32_t parity) {
+        if (*abort) return false;
+        if (tc::mbar_wait(bar + slot, parity, kWaitBudget)) return true;
+        *abort = 1;
+        if (status) atomicCAS(status, 0, (int)SA_ERR_TIMEOUT);
+        return false;
+    }
+};
+
+// the chunk's column vector k (128 floats) in stage s
+__device__ __forceinline__ float* colvec(uint8_t* sm, int mode, int s, int k) {
+    return reinterpret_cast<float*>(sm + off_cv(mode)) + (s * ncv(mode) + k) * 128;
+}
+
+// Exponent arguments (log2 units) of one thread's 32 columns:
+// x_j = c2 * s_j + (ce_j + rd2), -inf off the band when `partial`.
+__device__ __forceinline__ void group_args(const float (&sv)[32], const float* ce, float rd2,
+                                           float c2, bool partial, int r, int cg, int W,
+                                           float (&x)[32]) {
+    const uint64_t c2p = tc::pk2(c2, c2), rdp = tc::pk2(rd2, rd2);
+    const float4* c4 = reinterpret_cast<const float4*>(ce);
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+        const float4 cv = c4[q];
+        const uint64_t b0 = tc::add2(tc::pk2(cv.x, cv.y), rdp);
+        const uint64_t b1 = tc::add2(tc::pk2(cv.z, cv.w), rdp);
+        tc::upk2(tc::fma2(tc::pk2(sv[4 * q], sv[4 * q + 1]), c2p, b0), x[4 * q], x[4 * q + 1]);
+        tc::upk2(tc::fma2(tc::pk2(sv[4 * q + 2], sv[4 * q + 3]), c2p, b1), x[4 * q + 2],
+                 x[4 * q + 3]);
+    }
+    if (partial) {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+            const int d = r - (cg + j);
+            if ((unsigned)(d + W) > (unsigned)(2 * W)) x[j] = -INFINITY;
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+template <int MODE, bool ONLINE>
+__global__ void __launch_bounds__(NTHREADS, (MODE == LSE || MODE == WSUM) ? 2 : 1) tc_band_sweep(const SweepArgs a,
+                                                         const __grid_constant__ Maps maps,
+                                                         int* status) {
+    extern __shared__ uint8_t smraw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>(((uintptr_t)smraw + 1023) & ~(uintptr_t)1023);
+    constexpr int NST = nst(MODE), NSB = nsb(MODE), NCV = ncv(MODE);
+    constexpr bool DS = is_ds(MODE), HASX = has_x(MODE);
+    uint64_t* bar = reinterpret_cast<uint64_t*>(sm + off_bar(MODE));
+    uint32_t* tbase = reinterpret_cast<uint32_t*>(sm + off_bar(MODE) + 64 * 8);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tbase + 1);
+    float* red = reinterpret_cast<float*>(sm + off_red(MODE));
+    Ctl ctl{bar, abort_flag, status};
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int bh = blockIdx.y;
+    const int L = a.L, W = a.W;
+    const int r0 = blockIdx.x * 128;
+    const int cbeg = max(0, r0 - W);
+    const int cend = min(L, r0 + 127 + W + 1);
+    const int nch = (cend - cbeg + 127) / 128;
+    const uint8_t* mk = a.mask ? a.mask + (size_t)(bh / a.H) * L : nullptr;
+
+    if (threadIdx.x == 0) {
+        tc::mbar_init(bar + B_A, 1);
+        for (int s = 0; s < NST; ++s) {
+            tc::mbar_init(bar + B_FULL + s, 33);
+            tc::mbar_init(bar + B_EMPTY + s, 9);
+        }
+        for (int b = 0; b < 2; ++b) {
+            tc::mbar_init(bar + B_SFULL + b, 1);
+            tc::mbar_init(bar + B_SEMPTY + b, 8);
+            tc::mbar_init(bar + B_PFULL + b, 8);
+            tc::mbar_init(bar + B_PEMPTY + b, 1);
+        }
+        tc::mbar_init(bar + B_OFULL, 1);
+        tc::mbar_init(bar + B_DRAIN, 1);
+        *abort_flag = 0;
+        tc::fence_mbar_init();
+    }
+    if (warp == 0) {
+        tc::tmem_alloc(tbase, tmem_cols(MODE));
+        tc::tmem_relinquish();
+    }
+    tc::tc_fence_before();
+    __syncthreads();
+    tc::tc_fence_after();
+    const uint32_t tm = *tbase;
+    // TMEM columns: S buffer b at 128*b (DS: S at 0, G at 128); O at 256
+    const uint32_t tS = tm, tG = tm + 128, tO = tm + 256;
+
+    if (warp == 8) {
+        // ------------------------------------------------------------ loader
+        if (lane == 0) {
+            tc::prefetch_tmap(&maps.A);
+            tc::prefetch_tmap(&maps.B);
+            tc::mbar_expect_tx(bar + B_A, TILE * (DS ? 2 : 1));
+            tc::tma_load_3d(sm, &maps.A, bar + B_A, 0, r0, bh);
+            if (DS) tc::tma_load_3d(sm + off_a2(MODE), &maps.A2, bar + B_A, 0, r0, bh);
+        }
+        int issued = 0;
+        for (int c = 0; c < nch; ++c) {
+            const int s = c % NST;
+            if (c >= NST && !ctl.wait(B_EMPTY + s, ((c / NST) - 1) & 1)) break;
+            issued = c + 1;
+            const int c0 = cbeg + 128 * c;
+            uint8_t* st = sm + off_stage(MODE) + s * stage_bytes(MODE);
+            if (lane == 0) {
+                tc::mbar_expect_tx(bar + B_FULL + s, stage_bytes(MODE));
+                tc::tma_load_3d(st, &maps.B, bar + B_FULL + s, 0, c0, bh);
+                if (DS) tc::tma_load_3d(st + TILE, &maps.B2, bar + B_FULL + s, 0, c0, bh);
+                if (MODE == PV) tc::tma_load_3d(st + TILE, &maps.X, bar + B_FULL + s, 0, c0, bh);
+            }
+            // column vectors: -inf / 0 outside [cbeg, cend) and on masked columns
+            for (int t = lane; t < 128; t += 32) {
+                const int col = c0 + t;
+                const bool ok = col < cend && (mk == nullptr || mk[col] != 0);
+                colvec(sm, MODE, s, 0)[t] =
+                    (MODE == DSD) ? 0.f : (ok ? a.cd.at(bh, col) * kLog2e : -INFINITY);
+                if (MODE == WSUM) colvec(sm, MODE, s, 1)[t] = ok ? a.w.at(bh, col) : 0.f;
+                if (MODE == DS1) {
+#pragma unroll
+                    for (int k = 0; k < MAXT; ++k)
+                        if (k < a.nterms)
+                            colvec(sm, MODE, s, 1 + k)[t] =
+                                ok ? (a.cv[k].p ? a.cv[k].at(bh, col) : 1.f) : 0.f;
+                }
+                if (MODE == DSD) {
+#pragma unroll
+                    for (int k = 0; k < MAXT; ++k)
+                        if (k < a.nterms) {
+                            colvec(sm, MODE, s, k)[t] =
+                                ok ? a.ec[k].at(bh, col) * kLog2e : -INFINITY;
+                            colvec(sm, MODE, s, MAXT + k)[t] =
+                                (ok && a.cc[k].p) ? a.cc[k].at(bh, col) : 0.f;
+                        }
+                }
+            }
+            tc::mbar_arrive(bar + B_FULL + s);
+        }
+        // after an abort, let the tile loads already issued land before teardown
+        if (lane == 0 && *abort_flag) {
+            tc::mbar_wait(bar + B_A, 0, kWaitBudget);
+            for (int c = max(0, issued - NST); c < issued; ++c)
+                tc::mbar_wait(bar + B_FULL + c % NST, (c / NST) & 1, kWaitBudget);
+        }
+        __syncwarp();
+    } else if (warp == 9) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            const uint32_t id_s = tc::idesc_bf16(128, 128, false, false);
+            const uint32_t id_o = tc::idesc_bf16(128, 64, false, true);
+            const uint32_t sA = tc::smem_u32(sm), sA2 = tc::smem_u32(sm + off_a2(MODE));
+            const uint32_t sP = tc::smem_u32(sm + off_p(MODE));
+            auto issue_pv = [&](int c) -> bool {
+                const int pb = c & 1, s = c % NST;
+                if (!ctl.wait(B_PFULL + pb, (c >> 1) & 1)) return false;
+                tc::tc_fence_after();
+                const uint32_t sX = tc::smem_u32(sm + off_stage(MODE) + s * stage_bytes(MODE)) +
+                                    (MODE == PV ? TILE : 0);
+                const uint32_t pbase = sP + pb * 2 * TILE;
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    const uint64_t ad = tc::sdesc_sw128(pbase + (k >> 2) * TILE + (k & 3) * 32, 16, 1024);
+                    const uint64_t bd = tc::sdesc_sw128(sX + k * 2048, TILE, 1024);
+                    tc::mma_bf16(tO, ad, bd, id_o, (c > 0 || k > 0) ? 1u : 0u);
+                }
+                tc::tc_commit(bar + B_PEMPTY + pb);
+                tc::tc_commit(bar + B_EMPTY + s);
+                return true;
+            };
+            bool ok = ctl.wait(B_A, 0);
+            for (int c = 0; ok && c < nch; ++c) {
+                const int s = c % NST, b = c % NSB;
+                if (!ctl.wait(B_FULL + s, (c / NST) & 1)) { ok = false; break; }
+                if (c >= NSB && !ctl.wait(B_SEMPTY + b, ((c / NSB) - 1) & 1)) { ok = false; break; }
+                tc::tc_fence_after();
+                const uint32_t sB = tc::smem_u32(sm + off_stage(MODE) + s * stage_bytes(MODE));
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    tc::mma_bf16(tS + 128 * b, tc::sdesc_sw128(sA + 32 * k, 16, 1024),
+                                 tc::sdesc_sw128(sB + 32 * k, 16, 1024), id_s, k > 0);
+                }
+                if (DS) {
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        tc::mma_bf16(tG, tc::sdesc_sw128(sA2 + 32 * k, 16, 1024),
+                                     tc::sdesc_sw128(sB + TILE + 32 * k, 16, 1024), id_s, k > 0);
+                    }
+                }
+                tc::tc_commit(bar + B_SFULL + b);
+                if (!HASX) tc::tc_commit(bar + B_EMPTY + s);
+                if (HASX && c >= 1 && !issue_pv(c - 1)) { ok = false; break; }
+            }
+            if (HASX && ok && nch > 0) ok = issue_pv(nch - 1);
+            if (HASX) tc::tc_commit(bar + B_OFULL);
+            // drain: every MMA issued above has completed once this arrives
+            tc::tc_commit(bar + B_DRAIN);
+            tc::mbar_wait(bar + B_DRAIN, 0, kWaitBudget);
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------------ epilogue
+        const int qd = warp & 3, hf = warp >> 2;
+        const int lr = qd * 32 + lane;          // local row
+        const int r = r0 + lr;                  // global row
+        const bool rok = r < L && (mk == nullptr || mk[r] != 0);
+        const float c2 = a.c2;
+        // row-side values
+        float rd2 = 0.f;
+        if (r < L) {
+            if (MODE == LSE) rd2 = ONLINE ? 0.f : a.rd.at(bh, r) * kLog2e;
+            else if (MODE != DSD) rd2 = a.rd.at(bh, r) * kLog2e;
+        }
+        float rmod[MAXT], rmod2[MAXT];
+#pragma unroll
+        for (int k = 0; k < MAXT; ++k) {
+            rmod[k] = 0.f;
+            rmod2[k] = 0.f;
+            if (k < a.nterms && r < L) {
+                if (MODE == DS1) rmod[k] = a.rv[k].p ? a.rv[k].at(bh, r) : 1.f;
+                if (MODE == DSD) {
+                    rmod[k] = a.er[k].at(bh, r) * kLog2e;
+                    rmod2[k] = a.cr[k].p ? a.cr[k].at(bh, r) : 0.f;
+                }
+            }
+        }
+        float m = -INFINITY, acc = 0.f;   // LSE online max / running sum; WSUM sum
+        uint64_t accp[4] = {0, 0, 0, 0};  // packed partial sums (LSE with shift, WSUM)
+        const int rw0 = r0 + qd * 32;       // first row of this warp
+        const uint32_t lanebase = (uint32_t)(qd * 32) << 16;
+        uint8_t* Pb = sm + off_p(MODE);
+
+        for (int c = 0; c < nch; ++c) {
+            const int s = c % NST, b = c % NSB, pb = c & 1;
+            if (!ctl.wait(B_FULL + s, (c / NST) & 1)) break;
+            if (!ctl.wait(B_SFULL + b, (c / NSB) & 1)) break;
+            if (HASX && c >= 2 && !ctl.wait(B_PEMPTY + pb, ((c >> 1) - 1) & 1)) break;
+            tc::tc_fence_after();
+            const int c0 = cbeg + 128 * c;
+            const float* cvs = colvec(sm, MODE, s, 0) + 64 * hf;
+#pragma unroll 1
+            for (int g = 0; g < 2; ++g) {
+                float sv[32], gv[DS ? 32 : 1], pv[32];
+                {
+                    uint32_t u[32];
+                    tc::tmem_ld32(tS + 128 * b + lanebase + 64 * hf + 32 * g, u);
+                    tc::tmem_wait_ld();
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) sv[j] = __uint_as_float(u[j]);
+                    if (DS) {
+                        tc::tmem_ld32(tG + lanebase + 64 * hf + 32 * g, u);
+                        tc::tmem_wait_ld();
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) gv[j] = __uint_as_float(u[j]);
+                    }
+                }
+                if (g == 1) {  // every TMEM read of this chunk is done
+                    tc::tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) tc::mbar_arrive(bar + B_SEMPTY + b);
+                }
+                // band test for this warp's 32 rows x these 32 columns (warp-uniform)
+                const int cg = c0 + 64 * hf + 32 * g;
+                const bool all_in = (cg >= rw0 + 31 - W) && (cg + 31 <= rw0 + W);
+                const bool all_out = (cg + 31 < rw0 - W) || (cg > rw0 + 31 + W);
+                const float* ce = cvs + 32 * g;
+                if (MODE == LSE || MODE == WSUM || MODE == PV) {
+                    if (all_out) {
+                        if (MODE == PV) {
+#pragma unroll
+                            for (int j = 0; j < 32; ++j) pv[j] = 0.f;
+                        }
+                    } else {
+                        float x[32];
+                        group_args(sv, ce, rd2, c2, !all_in, r, cg, W, x);
+                        if (MODE == LSE && ONLINE) {
+                            float mloc = -INFINITY;
+#pragma unroll
+                            for (int j = 0; j < 32; ++j) mloc = fmaxf(mloc, x[j]);
+                            if (mloc > m) {
+                                acc *= ex2(m - mloc);
+                                m = mloc;
+                            }
+                            if (m != -INFINITY) {
+#pragma unroll
+                                for (int j = 0; j < 32; ++j) acc += ex2(x[j] - m);
+                            }
+                        } else if (MODE == LSE) {
+#pragma unroll
+                            for (int q = 0; q < 16; ++q)
+                                accp[q & 3] = tc::add2(accp[q & 3],
+                                                       tc::pk2(ex2(x[2 * q]), ex2(x[2 * q + 1])));
+                        } else if (MODE == WSUM) {
+                            const float4* w4 = reinterpret_cast<const float4*>(
+                                colvec(sm, MODE, s, 1) + 64 * hf + 32 * g);
+#pragma unroll
+                            for (int q = 0; q < 8; ++q) {
+                                const float4 wv = w4[q];
+                                accp[(2 * q) & 3] =
+                                    tc::fma2(tc::pk2(ex2(x[4 * q]), ex2(x[4 * q + 1])),
+                                             tc::pk2(wv.x, wv.y), accp[(2 * q) & 3]);
+                                accp[(2 * q + 1) & 3] =
+                                    tc::fma2(tc::pk2(ex2(x[4 * q + 2]), ex2(x[4 * q + 3])),
+                                             tc::pk2(wv.z, wv.w), accp[(2 * q + 1) & 3]);
+                            }
+                        } else {  // PV
+#pragma unroll
+                            for (int j = 0; j < 32; ++j) pv[j] = ex2(x[j]);
+                        }
+                    }
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        bool in = !all_out;
+                        if (!all_in && !all_out) {
+                            const int d = r - (cg + j);
+                            in = d <= W && d >= -W;
+                        }
+                        if (MODE == DSD) {
+                            float val = 0.f;
+#pragma unroll
+                            for (int k = 0; k < MAXT; ++k)
+                                if (k < a.nterms) {
+                                    const float ek = colvec(sm, MODE, s, k)[64 * hf + 32 * g + j];
+                                    const float pk = ex2(fmaf(c2, sv[j], rmod[k] + ek));
+                                    const float coef =
+                                        a.gk[k] * gv[j] + rmod2[k] +
+                                        colvec(sm, MODE, s, MAXT + k)[64 * hf + 32 * g + j];
+                                    val = fmaf(pk, coef, val);
+                                }
+                            pv[j] = in ? val : 0.f;
+                        } else {  // DS1
+                            const float x = in ? fmaf(c2, sv[j], ce[j] + rd2) : -INFINITY;
+                            float M = gv[j];
+#pragma unroll
+                            for (int k = 0; k < MAXT; ++k)
+                                if (k < a.nterms)
+                                    M = fmaf(rmod[k], colvec(sm, MODE, s, 1 + k)[64 * hf + 32 * g + j],
+                                             M);
+                            pv[j] = in ? ex2(x) * M : 0.f;
+                        }
+                    }
+                }
+                if (HASX) {
+                    uint8_t* dst = Pb + pb * 2 * TILE + hf * TILE;
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        uint4 w;
+                        w.x = tc::pack_bf16(pv[8 * q + 0], pv[8 * q + 1]);
+                        w.y = tc::pack_bf16(pv[8 * q + 2], pv[8 * q + 3]);
+                        w.z = tc::pack_bf16(pv[8 * q + 4], pv[8 * q + 5]);
+                        w.w = tc::pack_bf16(pv[8 * q + 6], pv[8 * q + 7]);
+                        *reinterpret_cast<uint4*>(dst + tc::sw128_off(lr, 4 * g + q)) = w;
+                    }
+                }
+            }
+            if (HASX) {
+                tc::fence_async_smem();
+                __syncwarp();
+                if (lane == 0) tc::mbar_arrive(bar + B_PFULL + pb);
+            }
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(bar + B_EMPTY + s);
+        }
+
+        // ---------------------------------------------------------- finish
+        if ((MODE == LSE && !ONLINE) || MODE == WSUM) {
+            float a0, a1, a2, a3, a4, a5, a6, a7;
+            tc::upk2(accp[0], a0, a1);
+            tc::upk2(accp[1], a2, a3);
+            tc::upk2(accp[2], a4, a5);
+            tc::upk2(accp[3], a6, a7);
+            acc = ((a0 + a1) + (a2 + a3)) + ((a4 + a5) + (a6 + a7));
+        }
+        const float ce_d = a.dustbin ? a.cd.at(bh, L) * kLog2e : 0.f;
+        if (MODE == LSE || MODE == WSUM) {
+            // combine the two column halves of each row
+            if (MODE == LSE && !ONLINE) m = 0.f;  // the sum is relative to the shift
+            red[hf * 256 + lr] = m;
+            red[hf * 256 + 128 + lr] = acc;
+            asm volatile("bar.sync 1, 256;" ::: "memory");
+            if (hf == 0 && r < L && !*abort_flag) {
+                float m1 = red[lr], s1 = red[128 + lr];
+                const float m2 = red[256 + lr], s2 = red[384 + lr];
+                float out = 0.f;
+                if (MODE == LSE) {
+                    if (ONLINE) {
+                        lse_merge(m1, s1, m2, s2);
+                        if (a.dustbin) lse_merge(m1, s1, a.sd2 + ce_d, 1.f);
+                        out = -(m1 + lg2(s1)) * kLn2;
+                    } else {
+                        float tot = s1 + s2;
+                        if (a.dustbin) tot += ex2(a.sd2 + ce_d + rd2);
+                        out = (rd2 - lg2(tot)) * kLn2;
+                    }
+                } else {
+                    float tot = s1 + s2;
+                    if (a.dustbin) tot += ex2(a.sd2 + rd2 + ce_d) * a.w.at(bh, L);
+                    const float bb = a.base.p ? a.base.at(bh, r) : 0.f;
+                    const float mu = a.mult.p ? a.mult.at(bh, r) : 1.f;
+                    out = bb + a.sgn * mu * tot;
+                }
+                a.out_vec.at(bh, r) = rok ? out : 0.f;
+            }
+        } else {
+            // O accumulator: this warp reads columns 32*hf..+31 of its lanes
+            const bool okw = ctl.wait(B_OFULL, 0);
+            float o[32];
+            if (okw) {
+                tc::tc_fence_after();
+                uint32_t u0[32];
+                tc::tmem_ld32(tO + lanebase + 32 * hf, u0);
+                tc::tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < 32; ++j) o[j] = __uint_as_float(u0[j]);
+            }
+            const float scale = DS ? a.out_scale : 1.f;
+            if (MODE == PV && a.dustbin && a.Xd && rok) {
+                const float p = ex2(a.sd2 + rd2 + ce_d);
+                const float* xd = a.Xd + (size_t)(bh % a.H) * 64 + 32 * hf;
+#pragma unroll
+                for (int j = 0; j < 32; ++j) o[j] = fmaf(p, xd[j], o[j]);
+            }
+#pragma unroll
+            for (int j = 0; j < 32; ++j) o[j] = rok ? o[j] * scale : 0.f;
+            float dot = 0.f;
+            if (okw && r < L) {
+                __nv_bfloat16* outp =
+                    reinterpret_cast<__nv_bfloat16*>(a.out_mat) + ((size_t)bh * L + r) * 64 + 32 * hf;
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    uint4 w;
+                    w.x = tc::pack_bf16(o[8 * q + 0], o[8 * q + 1]);
+                    w.y = tc::pack_bf16(o[8 * q + 2], o[8 * q + 3]);
+                    w.z = tc::pack_bf16(o[8 * q + 4], o[8 * q + 5]);
+                    w.w = tc::pack_bf16(o[8 * q + 6], o[8 * q + 7]);
+                    reinterpret_cast<uint4*>(outp)[q] = w;
+                }
+                if (MODE == PV && a.Y) {
+                    const __nv_bfloat16* yp = reinterpret_cast<const __nv_bfloat16*>(a.Y) +
+                                              ((size_t)bh * L + r) * 64 + 32 * hf;
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) dot = fmaf(__bfloat162float(yp[j]), o[j], dot);
+                }
+            }
+            if (MODE == PV && a.Y) {
+                red[hf * 128 + lr] = dot;
+                asm volatile("bar.sync 1, 256;" ::: "memory");
+                if (hf == 0 && r < L && a.out_vec.p && !*abort_flag)
+                    a.out_vec.at(bh, r) = rok ? red[lr] + red[128 + lr] : 0.f;
+            }
+        }
+    }
+
+    tc::tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc::tc_fence_after();
+        tc::tmem_dealloc(tm, tmem_cols(MODE));
+    }
+}
+
+}  // namespace tcs
+}  // namespace sa

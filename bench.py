@@ -340,8 +340,12 @@ def main():
     dom = max(kern.items(), key=lambda kv: kv[1][0])
     dom_kind, (dom_ms, dom_n) = dom[0], dom[1]
     avg_ms = dom_ms / dom_n
-    simt = dom_kind != "fused_sweep"
+    # bf16 storage without a dustbin runs on the tensor cores; the rest on FP32 SIMT
+    simt = not (w.dtype == "bf16" and not w.dustbin)
     achieved = CONTRACTIONS.get(dom_kind, 1) * unit_flops / (avg_ms * 1e-3) / 1e12
+    # exponentials: one per support entry per launch of a sweep (diagnostic ceiling)
+    mufu_peak = 148 * 16 * peaks["sm_max_mhz"] * 1e6
+    exp_rate = (omega / (avg_ms * 1e-3)) if dom_kind in ("lse_sweep", "fused_sweep", "wsum", "pv") else None
     if simt:
         peak = fp32_alu_peak_tflops(peaks["sm_max_mhz"])
         roof = {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
@@ -353,7 +357,9 @@ def main():
         roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                 "frac": achieved / peak, "traffic": None, "kernel": dom_kind,
                 "peak_source": f"{peaks['source']} bf16 dense (sustained)",
-                "launches_per_step": dom_n / args.steps, "avg_launch_ms": avg_ms}
+                "launches_per_step": dom_n / args.steps, "avg_launch_ms": avg_ms,
+                "exp_per_s": exp_rate, "exp_frac_of_mufu": (exp_rate / mufu_peak) if exp_rate else None,
+                "mufu_peak_per_s": mufu_peak}
     # the whole step against the method's roofline: (T + R + 9) band contractions at the
     # bf16 tensor peak vs the algorithmic bytes at the HBM peak, whichever is slower
     elt = 2 if w.dtype == "bf16" else 4

@@ -32,6 +32,15 @@ SMALL = [
     (160, 20, 0.7, 4, 2, "f32", "holes", True),
     (140, 11, 1.0, 2, 2, "bf16", None, True),
     (129, 1, 1.0, 3, 2, "bf16", "holes", False),
+    # tensor-core path (bf16, no dustbin): tiles of 128 rows x 128-column chunks
+    (17, 5, 0.8, 3, 2, "bf16", None, False),
+    (64, 0, 1.0, 2, 2, "bf16", None, False),
+    (100, 150, 1.0, 2, 2, "bf16", "holes", False),
+    (300, 200, 0.7, 0, 2, "bf16", None, False),
+    (384, 128, 1.0, 3, 1, "bf16", (200, 384), False),
+    (520, 64, 0.6, 4, 3, "bf16", "holes", False),
+    (700, 256, 1.0, 2, 4, "bf16", None, False),
+    (1000, 37, 0.9, 5, 2, "bf16", (600, 1000), False),
 ]
 
 
