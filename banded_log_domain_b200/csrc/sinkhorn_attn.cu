@@ -282,7 +282,7 @@ bool make_map(CUtensorMap* m, const void* ptr, int L, int BH) {
            CUDA_SUCCESS;
 }
 
-template <int MODE, bool ONLINE>
+template <int MODE, bool ONLINE, int NT>
 cudaError_t launch_tc(const simt::SweepArgs& a, int BH, cudaStream_t st, Tracer& tr,
                       int* status) {
     tcs::Maps maps;
@@ -293,11 +293,11 @@ cudaError_t launch_tc(const simt::SweepArgs& a, int BH, cudaStream_t st, Tracer&
     if (!ok) return cudaErrorInvalidValue;
     const dim3 grid((a.L + 127) / 128, BH);
     const int smem = tcs::smem_bytes(MODE);
-    cudaError_t e = cudaFuncSetAttribute(tcs::tc_band_sweep<MODE, ONLINE>,
+    cudaError_t e = cudaFuncSetAttribute(tcs::tc_band_sweep<MODE, ONLINE, NT>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     tr.begin(kind_of(MODE));
-    tcs::tc_band_sweep<MODE, ONLINE><<<grid, tcs::NTHREADS, smem, st>>>(a, maps, status);
+    tcs::tc_band_sweep<MODE, ONLINE, NT><<<grid, tcs::NTHREADS, smem, st>>>(a, maps, status);
     tr.end();
     return cudaGetLastError();
 }
@@ -308,8 +308,20 @@ cudaError_t launch_sweep(const simt::SweepArgs& a, int BH, cudaStream_t st, Trac
     // bf16 storage without a dustbin runs on the tensor cores
     if constexpr (std::is_same<T, __nv_bfloat16>::value) {
         if (!a.dustbin) {
-            if (MODE == simt::LSE && a.online) return launch_tc<MODE, true>(a, BH, st, tr, status);
-            return launch_tc<MODE, false>(a, BH, st, tr, status);
+            if constexpr (MODE == simt::LSE) {
+                if (a.online) return launch_tc<MODE, true, 0>(a, BH, st, tr, status);
+                return launch_tc<MODE, false, 0>(a, BH, st, tr, status);
+            } else if constexpr (MODE == simt::DS1 || MODE == simt::DSD) {
+                switch (a.nterms) {  // 2R terms, R = 1..4
+                    case 2: return launch_tc<MODE, false, 2>(a, BH, st, tr, status);
+                    case 4: return launch_tc<MODE, false, 4>(a, BH, st, tr, status);
+                    case 6: return launch_tc<MODE, false, 6>(a, BH, st, tr, status);
+                    case 8: return launch_tc<MODE, false, 8>(a, BH, st, tr, status);
+                    default: return cudaErrorInvalidValue;
+                }
+            } else {
+                return launch_tc<MODE, false, 0>(a, BH, st, tr, status);
+            }
         }
     }
     const int nblk = (a.L + simt::BM - 1) / simt::BM;

@@ -113,7 +113,8 @@ __device__ __forceinline__ void group_args(const float (&sv)[32], const float* c
 }
 
 // ---------------------------------------------------------------------------
-template <int MODE, bool ONLINE>
+// NT: number of modifier (DS1) or staircase (DSD) terms, 2R; 0 for the other modes.
+template <int MODE, bool ONLINE, int NT>
 __global__ void __launch_bounds__(NTHREADS, (MODE == LSE || MODE == WSUM) ? 2 : 1) tc_band_sweep(const SweepArgs a,
                                                          const __grid_constant__ Maps maps,
                                                          int* status) {
@@ -195,15 +196,14 @@ __global__ void __launch_bounds__(NTHREADS, (MODE == LSE || MODE == WSUM) ? 2 : 
                 if (MODE == WSUM) colvec(sm, MODE, s, 1)[t] = ok ? a.w.at(bh, col) : 0.f;
                 if (MODE == DS1) {
 #pragma unroll
-                    for (int k = 0; k < MAXT; ++k)
-                        if (k < a.nterms)
-                            colvec(sm, MODE, s, 1 + k)[t] =
-                                ok ? (a.cv[k].p ? a.cv[k].at(bh, col) : 1.f) : 0.f;
+                    for (int k = 0; k < NT; ++k)
+                        colvec(sm, MODE, s, 1 + k)[t] =
+                            ok ? (a.cv[k].p ? a.cv[k].at(bh, col) : 1.f) : 0.f;
                 }
                 if (MODE == DSD) {
 #pragma unroll
-                    for (int k = 0; k < MAXT; ++k)
-                        if (k < a.nterms) {
+                    for (int k = 0; k < NT; ++k)
+                        {
                             colvec(sm, MODE, s, k)[t] =
                                 ok ? a.ec[k].at(bh, col) * kLog2e : -INFINITY;
                             colvec(sm, MODE, s, MAXT + k)[t] =
@@ -287,12 +287,12 @@ __global__ void __launch_bounds__(NTHREADS, (MODE == LSE || MODE == WSUM) ? 2 : 
             if (MODE == LSE) rd2 = ONLINE ? 0.f : a.rd.at(bh, r) * kLog2e;
             else if (MODE != DSD) rd2 = a.rd.at(bh, r) * kLog2e;
         }
-        float rmod[MAXT], rmod2[MAXT];
+        float rmod[NT > 0 ? NT : 1], rmod2[NT > 0 ? NT : 1];
 #pragma unroll
-        for (int k = 0; k < MAXT; ++k) {
+        for (int k = 0; k < NT; ++k) {
             rmod[k] = 0.f;
             rmod2[k] = 0.f;
-            if (k < a.nterms && r < L) {
+            if (r < L) {
                 if (MODE == DS1) rmod[k] = a.rv[k].p ? a.rv[k].at(bh, r) : 1.f;
                 if (MODE == DSD) {
                     rmod[k] = a.er[k].at(bh, r) * kLog2e;
@@ -384,36 +384,65 @@ __global__ void __launch_bounds__(NTHREADS, (MODE == LSE || MODE == WSUM) ? 2 : 
                             for (int j = 0; j < 32; ++j) pv[j] = ex2(x[j]);
                         }
                     }
-                } else {
+                } else if (all_out) {
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) {
-                        bool in = !all_out;
-                        if (!all_in && !all_out) {
-                            const int d = r - (cg + j);
-                            in = d <= W && d >= -W;
+                    for (int j = 0; j < 32; ++j) pv[j] = 0.f;
+                } else if (MODE == DS1) {
+                    // dS = P * M,  M = G + sum_k rv_k[row] cv_k[col]
+                    float x[32];
+                    group_args(sv, ce, rd2, c2, !all_in, r, cg, W, x);
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) {
+                        uint64_t m01 = tc::pk2(gv[4 * q], gv[4 * q + 1]);
+                        uint64_t m23 = tc::pk2(gv[4 * q + 2], gv[4 * q + 3]);
+#pragma unroll
+                        for (int k = 0; k < NT; ++k) {
+                            const float4 cv = reinterpret_cast<const float4*>(
+                                colvec(sm, MODE, s, 1 + k) + 64 * hf + 32 * g)[q];
+                            const uint64_t rk = tc::pk2(rmod[k], rmod[k]);
+                            m01 = tc::fma2(rk, tc::pk2(cv.x, cv.y), m01);
+                            m23 = tc::fma2(rk, tc::pk2(cv.z, cv.w), m23);
                         }
-                        if (MODE == DSD) {
-                            float val = 0.f;
+                        float M0, M1, M2, M3;
+                        tc::upk2(m01, M0, M1);
+                        tc::upk2(m23, M2, M3);
+                        pv[4 * q] = ex2(x[4 * q]) * M0;
+                        pv[4 * q + 1] = ex2(x[4 * q + 1]) * M1;
+                        pv[4 * q + 2] = ex2(x[4 * q + 2]) * M2;
+                        pv[4 * q + 3] = ex2(x[4 * q + 3]) * M3;
+                    }
+                } else {
+                    // DSD: dS = sum_k exp(S + er_k[row] + ec_k[col]) (g_k G + cr_k[row] + cc_k[col])
+                    const uint64_t c2p = tc::pk2(c2, c2);
 #pragma unroll
-                            for (int k = 0; k < MAXT; ++k)
-                                if (k < a.nterms) {
-                                    const float ek = colvec(sm, MODE, s, k)[64 * hf + 32 * g + j];
-                                    const float pk = ex2(fmaf(c2, sv[j], rmod[k] + ek));
-                                    const float coef =
-                                        a.gk[k] * gv[j] + rmod2[k] +
-                                        colvec(sm, MODE, s, MAXT + k)[64 * hf + 32 * g + j];
-                                    val = fmaf(pk, coef, val);
-                                }
-                            pv[j] = in ? val : 0.f;
-                        } else {  // DS1
-                            const float x = in ? fmaf(c2, sv[j], ce[j] + rd2) : -INFINITY;
-                            float M = gv[j];
+                    for (int q = 0; q < 8; ++q) {
+                        float v4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                            for (int k = 0; k < MAXT; ++k)
-                                if (k < a.nterms)
-                                    M = fmaf(rmod[k], colvec(sm, MODE, s, 1 + k)[64 * hf + 32 * g + j],
-                                             M);
-                            pv[j] = in ? ex2(x) * M : 0.f;
+                        for (int k = 0; k < NT; ++k) {
+                            const float4 ev = reinterpret_cast<const float4*>(
+                                colvec(sm, MODE, s, k) + 64 * hf + 32 * g)[q];
+                            const float4 cv = reinterpret_cast<const float4*>(
+                                colvec(sm, MODE, s, MAXT + k) + 64 * hf + 32 * g)[q];
+                            const uint64_t rk = tc::pk2(rmod[k], rmod[k]);
+                            float x0, x1, x2, x3;
+                            tc::upk2(tc::fma2(tc::pk2(sv[4 * q], sv[4 * q + 1]), c2p,
+                                              tc::add2(tc::pk2(ev.x, ev.y), rk)), x0, x1);
+                            tc::upk2(tc::fma2(tc::pk2(sv[4 * q + 2], sv[4 * q + 3]), c2p,
+                                              tc::add2(tc::pk2(ev.z, ev.w), rk)), x2, x3);
+                            const float gk = a.gk[k], ck = rmod2[k];
+                            v4[0] = fmaf(ex2(x0), fmaf(gk, gv[4 * q], ck + cv.x), v4[0]);
+                            v4[1] = fmaf(ex2(x1), fmaf(gk, gv[4 * q + 1], ck + cv.y), v4[1]);
+                            v4[2] = fmaf(ex2(x2), fmaf(gk, gv[4 * q + 2], ck + cv.z), v4[2]);
+                            v4[3] = fmaf(ex2(x3), fmaf(gk, gv[4 * q + 3], ck + cv.w), v4[3]);
+                        }
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) pv[4 * q + e] = v4[e];
+                    }
+                    if (!all_in) {
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) {
+                            const int d = r - (cg + j);
+                            if ((unsigned)(d + W) > (unsigned)(2 * W)) pv[j] = 0.f;
                         }
                     }
                 }
