@@ -20,6 +20,7 @@
 // schedule runs the same sweeps with every staircase plan P^(r,r-1),
 // P^(r,r) formed by its own exponential.
 #include <cmath>
+#include <algorithm>
 #include <cstring>
 #include <mutex>
 
@@ -29,6 +30,7 @@
 
 #include "../../include/sinkhorn_attn.h"
 #include "simt_sweep.cuh"
+#include "tc_fused.cuh"
 #include "tc_sweep.cuh"
 
 namespace sa {
@@ -90,6 +92,36 @@ bool mask_ok(const void* x) {
         return false;
     }
     return at.type != cudaMemoryTypeUnregistered;
+}
+
+// The fused forward (one pass per iteration) applies to bf16 storage without a
+// dustbin, W <= 256, and at least two iterations (the first is two sweeps).
+bool fused_fwd(const sa_params* p) {
+    return p->dtype == SA_BF16 && !p->dustbin && p->W <= 256 && p->T + p->R >= 2;
+}
+
+// Forward workspace: status header; for the fused forward two ping-pong column
+// dual vectors and two buffers of per-row-block column partials.
+struct FwdLayout {
+    size_t va, vb, p0, p1, total;
+    int nblk, ncol, nch;
+};
+FwdLayout fwd_layout(const Dims& d, const sa_params* p) {
+    FwdLayout l{};
+    l.total = kHeader;
+    if (!fused_fwd(p)) return l;
+    l.nblk = (d.L + 127) / 128;
+    l.ncol = 2 * p->W + 128;
+    l.nch = (l.ncol + 127) / 128;
+    const size_t vec = align_up((size_t)d.BH * d.ld * sizeof(float));
+    const size_t part = align_up((size_t)d.BH * d.L * tcf::NSLOT * sizeof(float));
+    size_t o = kHeader;
+    l.va = o; o += vec;
+    l.vb = o; o += vec;
+    l.p0 = o; o += part;
+    l.p1 = o; o += part;
+    l.total = o;
+    return l;
 }
 
 // Backward workspace layout (float32 vectors of BH * ld elements each).
@@ -423,6 +455,97 @@ sa_status fwd_impl(const Ctx& x, const T* q, const T* k, const T* v, const uint8
     return SA_OK;
 }
 
+// Forward with fused iterations (bf16, see fused_fwd).  Where each iterate lives:
+//   u_m: the state's u0 row while m <= T (updated in place), u^(m-T) after;
+//   v_m: ping-pong workspace vectors while m < T, the state's v0 row at m = T,
+//        v^(m-T) after; v_0 = 0 is the (zeroed) state v0 row.
+sa_status fwd_fused(const Ctx& x, const __nv_bfloat16* q, const __nv_bfloat16* k,
+                    const __nv_bfloat16* v, const uint8_t* mask, __nv_bfloat16* o, float* state,
+                    char* ws) {
+    const Dims& d = x.d;
+    const int T = x.p->T, R = d.R, K = T + R;
+    const FwdLayout l = fwd_layout(d, x.p);
+    SA_CUDA(cudaMemsetAsync(state, 0, (size_t)d.BH * (2 * R + 2) * d.ld * sizeof(float), x.st));
+    float* VA = (float*)(ws + l.va);
+    float* VB = (float*)(ws + l.vb);
+    float* PART[2] = {(float*)(ws + l.p0), (float*)(ws + l.p1)};
+    auto u_home = [&](int m) { return Vec{state + (size_t)(m <= T ? 0 : 2 * (m - T)) * d.ld, x.sst}; };
+    auto v_home = [&](int m) {
+        if (m == 0) return Vec{state + (size_t)d.ld, x.sst};
+        if (m < T) return Vec{(m & 1) ? VA : VB, (long long)d.ld};
+        return Vec{state + (size_t)(2 * (m - T) + 1) * d.ld, x.sst};
+    };
+    auto mv = [](Vec a) { return MVec{const_cast<float*>(a.p), a.s}; };
+
+    // iteration 1: row sweep with a running max, then column sweep
+    simt::SweepArgs a = base_args(x);
+    a.mask = mask;
+    a.A = q; a.Bo = k;
+    a.cd = v_home(0);
+    a.rd = v_home(0);
+    a.online = 1;
+    a.out_vec = mv(u_home(1));
+    SA_CUDA((launch_sweep<__nv_bfloat16, simt::LSE>(a, d.BH, x.st, x.tr, x.status)));
+    a.A = k; a.Bo = q;
+    a.cd = u_home(1);
+    a.rd = v_home(0);
+    a.online = 0;
+    a.out_vec = mv(v_home(1));
+    SA_CUDA((launch_sweep<__nv_bfloat16, simt::LSE>(a, d.BH, x.st, x.tr, x.status)));
+
+    // iterations 2..K: one fused pass each
+    CUtensorMap mq, mk;
+    if (!make_map(&mq, q, d.L, d.BH) || !make_map(&mk, k, d.L, d.BH)) return SA_ERR_CUDA;
+    int dev = 0, nsm = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess)
+        cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+    const int ntiles = d.BH * l.nblk;
+    const dim3 grid(std::min(nsm, ntiles));
+    SA_CUDA(cudaFuncSetAttribute(tcf::tc_fused_iter, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 tcf::SMEM_BYTES));
+    tcf::FusedArgs f;
+    std::memset(&f, 0, sizeof(f));
+    f.L = d.L; f.W = x.p->W; f.H = d.H; f.BH = d.BH;
+    f.nblk = l.nblk; f.ncol = l.ncol; f.nch = l.nch;
+    f.c2 = x.c * kLog2e;
+    f.mask = mask;
+    f.status = x.status;
+    for (int it = 2; it <= K; ++it) {
+        f.u_prev = u_home(it - 1);
+        f.u_out = mv(u_home(it));
+        if (it == 2) {
+            f.v_src = v_home(1);
+            f.v_out = MVec{nullptr, 0};
+            f.part_in = nullptr;
+        } else {
+            f.v_src = v_home(it - 2);
+            f.v_out = mv(v_home(it - 1));
+            f.part_in = PART[(it - 1) & 1];
+        }
+        f.part_out = PART[it & 1];
+        x.tr.begin(SA_KERNEL_FUSED_SWEEP);
+        tcf::tc_fused_iter<<<grid, tcf::NTHREADS, tcf::SMEM_BYTES, x.st>>>(f, mq, mk);
+        x.tr.end();
+        SA_CUDA(cudaGetLastError());
+    }
+    // v_K from the last partials
+    f.v_src = v_home(K - 1);
+    f.part_in = PART[K & 1];
+    const long long n = (long long)d.BH * d.L;
+    SA_AUX(x.tr, tcf::k_finalize_v<<<(unsigned)((n + 255) / 256), 256, 0, x.st>>>(f, mv(v_home(K))));
+
+    // O = P^(R,R) V
+    simt::SweepArgs b = base_args(x);
+    b.mask = mask;
+    b.dust_cta = 0;
+    b.A = q; b.Bo = k; b.X = v;
+    b.rd = x.srow(2 * R);
+    b.cd = x.srow(2 * R + 1);
+    b.out_mat = o;
+    SA_CUDA((launch_sweep<__nv_bfloat16, simt::PV>(b, d.BH, x.st, x.tr, x.status)));
+    return SA_OK;
+}
+
 template <typename T>
 sa_status bwd_impl(const Ctx& x, const T* q, const T* k, const T* v, const uint8_t* mask,
                    const float* v_dust, const T* o, const T* dO, T* dq, T* dk, T* dv,
@@ -621,7 +744,7 @@ sa_status sinkhorn_attn_workspace_size(const sa_params* p, size_t* fwd_bytes, si
     Dims d;
     sa_status s = check_params(p, &d);
     if (s != SA_OK) return s;
-    if (fwd_bytes) *fwd_bytes = kHeader;
+    if (fwd_bytes) *fwd_bytes = fwd_layout(d, p).total;
     if (bwd_bytes) *bwd_bytes = bwd_layout(d).total;
     return SA_OK;
 }
@@ -632,7 +755,7 @@ sa_status sinkhorn_attn_fwd(const sa_params* p, const void* q, const void* k, co
     Dims d;
     sa_status s = check_params(p, &d);
     if (s != SA_OK) return s;
-    if (ws_bytes < kHeader) return SA_ERR_WORKSPACE;
+    if (ws_bytes < fwd_layout(d, p).total) return SA_ERR_WORKSPACE;
     if (d.BH == 0 || d.L == 0) return SA_OK;
     if (!device_ok(q) || !device_ok(k) || !device_ok(v) || !device_ok(o) || !device_ok(state) ||
         !device_ok(ws) || !mask_ok(mask))
@@ -652,6 +775,9 @@ sa_status sinkhorn_attn_fwd(const sa_params* p, const void* q, const void* k, co
     if (p->dtype == SA_F32)
         s = fwd_impl<float>(x, (const float*)q, (const float*)k, (const float*)v, mask, vd,
                             (float*)o, state);
+    else if (fused_fwd(p))
+        s = fwd_fused(x, (const __nv_bfloat16*)q, (const __nv_bfloat16*)k,
+                      (const __nv_bfloat16*)v, mask, (__nv_bfloat16*)o, state, (char*)ws);
     else
         s = fwd_impl<__nv_bfloat16>(x, (const __nv_bfloat16*)q, (const __nv_bfloat16*)k,
                                     (const __nv_bfloat16*)v, mask, vd, (__nv_bfloat16*)o, state);

@@ -33,14 +33,17 @@ __device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
                  "r"(bytes)
                  : "memory");
 }
+// Tests the phase; a thread whose phase is not complete is suspended by the
+// hardware until it completes or about 20 microseconds pass (the hint), so
+// waiting warps do not spin on the issue slots.
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(20000)
         : "memory");
     return ok != 0;
 }
@@ -146,6 +149,13 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo_byt
     d |= (uint64_t)1 << 46;
     d |= (uint64_t)2 << 61;
     return d;
+}
+// The descriptor of the same matrix `bytes` further on (bytes a multiple of
+// 16; shared-memory addresses stay below 256 KB, so the 14-bit start field
+// does not carry).  Building descriptors once and advancing them this way keeps
+// the single MMA-issuing thread from stalling on integer dependency chains.
+__device__ __forceinline__ uint64_t sdesc_add(uint64_t desc, uint32_t bytes) {
+    return desc + (uint64_t)(bytes >> 4);
 }
 // Instruction descriptor for kind::f16 with bf16 A and B and fp32 D.
 // a_mn / b_mn: operand stored MN-major (else K-major).

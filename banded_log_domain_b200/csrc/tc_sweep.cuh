@@ -67,7 +67,7 @@ __host__ __device__ constexpr int smem_bytes(int m) { return off_bar(m) + 64 * 8
 
 // barrier slots
 enum { B_A = 0, B_FULL = 1, B_EMPTY = 5, B_SFULL = 9, B_SEMPTY = 11, B_PFULL = 13, B_PEMPTY = 15,
-       B_OFULL = 17, B_DRAIN = 18, NBAR = 19 };
+       B_OFULL = 17, B_DRAIN = 18, B_EPI = 19, NBAR = 20 };
 
 struct Ctl {
     uint64_t* bar;
@@ -79,6 +79,15 @@ struct Ctl {
         *abort = 1;
         if (status) atomicCAS(status, 0, (int)SA_ERR_TIMEOUT);
         return false;
+    }
+    // every epilogue warp arrives once (after its lanes converge), then all
+    // lanes wait (bounded) for the phase
+    __device__ bool epi_sync(uint32_t& phase) {
+        __syncwarp();
+        if ((threadIdx.x & 31) == 0) tc::mbar_arrive(bar + B_EPI);
+        const bool ok = wait(B_EPI, phase & 1);
+        ++phase;
+        return ok;
     }
 };
 
@@ -151,6 +160,7 @@ __global__ void __launch_bounds__(NTHREADS, (MODE == LSE || MODE == WSUM) ? 2 : 
         }
         tc::mbar_init(bar + B_OFULL, 1);
         tc::mbar_init(bar + B_DRAIN, 1);
+        tc::mbar_init(bar + B_EPI, 8);
         *abort_flag = 0;
         tc::fence_mbar_init();
     }
@@ -225,20 +235,22 @@ __global__ void __launch_bounds__(NTHREADS, (MODE == LSE || MODE == WSUM) ? 2 : 
         if (lane == 0) {
             const uint32_t id_s = tc::idesc_bf16(128, 128, false, false);
             const uint32_t id_o = tc::idesc_bf16(128, 64, false, true);
-            const uint32_t sA = tc::smem_u32(sm), sA2 = tc::smem_u32(sm + off_a2(MODE));
-            const uint32_t sP = tc::smem_u32(sm + off_p(MODE));
+            // descriptors built once; offsets are added in 16-byte units
+            const uint64_t dA = tc::sdesc_sw128(tc::smem_u32(sm), 16, 1024);
+            const uint64_t dA2 = tc::sdesc_sw128(tc::smem_u32(sm + off_a2(MODE)), 16, 1024);
+            const uint64_t dStK = tc::sdesc_sw128(tc::smem_u32(sm + off_stage(MODE)), 16, 1024);
+            const uint64_t dStMN = tc::sdesc_sw128(tc::smem_u32(sm + off_stage(MODE)), TILE, 1024);
+            const uint64_t dP = tc::sdesc_sw128(tc::smem_u32(sm + off_p(MODE)), 16, 1024);
             auto issue_pv = [&](int c) -> bool {
                 const int pb = c & 1, s = c % NST;
                 if (!ctl.wait(B_PFULL + pb, (c >> 1) & 1)) return false;
                 tc::tc_fence_after();
-                const uint32_t sX = tc::smem_u32(sm + off_stage(MODE) + s * stage_bytes(MODE)) +
-                                    (MODE == PV ? TILE : 0);
-                const uint32_t pbase = sP + pb * 2 * TILE;
+                const uint64_t dX = tc::sdesc_add(dStMN, s * stage_bytes(MODE) + (MODE == PV ? TILE : 0));
+                const uint64_t dPb = tc::sdesc_add(dP, pb * 2 * TILE);
 #pragma unroll
                 for (int k = 0; k < 8; ++k) {
-                    const uint64_t ad = tc::sdesc_sw128(pbase + (k >> 2) * TILE + (k & 3) * 32, 16, 1024);
-                    const uint64_t bd = tc::sdesc_sw128(sX + k * 2048, TILE, 1024);
-                    tc::mma_bf16(tO, ad, bd, id_o, (c > 0 || k > 0) ? 1u : 0u);
+                    tc::mma_bf16(tO, tc::sdesc_add(dPb, (k >> 2) * TILE + (k & 3) * 32),
+                                 tc::sdesc_add(dX, k * 2048), id_o, (c > 0 || k > 0) ? 1u : 0u);
                 }
                 tc::tc_commit(bar + B_PEMPTY + pb);
                 tc::tc_commit(bar + B_EMPTY + s);
@@ -250,18 +262,16 @@ __global__ void __launch_bounds__(NTHREADS, (MODE == LSE || MODE == WSUM) ? 2 : 
                 if (!ctl.wait(B_FULL + s, (c / NST) & 1)) { ok = false; break; }
                 if (c >= NSB && !ctl.wait(B_SEMPTY + b, ((c / NSB) - 1) & 1)) { ok = false; break; }
                 tc::tc_fence_after();
-                const uint32_t sB = tc::smem_u32(sm + off_stage(MODE) + s * stage_bytes(MODE));
+                const uint64_t dB = tc::sdesc_add(dStK, s * stage_bytes(MODE));
 #pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    tc::mma_bf16(tS + 128 * b, tc::sdesc_sw128(sA + 32 * k, 16, 1024),
-                                 tc::sdesc_sw128(sB + 32 * k, 16, 1024), id_s, k > 0);
-                }
+                for (int k = 0; k < 4; ++k)
+                    tc::mma_bf16(tS + 128 * b, tc::sdesc_add(dA, 32 * k), tc::sdesc_add(dB, 32 * k),
+                                 id_s, k > 0);
                 if (DS) {
 #pragma unroll
-                    for (int k = 0; k < 4; ++k) {
-                        tc::mma_bf16(tG, tc::sdesc_sw128(sA2 + 32 * k, 16, 1024),
-                                     tc::sdesc_sw128(sB + TILE + 32 * k, 16, 1024), id_s, k > 0);
-                    }
+                    for (int k = 0; k < 4; ++k)
+                        tc::mma_bf16(tG, tc::sdesc_add(dA2, 32 * k), tc::sdesc_add(dB, TILE + 32 * k),
+                                     id_s, k > 0);
                 }
                 tc::tc_commit(bar + B_SFULL + b);
                 if (!HASX) tc::tc_commit(bar + B_EMPTY + s);
@@ -483,8 +493,9 @@ __global__ void __launch_bounds__(NTHREADS, (MODE == LSE || MODE == WSUM) ? 2 : 
             if (MODE == LSE && !ONLINE) m = 0.f;  // the sum is relative to the shift
             red[hf * 256 + lr] = m;
             red[hf * 256 + 128 + lr] = acc;
-            asm volatile("bar.sync 1, 256;" ::: "memory");
-            if (hf == 0 && r < L && !*abort_flag) {
+            uint32_t eph = 0;
+            const bool synced = ctl.epi_sync(eph);
+            if (synced && hf == 0 && r < L && !*abort_flag) {
                 float m1 = red[lr], s1 = red[128 + lr];
                 const float m2 = red[256 + lr], s2 = red[384 + lr];
                 float out = 0.f;
@@ -550,8 +561,9 @@ __global__ void __launch_bounds__(NTHREADS, (MODE == LSE || MODE == WSUM) ? 2 : 
             }
             if (MODE == PV && a.Y) {
                 red[hf * 128 + lr] = dot;
-                asm volatile("bar.sync 1, 256;" ::: "memory");
-                if (hf == 0 && r < L && a.out_vec.p && !*abort_flag)
+                uint32_t eph = 0;
+                const bool synced = ctl.epi_sync(eph);
+                if (synced && hf == 0 && r < L && a.out_vec.p && !*abort_flag)
                     a.out_vec.at(bh, r) = rok ? red[lr] + red[128 + lr] : 0.f;
             }
         }

@@ -59,7 +59,7 @@ def test_small_cases(case):
     r = parity.oracle_run(x, plans=plans, **kw)
     parity.compare(x, g, r, dtype=dtype, dustbin=db, schedules=("one_reference", "direct"),
                    label=str(case))
-    parity.compare_plans(g, r, plans, label=str(case))
+    parity.compare_plans(g, r, plans, dtype=dtype, label=str(case))
 
 
 def test_fully_padded_sequence_is_zero():
@@ -79,7 +79,7 @@ def _named(name, heads=None):
     r = parity.oracle_run(x, plans=[(2, 2)], heads=heads, **kw)
     parity.compare(x, g, r, dtype=w.dtype, dustbin=w.dustbin, heads=heads,
                    schedules=("one_reference", "direct"), label=name)
-    parity.compare_plans(g, r, [(2, 2)], heads=heads, label=name)
+    parity.compare_plans(g, r, [(2, 2)], dtype=w.dtype, heads=heads, label=name)
 
 
 def test_workload_small512():
