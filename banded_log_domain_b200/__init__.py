@@ -101,10 +101,12 @@ def _L():
     lib.sinkhorn_attn_debug_plan.argtypes = [P, ctypes.c_int, ctypes.c_int, vp, vp, vp, vp, vp,
                                              vp, vp, vp]
     lib.sinkhorn_attn_poll.argtypes = [vp, vp]
+    lib.sinkhorn_attn_debug_timeout.argtypes = [vp, ctypes.c_longlong, vp]
     lib.sinkhorn_attn_strerror.argtypes = [ctypes.c_int]
     lib.sinkhorn_attn_strerror.restype = ctypes.c_char_p
     for f in ("sinkhorn_attn_state_size", "sinkhorn_attn_workspace_size", "sinkhorn_attn_fwd",
-              "sinkhorn_attn_bwd", "sinkhorn_attn_debug_plan", "sinkhorn_attn_poll"):
+              "sinkhorn_attn_bwd", "sinkhorn_attn_debug_plan", "sinkhorn_attn_poll",
+              "sinkhorn_attn_debug_timeout"):
         getattr(lib, f).restype = ctypes.c_int
     _lib = lib
     return lib
@@ -117,7 +119,7 @@ def load():
 
 EXPORTS = ("sinkhorn_attn_state_size", "sinkhorn_attn_workspace_size", "sinkhorn_attn_fwd",
            "sinkhorn_attn_bwd", "sinkhorn_attn_bwd_static_ws", "sinkhorn_attn_debug_plan",
-           "sinkhorn_attn_poll", "sinkhorn_attn_strerror")
+           "sinkhorn_attn_poll", "sinkhorn_attn_strerror", "sinkhorn_attn_debug_timeout")
 
 
 def strerror(status: int) -> str:
@@ -276,6 +278,13 @@ def sinkhorn_attn_poll(ws) -> int:
 
 def sinkhorn_attn_strerror(status: int) -> str:
     return strerror(status)
+
+
+def sinkhorn_attn_debug_timeout(ws, budget_cycles: int = 1_000_000) -> int:
+    """Runs the library's bounded wait on a barrier nothing completes (test hook
+    for the failure path); the timeout lands in the status word of ``ws`` (a
+    CUDA tensor of at least 256 bytes) and is read by :func:`sinkhorn_attn_poll`."""
+    return int(_L().sinkhorn_attn_debug_timeout(_ptr(ws), int(budget_cycles), _stream(ws.device)))
 
 
 def score_scale(d: int, eps: float) -> float:

@@ -207,6 +207,21 @@ __global__ void k_dvd_reduce(const float* part, int B, int H, float* out) {
     out[g] = s;
 }
 
+// A wait that nothing completes: thread 0 waits on a fresh mbarrier (one
+// expected arrival, none made) for `budget` cycles through the library's
+// bounded wait, then records the timeout like any stalled pipeline stage.
+__global__ void k_stall(int* status, long long budget) {
+    __shared__ uint64_t bar;
+    if (threadIdx.x == 0) {
+        tc::mbar_init(&bar, 1);
+        tc::fence_mbar_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0 && !tc::mbar_wait(&bar, 0, budget))
+        atomicCAS(status, (int)SA_OK, (int)SA_ERR_TIMEOUT);
+    __syncthreads();
+}
+
 // Sets the status word when any element is NaN or Inf.
 template <typename T>
 __global__ void k_finite(const T* x, long long n, int* status) {
@@ -964,6 +979,13 @@ sa_status sinkhorn_attn_poll(void* ws, void* stream) {
     if (cudaMemcpy(ws, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess)
         return SA_ERR_CUDA;
     return (sa_status)h;
+}
+
+sa_status sinkhorn_attn_debug_timeout(void* ws, long long budget_cycles, void* stream) {
+    if (!ws || ((uintptr_t)ws & 15)) return SA_ERR_INVALID_ARG;
+    const long long b = budget_cycles < 1 ? 1 : (budget_cycles > 100000000LL ? 100000000LL : budget_cycles);
+    sa::k_stall<<<1, 32, 0, (cudaStream_t)stream>>>((int*)ws, b);
+    return cudaGetLastError() == cudaSuccess ? SA_OK : SA_ERR_CUDA;
 }
 
 const char* sinkhorn_attn_strerror(sa_status s) {

@@ -69,6 +69,29 @@ def fp32_alu_peak_tflops(sm_max_mhz):
 # algorithmic band contractions (2 d |Omega| FLOPs each) per launch of each kernel kind
 CONTRACTIONS = {"lse_sweep": 1, "fused_sweep": 1, "pv": 2, "wsum": 1, "ds": 3}
 
+# DRAM bytes (read + write) per launch from one ncu capture (profiles/), keyed by
+# (workload, kernel kind), with the SHA-256 of the kernel source the capture was
+# taken from: a changed source reports traffic as null until it is captured again.
+MEASURED_TRAFFIC = {
+    ("long32k", "fused_sweep"): (191.2e6, "banded_log_domain_b200/csrc/tc_fused.cuh",
+                                 "f7b219d71a10154bbd618f7631db54849bac5955dcb9fd8b0f1db432a5af97a4"),
+}
+
+
+def measured_traffic(workload, kind):
+    e = MEASURED_TRAFFIC.get((workload, kind))
+    if e is None:
+        return None
+    nbytes, src, digest = e
+    import hashlib
+    try:
+        with open(os.path.join(ROOT, src), "rb") as f:
+            if hashlib.sha256(f.read()).hexdigest() != digest:
+                return None
+    except OSError:
+        return None
+    return nbytes
+
 
 class ClockSampler:
     """nvidia-smi clocks / throttle reasons sampled every 200 ms."""
@@ -130,7 +153,9 @@ class ClockSampler:
                 "power_w_max": max(r["power"] for r in rows)}
 
 
-def dist_setup():
+def dist_setup(backend=None, timeout_s=120):
+    """One process per GPU (torchrun's RANK / LOCAL_RANK / WORLD_SIZE).  NCCL on
+    GPUs; the same code path runs on CPU with gloo (the multi-process tests)."""
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
@@ -139,18 +164,30 @@ def dist_setup():
 
         import torch.distributed as dist
 
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
+        if backend is None:
+            backend = "nccl" if torch.cuda.is_available() else "gloo"
+        kw = {}
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+            kw["device_id"] = torch.device("cuda", local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=timeout_s), **kw)
     return ws, rank, local
 
 
+def _coll_device():
+    import torch.distributed as dist
+
+    return "cuda" if dist.get_backend() == "nccl" else "cpu"
+
+
 def allreduce_max(x: float, ws: int) -> float:
+    """The largest value over the ranks (per-step device time: the job ends with
+    its slowest rank)."""
     if ws == 1:
         return x
     import torch.distributed as dist
 
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=_coll_device())
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 
@@ -160,6 +197,12 @@ def barrier(ws):
         import torch.distributed as dist
 
         dist.barrier()
+
+
+def whole_job_value(ws: int, units_per_rank: float, ms_per_step: float) -> float:
+    """Weak scaling: every rank processes its own copy of the workload, so the
+    job's throughput is all ranks' units over the slowest rank's step time."""
+    return ws * units_per_rank / (ms_per_step * 1e-3)
 
 
 # ---------------------------------------------------------------------------
@@ -326,7 +369,7 @@ def main():
     total_ms = allreduce_max(sum(step_ms), ws)
     ms_per_step = total_ms / args.steps
     units = w.B * w.H * w.L
-    value = ws * units / (ms_per_step * 1e-3)
+    value = whole_job_value(ws, units, ms_per_step)
 
     peaks = load_peaks()
     # per-problem support size (valid tokens; workloads with masks use their mean)
@@ -355,7 +398,8 @@ def main():
     else:
         peak = peaks["bf16_tflops_sustained"]
         roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                "frac": achieved / peak, "traffic": None, "kernel": dom_kind,
+                "frac": achieved / peak, "traffic": measured_traffic(w.name, dom_kind),
+                "kernel": dom_kind,
                 "peak_source": f"{peaks['source']} bf16 dense (sustained)",
                 "launches_per_step": dom_n / args.steps, "avg_launch_ms": avg_ms,
                 "exp_per_s": exp_rate, "exp_frac_of_mufu": (exp_rate / mufu_peak) if exp_rate else None,

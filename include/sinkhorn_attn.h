@@ -191,6 +191,18 @@ sa_status sinkhorn_attn_poll(void* ws, void* stream);
 /* Static English description of a status code. */
 const char* sinkhorn_attn_strerror(sa_status s);
 
+/* Test hook for the failure path; no counterpart in the pages.  Launches on
+ * `stream` one CTA whose thread waits, through the same bounded mbarrier wait
+ * every kernel of this library uses, on a barrier that nothing ever arrives on;
+ * after `budget_cycles` SM clock cycles (clamped to [1, 1e8], at most about
+ * 50 ms) the wait gives up and records SA_ERR_TIMEOUT in the status word of
+ * `ws` (a workspace of at least 256 bytes, device memory), exactly as a
+ * stalled pipeline stage would.  Nothing faults and the CUDA context stays
+ * usable; sinkhorn_attn_poll(ws, stream) then returns SA_ERR_TIMEOUT.
+ * Returns SA_ERR_INVALID_ARG for a null or misaligned `ws`, SA_ERR_CUDA on a
+ * launch error, else SA_OK. */
+sa_status sinkhorn_attn_debug_timeout(void* ws, long long budget_cycles, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

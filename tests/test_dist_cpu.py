@@ -1,0 +1,112 @@
+"""The multi-process path of bench.py on CPU: two gloo ranks run the same
+setup, barrier and max-over-ranks code that the GPU runs use with NCCL, and a
+rank that fails before a collective makes the other rank's collective end with
+an error (short process-group timeout) instead of hanging."""
+from __future__ import annotations
+
+import multiprocessing as mp
+import os
+import socket
+import time
+
+import pytest
+
+import bench
+
+
+def _free_port() -> int:
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _env(rank, ws, port):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), WORLD_SIZE=str(ws),
+                      RANK=str(rank), LOCAL_RANK=str(rank))
+
+
+def _worker_max(rank, ws, port, q):
+    _env(rank, ws, port)
+    import torch.distributed as dist
+
+    try:
+        w, r, local = bench.dist_setup(backend="gloo", timeout_s=30)
+        bench.barrier(w)
+        step_ms = 10.0 + 5.0 * r  # rank 1 is the slower one
+        slowest = bench.allreduce_max(step_ms, w)
+        value = bench.whole_job_value(w, 1000.0, slowest)
+        bench.barrier(w)
+        q.put((r, w, local, slowest, value))
+    finally:
+        if dist.is_initialized():
+            dist.destroy_process_group()
+
+
+def _worker_fail(rank, ws, port, q):
+    _env(rank, ws, port)
+    import torch.distributed as dist
+
+    w, r, _ = bench.dist_setup(backend="gloo", timeout_s=5)
+    bench.barrier(w)
+    if r == 1:
+        os._exit(3)  # leaves between steps, with no collective in flight
+    t0 = time.time()
+    try:
+        bench.allreduce_max(1.0, w)
+        q.put(("no error", time.time() - t0))
+    except Exception as e:  # noqa: BLE001 - any backend error is the expected outcome
+        q.put((type(e).__name__, time.time() - t0))
+    finally:
+        try:
+            dist.destroy_process_group()
+        except Exception:  # noqa: BLE001
+            pass
+
+
+def _run(target, ws=2, join_s=90):
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    ps = [ctx.Process(target=target, args=(r, ws, port, q)) for r in range(ws)]
+    for p in ps:
+        p.start()
+    for p in ps:
+        p.join(join_s)
+    for p in ps:
+        if p.is_alive():
+            p.kill()
+            pytest.fail("a rank did not finish")
+    out = []
+    while not q.empty():
+        out.append(q.get())
+    return ps, out
+
+
+def test_two_ranks_max_over_ranks_and_whole_job_value():
+    ps, out = _run(_worker_max)
+    assert all(p.exitcode == 0 for p in ps)
+    assert sorted(o[0] for o in out) == [0, 1]
+    for r, w, local, slowest, value in out:
+        assert w == 2 and local == r
+        assert slowest == 15.0  # the max over ranks, seen by every rank
+        assert value == pytest.approx(2 * 1000.0 / 0.015)
+
+
+def test_failed_rank_ends_the_others_collective_with_an_error():
+    ps, out = _run(_worker_fail)
+    assert ps[1].exitcode == 3
+    assert len(out) == 1
+    name, dt = out[0]
+    assert name != "no error"
+    assert dt < 60.0
+
+
+def test_reference_arm_prints_on_rank_zero_only(capsys, monkeypatch):
+    monkeypatch.setenv("RANK", "1")
+    monkeypatch.setenv("WORLD_SIZE", "2")
+
+    class A:
+        schedule, steps, warmup = "one_reference", 1, 0
+
+    bench.run_reference(A(), bench.workloads.WORKLOADS["small512"])
+    assert capsys.readouterr().out == ""
