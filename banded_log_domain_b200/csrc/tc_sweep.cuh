@@ -197,28 +197,55 @@ __global__ void __launch_bounds__(NTHREADS, (MODE == LSE || MODE == WSUM) ? 2 : 
                 if (DS) tc::tma_load_3d(st + TILE, &maps.B2, bar + B_FULL + s, 0, c0, bh);
                 if (MODE == PV) tc::tma_load_3d(st + TILE, &maps.X, bar + B_FULL + s, 0, c0, bh);
             }
-            // column vectors: -inf / 0 outside [cbeg, cend) and on masked columns
-            for (int t = lane; t < 128; t += 32) {
-                const int col = c0 + t;
-                const bool ok = col < cend && (mk == nullptr || mk[col] != 0);
-                colvec(sm, MODE, s, 0)[t] =
-                    (MODE == DSD) ? 0.f : (ok ? a.cd.at(bh, col) * kLog2e : -INFINITY);
-                if (MODE == WSUM) colvec(sm, MODE, s, 1)[t] = ok ? a.w.at(bh, col) : 0.f;
-                if (MODE == DS1) {
+            // column vectors: -inf / 0 outside [cbeg, cend) and on masked columns.
+            // Every load of the chunk (4 columns per lane, each vector, the mask)
+            // is issued before any value is used or stored.
+            {
+                constexpr int NV = MODE == WSUM ? 2 : (MODE == DS1 ? 1 + NT : (MODE == DSD ? 2 * NT : 1));
+                float val[4][NV > 0 ? NV : 1];
+                bool inr[4], mok[4];
 #pragma unroll
-                    for (int k = 0; k < NT; ++k)
-                        colvec(sm, MODE, s, 1 + k)[t] =
-                            ok ? (a.cv[k].p ? a.cv[k].at(bh, col) : 1.f) : 0.f;
-                }
-                if (MODE == DSD) {
+                for (int k = 0; k < 4; ++k) {
+                    const int col = c0 + 32 * k + lane;
+                    inr[k] = col < cend;
+                    mok[k] = true;
 #pragma unroll
-                    for (int k = 0; k < NT; ++k)
-                        {
-                            colvec(sm, MODE, s, k)[t] =
-                                ok ? a.ec[k].at(bh, col) * kLog2e : -INFINITY;
-                            colvec(sm, MODE, s, MAXT + k)[t] =
-                                (ok && a.cc[k].p) ? a.cc[k].at(bh, col) : 0.f;
+                    for (int e = 0; e < NV; ++e) val[k][e] = 0.f;
+                    if (inr[k]) {
+                        if (mk) mok[k] = mk[col] != 0;
+                        if (MODE != DSD) val[k][0] = a.cd.at(bh, col);
+                        if (MODE == WSUM) val[k][1] = a.w.at(bh, col);
+                        if (MODE == DS1) {
+#pragma unroll
+                            for (int e = 0; e < NT; ++e) val[k][1 + e] = a.cv[e].p ? a.cv[e].at(bh, col) : 1.f;
                         }
+                        if (MODE == DSD) {
+#pragma unroll
+                            for (int e = 0; e < NT; ++e) {
+                                val[k][e] = a.ec[e].at(bh, col);
+                                val[k][NT + e] = a.cc[e].p ? a.cc[e].at(bh, col) : 0.f;
+                            }
+                        }
+                    }
+                }
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const int t = 32 * k + lane;
+                    const bool ok = inr[k] && mok[k];
+                    colvec(sm, MODE, s, 0)[t] =
+                        (MODE == DSD) ? 0.f : (ok ? val[k][0] * kLog2e : -INFINITY);
+                    if (MODE == WSUM) colvec(sm, MODE, s, 1)[t] = ok ? val[k][1] : 0.f;
+                    if (MODE == DS1) {
+#pragma unroll
+                        for (int e = 0; e < NT; ++e) colvec(sm, MODE, s, 1 + e)[t] = ok ? val[k][1 + e] : 0.f;
+                    }
+                    if (MODE == DSD) {
+#pragma unroll
+                        for (int e = 0; e < NT; ++e) {
+                            colvec(sm, MODE, s, e)[t] = ok ? val[k][e] * kLog2e : -INFINITY;
+                            colvec(sm, MODE, s, MAXT + e)[t] = ok ? val[k][NT + e] : 0.f;
+                        }
+                    }
                 }
             }
             tc::mbar_arrive(bar + B_FULL + s);
