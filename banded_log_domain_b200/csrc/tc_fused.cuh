@@ -192,6 +192,63 @@ __device__ __forceinline__ void group_exp(uint32_t (&u)[32], const float* cvp, f
     }
 }
 
+// One warp forms 128 column duals of chunk `cb` of the tile at row block r0 of
+// problem bh into `cv` (v * log2(e) on valid columns, -inf outside [0, L) and on
+// masked columns; entries of a chunk outside the tile's band are masked by the
+// epilogue, so a column's value does not depend on the tile), and with
+// `do_rows` the tile's 128 row duals into `rows` (log2 units, -inf on rows past
+// L or masked).  Every load is issued before any value is used.  v_{k-1} of a
+// column is written to v_out by the CTA whose range [t0, t1) holds the column's
+// own row block.
+__device__ __forceinline__ void dual_batch(const FusedArgs& a, int bh, int r0, const uint8_t* mk_,
+                                           int cb, bool do_cols, bool do_rows, float* cv, float* rows,
+                                           int t0, int t1, int lane) {
+    const int L = a.L, W = a.W;
+    float4 p0[4], p1[4];
+    float vs[4], ur[4];
+    bool inr[4], mok[4], rin[4], rmk[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const int cc = cb * 128 + 32 * k + lane, col = r0 - W + cc;
+        inr[k] = do_cols && col >= 0 && col < L;
+        mok[k] = true;
+        vs[k] = 0.f;
+        p0[k] = p1[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (inr[k]) {
+            if (mk_) mok[k] = mk_[col] != 0;
+            vs[k] = a.v_src.at(bh, col);
+            if (a.part_in) {
+                const float4* pp = reinterpret_cast<const float4*>(a.part_in + ((size_t)bh * L + col) * NSLOT);
+                p0[k] = pp[0];
+                p1[k] = pp[1];
+            }
+        }
+        const int r = r0 + 32 * k + lane;
+        rin[k] = do_rows && r < L;
+        rmk[k] = true;
+        ur[k] = 0.f;
+        if (rin[k]) {
+            if (mk_) rmk[k] = mk_[r] != 0;
+            ur[k] = a.u_prev.at(bh, r);
+        }
+    }
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        if (do_cols) {
+            const int cc = cb * 128 + 32 * k + lane, col = r0 - W + cc;
+            const bool valid = inr[k] && mok[k];
+            float v = vs[k];
+            if (a.part_in) v -= lg2(partial_sum(a, col, p0[k], p1[k])) * kLn2;
+            if (a.part_in && a.v_out.p && inr[k]) {
+                const int owner = bh * a.nblk + col / 128;
+                if (owner >= t0 && owner < t1) a.v_out.at(bh, col) = valid ? v : 0.f;
+            }
+            cv[32 * k + lane] = valid ? v * kLog2e : -INFINITY;
+        }
+        if (do_rows) rows[32 * k + lane] = (rin[k] && rmk[k]) ? ur[k] * kLog2e : -INFINITY;
+    }
+}
+
 __global__ void __launch_bounds__(NTHREADS, 1) tc_fused_iter(const FusedArgs a,
                                                             const __grid_constant__ CUtensorMap mq,
                                                             const __grid_constant__ CUtensorMap mk) {
@@ -251,12 +308,18 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fused_iter(const FusedArgs a,
     // (even K steps) and 256 + 32c + 16 (odd K steps)
     const uint32_t tS = tm, tD = tm + 256;
 
+    // the first tile's duals (all its chunks at once), by warps 0..nch-1 and
+    // the last epilogue warp for the rows; ring slots 0..nch-1
+    if (ntl >= 1 && (warp < nch || warp == NEPI - 1)) {
+        const int bh = t0 / nblk, r0 = (t0 % nblk) * 128;
+        const uint8_t* mk_ = a.mask ? a.mask + (size_t)(bh / a.H) * L : nullptr;
+        dual_batch(a, bh, r0, mk_, warp, warp < nch, warp == NEPI - 1, cvring + warp * 128,
+                   rowring, t0, t1, lane);
+    }
+    __syncthreads();
+
     if (warp == W_CV) {
         // ------------------------------------------------------------ column and row duals
-        // A column's value does not depend on the tile: v * log2(e) on valid
-        // columns, -inf outside [0, L) and on masked columns (entries of the
-        // chunk outside the tile's band are masked by the epilogue).
-        const int ln = lane;
         ChunkIds ids;
         for (int it = 0; it < ntl; ++it) {
             const int t = t0 + it, bh = t / nblk, rb = t % nblk, r0 = rb * 128;
@@ -267,55 +330,11 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fused_iter(const FusedArgs a,
             // used.  The tile's row duals (log2 units, -inf on rows past L or
             // masked) come with the first batch; a tile's rows are written only
             // at the end of that tile.
-            for (int cb = first; cb < nch; ++cb) {
-                float4 p0[4], p1[4];
-                float vs[4], ur[4];
-                bool inr[4], mok[4], rin[4], rmk[4];
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const int cc = cb * 128 + 32 * k + lane, col = r0 - W + cc;
-                    inr[k] = col >= 0 && col < L;
-                    mok[k] = true;
-                    vs[k] = 0.f;
-                    p0[k] = p1[k] = make_float4(0.f, 0.f, 0.f, 0.f);
-                    if (inr[k]) {
-                        if (mk_) mok[k] = mk_[col] != 0;
-                        vs[k] = a.v_src.at(bh, col);
-                        if (a.part_in) {
-                            const float4* pp = reinterpret_cast<const float4*>(
-                                a.part_in + ((size_t)bh * L + col) * NSLOT);
-                            p0[k] = pp[0];
-                            p1[k] = pp[1];
-                        }
-                    }
-                    const int r = r0 + 32 * k + lane;
-                    rin[k] = cb == first && r < L;
-                    rmk[k] = true;
-                    ur[k] = 0.f;
-                    if (rin[k]) {
-                        if (mk_) rmk[k] = mk_[r] != 0;
-                        ur[k] = a.u_prev.at(bh, r);
-                    }
-                }
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const int cc = cb * 128 + 32 * k + lane, col = r0 - W + cc;
-                    const bool valid = inr[k] && mok[k];
-                    float v = vs[k];
-                    if (a.part_in) v -= lg2(partial_sum(a, col, p0[k], p1[k])) * kLn2;
-                    // v_{k-1} of a column is written by the CTA whose range holds
-                    // the column's own row block
-                    if (a.part_in && a.v_out.p && inr[k]) {
-                        const int owner = bh * nblk + col / 128;
-                        if (owner >= t0 && owner < t1) a.v_out.at(bh, col) = valid ? v : 0.f;
-                    }
-                    cvring[((ids.base + cb) % NCVS) * 128 + 32 * k + lane] =
-                        valid ? v * kLog2e : -INFINITY;
-                    if (cb == first)
-                        rowring[(it & 1) * 128 + 32 * k + lane] =
-                            (rin[k] && rmk[k]) ? ur[k] * kLog2e : -INFINITY;
-                }
-            }
+            if (it >= 1)  // tile 0's duals were formed by every warp before the roles split
+                for (int cb = first; cb < nch; ++cb)
+                    dual_batch(a, bh, r0, mk_, cb, true, cb == first,
+                               cvring + ((ids.base + cb) % NCVS) * 128, rowring + (it & 1) * 128,
+                               t0, t1, lane);
             tc::mbar_arrive(bar + B_CVFULL + (it & 1));
         }
     } else if (warp == W_LOAD) {
