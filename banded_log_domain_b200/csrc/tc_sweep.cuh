@@ -46,7 +46,7 @@ struct Maps {
 
 __host__ __device__ constexpr bool is_ds(int m) { return m == DS1 || m == DSD; }
 __host__ __device__ constexpr bool has_x(int m) { return m == PV || is_ds(m); }
-__host__ __device__ constexpr int nst(int m) { return is_ds(m) ? 2 : (m == PV ? 3 : 4); }
+__host__ __device__ constexpr int nst(int m) { return is_ds(m) ? 3 : (m == PV ? 3 : 4); }
 __host__ __device__ constexpr int nsb(int m) { return is_ds(m) ? 1 : 2; }
 __host__ __device__ constexpr int ncv(int m) {
     return m == WSUM ? 2 : (m == DS1 ? 1 + MAXT : (m == DSD ? 2 * MAXT : 1));
@@ -351,26 +351,45 @@ __global__ void __launch_bounds__(NTHREADS, (MODE == LSE || MODE == WSUM) ? 2 : 
             tc::tc_fence_after();
             const int c0 = cbeg + 128 * c;
             const float* cvs = colvec(sm, MODE, s, 0) + 64 * hf;
+            // Modes with a matrix output (one CTA per SM, registers to spare) read all
+            // of this warp's scores of the chunk (and the dO V^T tile) with one wait
+            // and free the TMEM buffer at once; the others read a group at a time.
+            constexpr bool UPFRONT = MODE == PV;
+            uint32_t su[UPFRONT ? 2 : 1][32], gu[UPFRONT && DS ? 2 : 1][32];
+            if (UPFRONT) {
+#pragma unroll
+                for (int g = 0; g < 2; ++g) {
+                    tc::tmem_ld32(tS + 128 * b + lanebase + 64 * hf + 32 * g, su[UPFRONT ? g : 0]);
+                    if (DS) tc::tmem_ld32(tG + lanebase + 64 * hf + 32 * g, gu[UPFRONT && DS ? g : 0]);
+                }
+                tc::tmem_wait_ld();
+                tc::tc_fence_before();
+                __syncwarp();
+                if (lane == 0) tc::mbar_arrive(bar + B_SEMPTY + b);
+            }
 #pragma unroll 1
             for (int g = 0; g < 2; ++g) {
                 float sv[32], gv[DS ? 32 : 1], pv[32];
-                {
-                    uint32_t u[32];
-                    tc::tmem_ld32(tS + 128 * b + lanebase + 64 * hf + 32 * g, u);
+                if (UPFRONT) {
+                    // select, not index: the loop over g stays rolled and su in registers
+#pragma unroll
+                    for (int j = 0; j < 32; ++j)
+                        sv[j] = __uint_as_float(g ? su[UPFRONT ? 1 : 0][j] : su[0][j]);
+                } else {
+                    tc::tmem_ld32(tS + 128 * b + lanebase + 64 * hf + 32 * g, su[0]);
+                    if (DS) tc::tmem_ld32(tG + lanebase + 64 * hf + 32 * g, gu[0]);
                     tc::tmem_wait_ld();
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) sv[j] = __uint_as_float(u[j]);
+                    for (int j = 0; j < 32; ++j) sv[j] = __uint_as_float(su[0][j]);
                     if (DS) {
-                        tc::tmem_ld32(tG + lanebase + 64 * hf + 32 * g, u);
-                        tc::tmem_wait_ld();
 #pragma unroll
-                        for (int j = 0; j < 32; ++j) gv[j] = __uint_as_float(u[j]);
+                        for (int j = 0; j < 32; ++j) gv[j] = __uint_as_float(gu[0][j]);
                     }
-                }
-                if (g == 1) {  // every TMEM read of this chunk is done
-                    tc::tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) tc::mbar_arrive(bar + B_SEMPTY + b);
+                    if (g == 1) {  // every TMEM read of this chunk is done
+                        tc::tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) tc::mbar_arrive(bar + B_SEMPTY + b);
+                    }
                 }
                 // band test for this warp's 32 rows x these 32 columns (warp-uniform)
                 const int cg = c0 + 64 * hf + 32 * g;
