@@ -344,7 +344,7 @@ cudaError_t launch_tc(const simt::SweepArgs& a, int BH, cudaStream_t st, Tracer&
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     tr.begin(kind_of(MODE));
-    tcs::tc_band_sweep<MODE, ONLINE, NT><<<grid, tcs::NTHREADS, smem, st>>>(a, maps, status);
+    tcs::tc_band_sweep<MODE, ONLINE, NT><<<grid, tcs::nthreads(MODE), smem, st>>>(a, maps, status);
     tr.end();
     return cudaGetLastError();
 }

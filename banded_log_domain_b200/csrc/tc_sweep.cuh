@@ -36,7 +36,11 @@ using simt::SweepArgs;
 using simt::MAXT;
 constexpr int LSE = simt::LSE, WSUM = simt::WSUM, PV = simt::PV, DS1 = simt::DS1,
               DSD = simt::DSD;
-constexpr int NTHREADS = 320;
+// Epilogue warps: 16 for PV (one CTA per SM, each warp 32 columns of a chunk),
+// 8 for the others (each warp 64 columns; LSE and WSUM run two CTAs per SM, the
+// dS modes need the registers); then the loader warp and the MMA warp.
+__host__ __device__ constexpr int nepi(int m) { return m == simt::PV ? 16 : 8; }
+__host__ __device__ constexpr int nthreads(int m) { return (nepi(m) + 2) * 32; }
 constexpr int TILE = 16384;  // one 128 x 64 bf16 tile
 constexpr long long kWaitBudget = 4000000000LL;  // clock cycles (about 2 s)
 
@@ -124,13 +128,15 @@ __device__ __forceinline__ void group_args(const float (&sv)[32], const float* c
 // ---------------------------------------------------------------------------
 // NT: number of modifier (DS1) or staircase (DSD) terms, 2R; 0 for the other modes.
 template <int MODE, bool ONLINE, int NT>
-__global__ void __launch_bounds__(NTHREADS, (MODE == LSE || MODE == WSUM) ? 2 : 1) tc_band_sweep(const SweepArgs a,
+__global__ void __launch_bounds__(nthreads(MODE), (MODE == LSE || MODE == WSUM) ? 2 : 1) tc_band_sweep(const SweepArgs a,
                                                          const __grid_constant__ Maps maps,
                                                          int* status) {
     extern __shared__ uint8_t smraw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>(((uintptr_t)smraw + 1023) & ~(uintptr_t)1023);
     constexpr int NST = nst(MODE), NSB = nsb(MODE), NCV = ncv(MODE);
     constexpr bool DS = is_ds(MODE), HASX = has_x(MODE);
+    constexpr int NEPI = nepi(MODE), NPART = NEPI / 4, PW = 128 / NPART, NG = PW / 32;
+    constexpr int W_LOAD = NEPI, W_MMA = NEPI + 1;
     uint64_t* bar = reinterpret_cast<uint64_t*>(sm + off_bar(MODE));
     uint32_t* tbase = reinterpret_cast<uint32_t*>(sm + off_bar(MODE) + 64 * 8);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tbase + 1);
@@ -150,17 +156,17 @@ __global__ void __launch_bounds__(NTHREADS, (MODE == LSE || MODE == WSUM) ? 2 : 
         tc::mbar_init(bar + B_A, 1);
         for (int s = 0; s < NST; ++s) {
             tc::mbar_init(bar + B_FULL + s, 33);
-            tc::mbar_init(bar + B_EMPTY + s, 9);
+            tc::mbar_init(bar + B_EMPTY + s, NEPI + 1);
         }
         for (int b = 0; b < 2; ++b) {
             tc::mbar_init(bar + B_SFULL + b, 1);
-            tc::mbar_init(bar + B_SEMPTY + b, 8);
-            tc::mbar_init(bar + B_PFULL + b, 8);
+            tc::mbar_init(bar + B_SEMPTY + b, NEPI);
+            tc::mbar_init(bar + B_PFULL + b, NEPI);
             tc::mbar_init(bar + B_PEMPTY + b, 1);
         }
         tc::mbar_init(bar + B_OFULL, 1);
         tc::mbar_init(bar + B_DRAIN, 1);
-        tc::mbar_init(bar + B_EPI, 8);
+        tc::mbar_init(bar + B_EPI, NEPI);
         *abort_flag = 0;
         tc::fence_mbar_init();
     }
@@ -175,7 +181,7 @@ __global__ void __launch_bounds__(NTHREADS, (MODE == LSE || MODE == WSUM) ? 2 : 
     // TMEM columns: S buffer b at 128*b (DS: S at 0, G at 128); O at 256
     const uint32_t tS = tm, tG = tm + 128, tO = tm + 256;
 
-    if (warp == 8) {
+    if (warp == W_LOAD) {
         // ------------------------------------------------------------ loader
         if (lane == 0) {
             tc::prefetch_tmap(&maps.A);
@@ -257,7 +263,7 @@ __global__ void __launch_bounds__(NTHREADS, (MODE == LSE || MODE == WSUM) ? 2 : 
                 tc::mbar_wait(bar + B_FULL + c % NST, (c / NST) & 1, kWaitBudget);
         }
         __syncwarp();
-    } else if (warp == 9) {
+    } else if (warp == W_MMA) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             const uint32_t id_s = tc::idesc_bf16(128, 128, false, false);
@@ -313,7 +319,7 @@ __global__ void __launch_bounds__(NTHREADS, (MODE == LSE || MODE == WSUM) ? 2 : 
         __syncwarp();
     } else {
         // ------------------------------------------------------------ epilogue
-        const int qd = warp & 3, hf = warp >> 2;
+        const int qd = warp & 3, pt = warp >> 2;  // part pt: columns PW*pt..PW*pt+PW-1 of a chunk
         const int lr = qd * 32 + lane;          // local row
         const int r = r0 + lr;                  // global row
         const bool rok = r < L && (mk == nullptr || mk[r] != 0);
@@ -350,17 +356,17 @@ __global__ void __launch_bounds__(NTHREADS, (MODE == LSE || MODE == WSUM) ? 2 : 
             if (HASX && c >= 2 && !ctl.wait(B_PEMPTY + pb, ((c >> 1) - 1) & 1)) break;
             tc::tc_fence_after();
             const int c0 = cbeg + 128 * c;
-            const float* cvs = colvec(sm, MODE, s, 0) + 64 * hf;
+            const float* cvs = colvec(sm, MODE, s, 0) + PW * pt;
             // Modes with a matrix output (one CTA per SM, registers to spare) read all
             // of this warp's scores of the chunk (and the dO V^T tile) with one wait
             // and free the TMEM buffer at once; the others read a group at a time.
             constexpr bool UPFRONT = MODE == PV;
-            uint32_t su[UPFRONT ? 2 : 1][32], gu[UPFRONT && DS ? 2 : 1][32];
+            uint32_t su[UPFRONT ? NG : 1][32], gu[UPFRONT && DS ? NG : 1][32];
             if (UPFRONT) {
 #pragma unroll
-                for (int g = 0; g < 2; ++g) {
-                    tc::tmem_ld32(tS + 128 * b + lanebase + 64 * hf + 32 * g, su[UPFRONT ? g : 0]);
-                    if (DS) tc::tmem_ld32(tG + lanebase + 64 * hf + 32 * g, gu[UPFRONT && DS ? g : 0]);
+                for (int g = 0; g < NG; ++g) {
+                    tc::tmem_ld32(tS + 128 * b + lanebase + PW * pt + 32 * g, su[UPFRONT ? g : 0]);
+                    if (DS) tc::tmem_ld32(tG + lanebase + PW * pt + 32 * g, gu[UPFRONT && DS ? g : 0]);
                 }
                 tc::tmem_wait_ld();
                 tc::tc_fence_before();
@@ -368,16 +374,16 @@ __global__ void __launch_bounds__(NTHREADS, (MODE == LSE || MODE == WSUM) ? 2 : 
                 if (lane == 0) tc::mbar_arrive(bar + B_SEMPTY + b);
             }
 #pragma unroll 1
-            for (int g = 0; g < 2; ++g) {
+            for (int g = 0; g < NG; ++g) {
                 float sv[32], gv[DS ? 32 : 1], pv[32];
                 if (UPFRONT) {
                     // select, not index: the loop over g stays rolled and su in registers
 #pragma unroll
                     for (int j = 0; j < 32; ++j)
-                        sv[j] = __uint_as_float(g ? su[UPFRONT ? 1 : 0][j] : su[0][j]);
+                        sv[j] = __uint_as_float(g ? su[(UPFRONT && NG > 1) ? 1 : 0][j] : su[0][j]);
                 } else {
-                    tc::tmem_ld32(tS + 128 * b + lanebase + 64 * hf + 32 * g, su[0]);
-                    if (DS) tc::tmem_ld32(tG + lanebase + 64 * hf + 32 * g, gu[0]);
+                    tc::tmem_ld32(tS + 128 * b + lanebase + PW * pt + 32 * g, su[0]);
+                    if (DS) tc::tmem_ld32(tG + lanebase + PW * pt + 32 * g, gu[0]);
                     tc::tmem_wait_ld();
 #pragma unroll
                     for (int j = 0; j < 32; ++j) sv[j] = __uint_as_float(su[0][j]);
@@ -385,14 +391,14 @@ __global__ void __launch_bounds__(NTHREADS, (MODE == LSE || MODE == WSUM) ? 2 : 
 #pragma unroll
                         for (int j = 0; j < 32; ++j) gv[j] = __uint_as_float(gu[0][j]);
                     }
-                    if (g == 1) {  // every TMEM read of this chunk is done
+                    if (g == NG - 1) {  // every TMEM read of this chunk is done
                         tc::tc_fence_before();
                         __syncwarp();
                         if (lane == 0) tc::mbar_arrive(bar + B_SEMPTY + b);
                     }
                 }
                 // band test for this warp's 32 rows x these 32 columns (warp-uniform)
-                const int cg = c0 + 64 * hf + 32 * g;
+                const int cg = c0 + PW * pt + 32 * g;
                 const bool all_in = (cg >= rw0 + 31 - W) && (cg + 31 <= rw0 + W);
                 const bool all_out = (cg + 31 < rw0 - W) || (cg > rw0 + 31 + W);
                 const float* ce = cvs + 32 * g;
@@ -424,7 +430,7 @@ __global__ void __launch_bounds__(NTHREADS, (MODE == LSE || MODE == WSUM) ? 2 : 
                                                        tc::pk2(ex2(x[2 * q]), ex2(x[2 * q + 1])));
                         } else if (MODE == WSUM) {
                             const float4* w4 = reinterpret_cast<const float4*>(
-                                colvec(sm, MODE, s, 1) + 64 * hf + 32 * g);
+                                colvec(sm, MODE, s, 1) + PW * pt + 32 * g);
 #pragma unroll
                             for (int q = 0; q < 8; ++q) {
                                 const float4 wv = w4[q];
@@ -454,7 +460,7 @@ __global__ void __launch_bounds__(NTHREADS, (MODE == LSE || MODE == WSUM) ? 2 : 
 #pragma unroll
                         for (int k = 0; k < NT; ++k) {
                             const float4 cv = reinterpret_cast<const float4*>(
-                                colvec(sm, MODE, s, 1 + k) + 64 * hf + 32 * g)[q];
+                                colvec(sm, MODE, s, 1 + k) + PW * pt + 32 * g)[q];
                             const uint64_t rk = tc::pk2(rmod[k], rmod[k]);
                             m01 = tc::fma2(rk, tc::pk2(cv.x, cv.y), m01);
                             m23 = tc::fma2(rk, tc::pk2(cv.z, cv.w), m23);
@@ -476,9 +482,9 @@ __global__ void __launch_bounds__(NTHREADS, (MODE == LSE || MODE == WSUM) ? 2 : 
 #pragma unroll
                         for (int k = 0; k < NT; ++k) {
                             const float4 ev = reinterpret_cast<const float4*>(
-                                colvec(sm, MODE, s, k) + 64 * hf + 32 * g)[q];
+                                colvec(sm, MODE, s, k) + PW * pt + 32 * g)[q];
                             const float4 cv = reinterpret_cast<const float4*>(
-                                colvec(sm, MODE, s, MAXT + k) + 64 * hf + 32 * g)[q];
+                                colvec(sm, MODE, s, MAXT + k) + PW * pt + 32 * g)[q];
                             const uint64_t rk = tc::pk2(rmod[k], rmod[k]);
                             float x0, x1, x2, x3;
                             tc::upk2(tc::fma2(tc::pk2(sv[4 * q], sv[4 * q + 1]), c2p,
@@ -503,7 +509,8 @@ __global__ void __launch_bounds__(NTHREADS, (MODE == LSE || MODE == WSUM) ? 2 : 
                     }
                 }
                 if (HASX) {
-                    uint8_t* dst = Pb + pb * 2 * TILE + hf * TILE;
+                    const int jc = PW * pt + 32 * g;  // first column of the group within the chunk
+                    uint8_t* dst = Pb + pb * 2 * TILE + (jc >> 6) * TILE;
 #pragma unroll
                     for (int q = 0; q < 4; ++q) {
                         uint4 w;
@@ -511,7 +518,7 @@ __global__ void __launch_bounds__(NTHREADS, (MODE == LSE || MODE == WSUM) ? 2 : 
                         w.y = tc::pack_bf16(pv[8 * q + 2], pv[8 * q + 3]);
                         w.z = tc::pack_bf16(pv[8 * q + 4], pv[8 * q + 5]);
                         w.w = tc::pack_bf16(pv[8 * q + 6], pv[8 * q + 7]);
-                        *reinterpret_cast<uint4*>(dst + tc::sw128_off(lr, 4 * g + q)) = w;
+                        *reinterpret_cast<uint4*>(dst + tc::sw128_off(lr, ((jc & 63) >> 3) + q)) = w;
                     }
                 }
             }
@@ -537,11 +544,11 @@ __global__ void __launch_bounds__(NTHREADS, (MODE == LSE || MODE == WSUM) ? 2 : 
         if (MODE == LSE || MODE == WSUM) {
             // combine the two column halves of each row
             if (MODE == LSE && !ONLINE) m = 0.f;  // the sum is relative to the shift
-            red[hf * 256 + lr] = m;
-            red[hf * 256 + 128 + lr] = acc;
+            red[pt * 256 + lr] = m;
+            red[pt * 256 + 128 + lr] = acc;
             uint32_t eph = 0;
             const bool synced = ctl.epi_sync(eph);
-            if (synced && hf == 0 && r < L && !*abort_flag) {
+            if (synced && pt == 0 && r < L && !*abort_flag) {
                 float m1 = red[lr], s1 = red[128 + lr];
                 const float m2 = red[256 + lr], s2 = red[384 + lr];
                 float out = 0.f;
@@ -565,32 +572,34 @@ __global__ void __launch_bounds__(NTHREADS, (MODE == LSE || MODE == WSUM) ? 2 : 
                 a.out_vec.at(bh, r) = rok ? out : 0.f;
             }
         } else {
-            // O accumulator: this warp reads columns 32*hf..+31 of its lanes
+            // O accumulator: this warp reads columns OW*pt..OW*pt+OW-1 of its lanes
+            constexpr int OW = 64 / NPART;
             const bool okw = ctl.wait(B_OFULL, 0);
-            float o[32];
+            float o[OW];
             if (okw) {
                 tc::tc_fence_after();
-                uint32_t u0[32];
-                tc::tmem_ld32(tO + lanebase + 32 * hf, u0);
+                uint32_t u0[OW];
+                if constexpr (OW == 32) tc::tmem_ld32(tO + lanebase + OW * pt, u0);
+                else tc::tmem_ld16(tO + lanebase + OW * pt, u0);
                 tc::tmem_wait_ld();
 #pragma unroll
-                for (int j = 0; j < 32; ++j) o[j] = __uint_as_float(u0[j]);
+                for (int j = 0; j < OW; ++j) o[j] = __uint_as_float(u0[j]);
             }
             const float scale = DS ? a.out_scale : 1.f;
             if (MODE == PV && a.dustbin && a.Xd && rok) {
                 const float p = ex2(a.sd2 + rd2 + ce_d);
-                const float* xd = a.Xd + (size_t)(bh % a.H) * 64 + 32 * hf;
+                const float* xd = a.Xd + (size_t)(bh % a.H) * 64 + OW * pt;
 #pragma unroll
-                for (int j = 0; j < 32; ++j) o[j] = fmaf(p, xd[j], o[j]);
+                for (int j = 0; j < OW; ++j) o[j] = fmaf(p, xd[j], o[j]);
             }
 #pragma unroll
-            for (int j = 0; j < 32; ++j) o[j] = rok ? o[j] * scale : 0.f;
+            for (int j = 0; j < OW; ++j) o[j] = rok ? o[j] * scale : 0.f;
             float dot = 0.f;
             if (okw && r < L) {
                 __nv_bfloat16* outp =
-                    reinterpret_cast<__nv_bfloat16*>(a.out_mat) + ((size_t)bh * L + r) * 64 + 32 * hf;
+                    reinterpret_cast<__nv_bfloat16*>(a.out_mat) + ((size_t)bh * L + r) * 64 + OW * pt;
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
+                for (int q = 0; q < OW / 8; ++q) {
                     uint4 w;
                     w.x = tc::pack_bf16(o[8 * q + 0], o[8 * q + 1]);
                     w.y = tc::pack_bf16(o[8 * q + 2], o[8 * q + 3]);
@@ -600,17 +609,21 @@ __global__ void __launch_bounds__(NTHREADS, (MODE == LSE || MODE == WSUM) ? 2 : 
                 }
                 if (MODE == PV && a.Y) {
                     const __nv_bfloat16* yp = reinterpret_cast<const __nv_bfloat16*>(a.Y) +
-                                              ((size_t)bh * L + r) * 64 + 32 * hf;
+                                              ((size_t)bh * L + r) * 64 + OW * pt;
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) dot = fmaf(__bfloat162float(yp[j]), o[j], dot);
+                    for (int j = 0; j < OW; ++j) dot = fmaf(__bfloat162float(yp[j]), o[j], dot);
                 }
             }
             if (MODE == PV && a.Y) {
-                red[hf * 128 + lr] = dot;
+                red[pt * 128 + lr] = dot;
                 uint32_t eph = 0;
                 const bool synced = ctl.epi_sync(eph);
-                if (synced && hf == 0 && r < L && a.out_vec.p && !*abort_flag)
-                    a.out_vec.at(bh, r) = rok ? red[lr] + red[128 + lr] : 0.f;
+                if (synced && pt == 0 && r < L && a.out_vec.p && !*abort_flag) {
+                    float tot = 0.f;
+#pragma unroll
+                    for (int k = 0; k < NPART; ++k) tot += red[k * 128 + lr];
+                    a.out_vec.at(bh, r) = rok ? tot : 0.f;
+                }
             }
         }
     }
