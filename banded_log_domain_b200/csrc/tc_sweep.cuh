@@ -323,6 +323,20 @@ __global__ void __launch_bounds__(nthreads(MODE), (MODE == LSE || MODE == WSUM) 
         const int lr = qd * 32 + lane;          // local row
         const int r = r0 + lr;                  // global row
         const bool rok = r < L && (mk == nullptr || mk[r] != 0);
+        // PV with a row dot: this thread's slice of the Y row, loaded now so that
+        // the load's latency is hidden behind the chunk loop
+        constexpr int OWY = 64 / NPART;
+        uint4 yq[MODE == PV ? OWY / 8 : 1];
+        if (MODE == PV) {
+#pragma unroll
+            for (int q = 0; q < (MODE == PV ? OWY / 8 : 1); ++q) yq[q] = make_uint4(0, 0, 0, 0);
+            if (a.Y && r < L) {
+                const uint4* yp = reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(a.Y) +
+                                                                 ((size_t)bh * L + r) * 64 + OWY * pt);
+#pragma unroll
+                for (int q = 0; q < (MODE == PV ? OWY / 8 : 1); ++q) yq[q] = yp[q];
+            }
+        }
         const float c2 = a.c2;
         // row-side values
         float rd2 = 0.f;
@@ -608,10 +622,16 @@ __global__ void __launch_bounds__(nthreads(MODE), (MODE == LSE || MODE == WSUM) 
                     reinterpret_cast<uint4*>(outp)[q] = w;
                 }
                 if (MODE == PV && a.Y) {
-                    const __nv_bfloat16* yp = reinterpret_cast<const __nv_bfloat16*>(a.Y) +
-                                              ((size_t)bh * L + r) * 64 + OW * pt;
 #pragma unroll
-                    for (int j = 0; j < OW; ++j) dot = fmaf(__bfloat162float(yp[j]), o[j], dot);
+                    for (int q = 0; q < OW / 8; ++q) {
+                        const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&yq[MODE == PV ? q : 0]);
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float2 f = __bfloat1622float2(h[e]);
+                            dot = fmaf(f.x, o[8 * q + 2 * e], dot);
+                            dot = fmaf(f.y, o[8 * q + 2 * e + 1], dot);
+                        }
+                    }
                 }
             }
             if (MODE == PV && a.Y) {
