@@ -338,13 +338,22 @@ cudaError_t launch_tc(const simt::SweepArgs& a, int BH, cudaStream_t st, Tracer&
     if (tcs::is_ds(MODE)) ok = ok && make_map(&maps.A2, a.A2, a.L, BH) && make_map(&maps.B2, a.B2, a.L, BH);
     if (MODE == simt::PV) ok = ok && make_map(&maps.X, a.X, a.L, BH);
     if (!ok) return cudaErrorInvalidValue;
-    const dim3 grid((a.L + 127) / 128, BH);
+    // persistent: one CTA per SM (two for LSE and WSUM), each a contiguous tile range
+    static int nsm = 0;
+    if (nsm == 0) {
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || nsm <= 0)
+            nsm = 148;
+    }
+    const long long ntiles = (long long)((a.L + 127) / 128) * BH;
+    const dim3 grid((unsigned)std::min<long long>(ntiles, (long long)nsm * tcs::ctas_per_sm(MODE)));
     const int smem = tcs::smem_bytes(MODE);
     cudaError_t e = cudaFuncSetAttribute(tcs::tc_band_sweep<MODE, ONLINE, NT>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     tr.begin(kind_of(MODE));
-    tcs::tc_band_sweep<MODE, ONLINE, NT><<<grid, tcs::nthreads(MODE), smem, st>>>(a, maps, status);
+    tcs::tc_band_sweep<MODE, ONLINE, NT><<<grid, tcs::nthreads(MODE), smem, st>>>(a, maps, status, BH);
     tr.end();
     return cudaGetLastError();
 }

@@ -60,18 +60,26 @@ __host__ __device__ constexpr int stage_bytes(int m) {
 }
 __host__ __device__ constexpr int tmem_cols(int m) { return has_x(m) ? 512 : 256; }
 
+// row-block operand buffers: two (tile parity) of A for the modes without a second
+// score operand; one of A and A2 for the dS modes (their shared memory is full)
+__host__ __device__ constexpr int nab(int m) { return is_ds(m) ? 1 : 2; }
+// CTAs per SM (LSE and WSUM fit twice)
+__host__ __device__ constexpr int ctas_per_sm(int m) { return (m == LSE || m == WSUM) ? 2 : 1; }
+
 // shared-memory carve-up (offsets from a 1024-aligned base)
+__host__ __device__ constexpr int off_a(int m, int i) { return TILE * i; }
 __host__ __device__ constexpr int off_a2(int m) { return TILE; }
-__host__ __device__ constexpr int off_stage(int m) { return TILE * (is_ds(m) ? 2 : 1); }
+__host__ __device__ constexpr int off_stage(int m) { return 2 * TILE; }
 __host__ __device__ constexpr int off_p(int m) { return off_stage(m) + nst(m) * stage_bytes(m); }
 __host__ __device__ constexpr int off_cv(int m) { return off_p(m) + (has_x(m) ? 2 * 2 * TILE : 0); }
 __host__ __device__ constexpr int off_red(int m) { return off_cv(m) + nst(m) * ncv(m) * 128 * 4; }
-__host__ __device__ constexpr int off_bar(int m) { return off_red(m) + 4 * 128 * 4; }
+__host__ __device__ constexpr int off_bar(int m) { return off_red(m) + 2 * 4 * 128 * 4; }
 __host__ __device__ constexpr int smem_bytes(int m) { return off_bar(m) + 64 * 8 + 64 + 1024; }
 
-// barrier slots
-enum { B_A = 0, B_FULL = 1, B_EMPTY = 5, B_SFULL = 9, B_SEMPTY = 11, B_PFULL = 13, B_PEMPTY = 15,
-       B_OFULL = 17, B_DRAIN = 18, B_EPI = 19, NBAR = 20 };
+// barrier slots (pairs indexed by tile parity, chunk parity or buffer)
+enum { B_AFULL = 0, B_AEMPTY = 2, B_FULL = 4, B_EMPTY = 8, B_SFULL = 12, B_SEMPTY = 14,
+       B_PFULL = 16, B_PEMPTY = 18, B_OFULL = 20, B_OEMPTY = 22, B_DRAIN = 24, B_EPI = 25,
+       NBAR = 26 };
 
 struct Ctl {
     uint64_t* bar;
@@ -127,13 +135,18 @@ __device__ __forceinline__ void group_args(const float (&sv)[32], const float* c
 
 // ---------------------------------------------------------------------------
 // NT: number of modifier (DS1) or staircase (DSD) terms, 2R; 0 for the other modes.
+// Persistent: each CTA walks a contiguous range of (problem, row block) tiles;
+// the chunk pipelines (operand stages, score buffers, P buffers) run on one chunk
+// counter across tiles, the row-block operand is double-buffered by tile parity
+// (single for the dS modes), and the output accumulator of the PV-shaped modes
+// is double-buffered in TMEM, so one tile's setup overlaps the previous tile.
 template <int MODE, bool ONLINE, int NT>
-__global__ void __launch_bounds__(nthreads(MODE), (MODE == LSE || MODE == WSUM) ? 2 : 1) tc_band_sweep(const SweepArgs a,
+__global__ void __launch_bounds__(nthreads(MODE), ctas_per_sm(MODE)) tc_band_sweep(const SweepArgs a,
                                                          const __grid_constant__ Maps maps,
-                                                         int* status) {
+                                                         int* status, int BH) {
     extern __shared__ uint8_t smraw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>(((uintptr_t)smraw + 1023) & ~(uintptr_t)1023);
-    constexpr int NST = nst(MODE), NSB = nsb(MODE), NCV = ncv(MODE);
+    constexpr int NST = nst(MODE), NSB = nsb(MODE), NAB = nab(MODE);
     constexpr bool DS = is_ds(MODE), HASX = has_x(MODE);
     constexpr int NEPI = nepi(MODE), NPART = NEPI / 4, PW = 128 / NPART, NG = PW / 32;
     constexpr int W_LOAD = NEPI, W_MMA = NEPI + 1;
@@ -144,27 +157,45 @@ __global__ void __launch_bounds__(nthreads(MODE), (MODE == LSE || MODE == WSUM) 
     Ctl ctl{bar, abort_flag, status};
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int bh = blockIdx.y;
     const int L = a.L, W = a.W;
-    const int r0 = blockIdx.x * 128;
-    const int cbeg = max(0, r0 - W);
-    const int cend = min(L, r0 + 127 + W + 1);
-    const int nch = (cend - cbeg + 127) / 128;
-    const uint8_t* mk = a.mask ? a.mask + (size_t)(bh / a.H) * L : nullptr;
+    const int nblk = (L + 127) / 128;
+    // this CTA's contiguous tile range [t0, t1)
+    const int ntiles = BH * nblk;
+    const int t0 = (int)(((long long)blockIdx.x * ntiles) / gridDim.x);
+    const int t1 = (int)(((long long)(blockIdx.x + 1) * ntiles) / gridDim.x);
+    const int ntl = t1 - t0;
+    // geometry of tile it of the range
+    struct Tile {
+        int bh, r0, cbeg, cend, nch;
+        const uint8_t* mk;
+    };
+    auto tile = [&](int it) {
+        Tile g;
+        const int t = t0 + it;
+        g.bh = t / nblk;
+        g.r0 = (t % nblk) * 128;
+        g.cbeg = max(0, g.r0 - W);
+        g.cend = min(L, g.r0 + 127 + W + 1);
+        g.nch = (g.cend - g.cbeg + 127) / 128;
+        g.mk = a.mask ? a.mask + (size_t)(g.bh / a.H) * L : nullptr;
+        return g;
+    };
 
     if (threadIdx.x == 0) {
-        tc::mbar_init(bar + B_A, 1);
+        for (int i = 0; i < 2; ++i) {
+            tc::mbar_init(bar + B_AFULL + i, 1);
+            tc::mbar_init(bar + B_AEMPTY + i, 1);
+            tc::mbar_init(bar + B_SFULL + i, 1);
+            tc::mbar_init(bar + B_SEMPTY + i, NEPI);
+            tc::mbar_init(bar + B_PFULL + i, NEPI);
+            tc::mbar_init(bar + B_PEMPTY + i, 1);
+            tc::mbar_init(bar + B_OFULL + i, 1);
+            tc::mbar_init(bar + B_OEMPTY + i, NEPI);
+        }
         for (int s = 0; s < NST; ++s) {
             tc::mbar_init(bar + B_FULL + s, 33);
             tc::mbar_init(bar + B_EMPTY + s, NEPI + 1);
         }
-        for (int b = 0; b < 2; ++b) {
-            tc::mbar_init(bar + B_SFULL + b, 1);
-            tc::mbar_init(bar + B_SEMPTY + b, NEPI);
-            tc::mbar_init(bar + B_PFULL + b, NEPI);
-            tc::mbar_init(bar + B_PEMPTY + b, 1);
-        }
-        tc::mbar_init(bar + B_OFULL, 1);
         tc::mbar_init(bar + B_DRAIN, 1);
         tc::mbar_init(bar + B_EPI, NEPI);
         *abort_flag = 0;
@@ -178,7 +209,7 @@ __global__ void __launch_bounds__(nthreads(MODE), (MODE == LSE || MODE == WSUM) 
     __syncthreads();
     tc::tc_fence_after();
     const uint32_t tm = *tbase;
-    // TMEM columns: S buffer b at 128*b (DS: S at 0, G at 128); O at 256
+    // TMEM columns: S buffer b at 128*b (DS: S at 0, G at 128); O buffer ob at 256 + 64*ob
     const uint32_t tS = tm, tG = tm + 128, tO = tm + 256;
 
     if (warp == W_LOAD) {
@@ -186,81 +217,95 @@ __global__ void __launch_bounds__(nthreads(MODE), (MODE == LSE || MODE == WSUM) 
         if (lane == 0) {
             tc::prefetch_tmap(&maps.A);
             tc::prefetch_tmap(&maps.B);
-            tc::mbar_expect_tx(bar + B_A, TILE * (DS ? 2 : 1));
-            tc::tma_load_3d(sm, &maps.A, bar + B_A, 0, r0, bh);
-            if (DS) tc::tma_load_3d(sm + off_a2(MODE), &maps.A2, bar + B_A, 0, r0, bh);
         }
-        int issued = 0;
-        for (int c = 0; c < nch; ++c) {
-            const int s = c % NST;
-            if (c >= NST && !ctl.wait(B_EMPTY + s, ((c / NST) - 1) & 1)) break;
-            issued = c + 1;
-            const int c0 = cbeg + 128 * c;
-            uint8_t* st = sm + off_stage(MODE) + s * stage_bytes(MODE);
+        int gc = 0, issued = 0, a_issued = 0;
+        bool ok = true;
+        for (int it = 0; ok && it < ntl; ++it) {
+            const Tile tl = tile(it);
+            const int ab = it % NAB;
             if (lane == 0) {
-                tc::mbar_expect_tx(bar + B_FULL + s, stage_bytes(MODE));
-                tc::tma_load_3d(st, &maps.B, bar + B_FULL + s, 0, c0, bh);
-                if (DS) tc::tma_load_3d(st + TILE, &maps.B2, bar + B_FULL + s, 0, c0, bh);
-                if (MODE == PV) tc::tma_load_3d(st + TILE, &maps.X, bar + B_FULL + s, 0, c0, bh);
+                if (it >= NAB && !ctl.wait(B_AEMPTY + ab, ((it / NAB) - 1) & 1)) ok = false;
+                if (ok) {
+                    tc::mbar_expect_tx(bar + B_AFULL + ab, TILE * (DS ? 2 : 1));
+                    tc::tma_load_3d(sm + off_a(MODE, ab), &maps.A, bar + B_AFULL + ab, 0, tl.r0, tl.bh);
+                    if (DS) tc::tma_load_3d(sm + off_a2(MODE), &maps.A2, bar + B_AFULL + ab, 0, tl.r0, tl.bh);
+                    a_issued = it + 1;
+                }
             }
-            // column vectors: -inf / 0 outside [cbeg, cend) and on masked columns.
-            // Every load of the chunk (4 columns per lane, each vector, the mask)
-            // is issued before any value is used or stored.
-            {
-                constexpr int NV = MODE == WSUM ? 2 : (MODE == DS1 ? 1 + NT : (MODE == DSD ? 2 * NT : 1));
-                float val[4][NV > 0 ? NV : 1];
-                bool inr[4], mok[4];
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const int col = c0 + 32 * k + lane;
-                    inr[k] = col < cend;
-                    mok[k] = true;
-#pragma unroll
-                    for (int e = 0; e < NV; ++e) val[k][e] = 0.f;
-                    if (inr[k]) {
-                        if (mk) mok[k] = mk[col] != 0;
-                        if (MODE != DSD) val[k][0] = a.cd.at(bh, col);
-                        if (MODE == WSUM) val[k][1] = a.w.at(bh, col);
+            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+            for (int c = 0; ok && c < tl.nch; ++c, ++gc) {
+                const int s = gc % NST;
+                if (gc >= NST && !ctl.wait(B_EMPTY + s, ((gc / NST) - 1) & 1)) { ok = false; break; }
+                issued = gc + 1;
+                const int c0 = tl.cbeg + 128 * c, cend = tl.cend, bh = tl.bh;
+                const uint8_t* mk = tl.mk;
+                uint8_t* st = sm + off_stage(MODE) + s * stage_bytes(MODE);
+                if (lane == 0) {
+                    tc::mbar_expect_tx(bar + B_FULL + s, stage_bytes(MODE));
+                    tc::tma_load_3d(st, &maps.B, bar + B_FULL + s, 0, c0, bh);
+                    if (DS) tc::tma_load_3d(st + TILE, &maps.B2, bar + B_FULL + s, 0, c0, bh);
+                    if (MODE == PV) tc::tma_load_3d(st + TILE, &maps.X, bar + B_FULL + s, 0, c0, bh);
+                }
+                // column vectors: -inf / 0 outside [cbeg, cend) and on masked columns.
+                // Every load of the chunk (4 columns per lane, each vector, the mask)
+                // is issued before any value is used or stored.
+                {
+                    constexpr int NV = MODE == WSUM ? 2 : (MODE == DS1 ? 1 + NT : (MODE == DSD ? 2 * NT : 1));
+                    float val[4][NV > 0 ? NV : 1];
+                    bool inr[4], mok[4];
+    #pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const int col = c0 + 32 * k + lane;
+                        inr[k] = col < cend;
+                        mok[k] = true;
+    #pragma unroll
+                        for (int e = 0; e < NV; ++e) val[k][e] = 0.f;
+                        if (inr[k]) {
+                            if (mk) mok[k] = mk[col] != 0;
+                            if (MODE != DSD) val[k][0] = a.cd.at(bh, col);
+                            if (MODE == WSUM) val[k][1] = a.w.at(bh, col);
+                            if (MODE == DS1) {
+    #pragma unroll
+                                for (int e = 0; e < NT; ++e) val[k][1 + e] = a.cv[e].p ? a.cv[e].at(bh, col) : 1.f;
+                            }
+                            if (MODE == DSD) {
+    #pragma unroll
+                                for (int e = 0; e < NT; ++e) {
+                                    val[k][e] = a.ec[e].at(bh, col);
+                                    val[k][NT + e] = a.cc[e].p ? a.cc[e].at(bh, col) : 0.f;
+                                }
+                            }
+                        }
+                    }
+    #pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const int t = 32 * k + lane;
+                        const bool ok = inr[k] && mok[k];
+                        colvec(sm, MODE, s, 0)[t] =
+                            (MODE == DSD) ? 0.f : (ok ? val[k][0] * kLog2e : -INFINITY);
+                        if (MODE == WSUM) colvec(sm, MODE, s, 1)[t] = ok ? val[k][1] : 0.f;
                         if (MODE == DS1) {
-#pragma unroll
-                            for (int e = 0; e < NT; ++e) val[k][1 + e] = a.cv[e].p ? a.cv[e].at(bh, col) : 1.f;
+    #pragma unroll
+                            for (int e = 0; e < NT; ++e) colvec(sm, MODE, s, 1 + e)[t] = ok ? val[k][1 + e] : 0.f;
                         }
                         if (MODE == DSD) {
-#pragma unroll
+    #pragma unroll
                             for (int e = 0; e < NT; ++e) {
-                                val[k][e] = a.ec[e].at(bh, col);
-                                val[k][NT + e] = a.cc[e].p ? a.cc[e].at(bh, col) : 0.f;
+                                colvec(sm, MODE, s, e)[t] = ok ? val[k][e] * kLog2e : -INFINITY;
+                                colvec(sm, MODE, s, MAXT + e)[t] = ok ? val[k][NT + e] : 0.f;
                             }
                         }
                     }
                 }
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const int t = 32 * k + lane;
-                    const bool ok = inr[k] && mok[k];
-                    colvec(sm, MODE, s, 0)[t] =
-                        (MODE == DSD) ? 0.f : (ok ? val[k][0] * kLog2e : -INFINITY);
-                    if (MODE == WSUM) colvec(sm, MODE, s, 1)[t] = ok ? val[k][1] : 0.f;
-                    if (MODE == DS1) {
-#pragma unroll
-                        for (int e = 0; e < NT; ++e) colvec(sm, MODE, s, 1 + e)[t] = ok ? val[k][1 + e] : 0.f;
-                    }
-                    if (MODE == DSD) {
-#pragma unroll
-                        for (int e = 0; e < NT; ++e) {
-                            colvec(sm, MODE, s, e)[t] = ok ? val[k][e] * kLog2e : -INFINITY;
-                            colvec(sm, MODE, s, MAXT + e)[t] = ok ? val[k][NT + e] : 0.f;
-                        }
-                    }
-                }
+                tc::mbar_arrive(bar + B_FULL + s);
             }
-            tc::mbar_arrive(bar + B_FULL + s);
         }
         // after an abort, let the tile loads already issued land before teardown
         if (lane == 0 && *abort_flag) {
-            tc::mbar_wait(bar + B_A, 0, kWaitBudget);
-            for (int c = max(0, issued - NST); c < issued; ++c)
-                tc::mbar_wait(bar + B_FULL + c % NST, (c / NST) & 1, kWaitBudget);
+            for (int x = max(0, a_issued - NAB); x < a_issued; ++x)
+                tc::mbar_wait(bar + B_AFULL + x % NAB, (x / NAB) & 1, kWaitBudget);
+            for (int x = max(0, issued - NST); x < issued; ++x)
+                tc::mbar_wait(bar + B_FULL + x % NST, (x / NST) & 1, kWaitBudget);
         }
         __syncwarp();
     } else if (warp == W_MMA) {
@@ -269,49 +314,65 @@ __global__ void __launch_bounds__(nthreads(MODE), (MODE == LSE || MODE == WSUM) 
             const uint32_t id_s = tc::idesc_bf16(128, 128, false, false);
             const uint32_t id_o = tc::idesc_bf16(128, 64, false, true);
             // descriptors built once; offsets are added in 16-byte units
-            const uint64_t dA = tc::sdesc_sw128(tc::smem_u32(sm), 16, 1024);
+            const uint64_t dA0 = tc::sdesc_sw128(tc::smem_u32(sm), 16, 1024);
             const uint64_t dA2 = tc::sdesc_sw128(tc::smem_u32(sm + off_a2(MODE)), 16, 1024);
             const uint64_t dStK = tc::sdesc_sw128(tc::smem_u32(sm + off_stage(MODE)), 16, 1024);
             const uint64_t dStMN = tc::sdesc_sw128(tc::smem_u32(sm + off_stage(MODE)), TILE, 1024);
             const uint64_t dP = tc::sdesc_sw128(tc::smem_u32(sm + off_p(MODE)), 16, 1024);
-            auto issue_pv = [&](int c) -> bool {
-                const int pb = c & 1, s = c % NST;
-                if (!ctl.wait(B_PFULL + pb, (c >> 1) & 1)) return false;
+            // O += P X of chunk c (global chunk g) of tile it (nch chunks)
+            auto issue_pv = [&](int g, int it, int c, int nch) -> bool {
+                const int pb = g & 1, s = g % NST, ob = it & 1;
+                // the epilogue has read this O buffer's previous tile (it - 2)
+                if (c == 0 && it >= 2 && !ctl.wait(B_OEMPTY + ob, ((it >> 1) - 1) & 1)) return false;
+                if (!ctl.wait(B_PFULL + pb, (g >> 1) & 1)) return false;
                 tc::tc_fence_after();
                 const uint64_t dX = tc::sdesc_add(dStMN, s * stage_bytes(MODE) + (MODE == PV ? TILE : 0));
                 const uint64_t dPb = tc::sdesc_add(dP, pb * 2 * TILE);
 #pragma unroll
                 for (int k = 0; k < 8; ++k) {
-                    tc::mma_bf16(tO, tc::sdesc_add(dPb, (k >> 2) * TILE + (k & 3) * 32),
+                    tc::mma_bf16(tO + 64 * ob, tc::sdesc_add(dPb, (k >> 2) * TILE + (k & 3) * 32),
                                  tc::sdesc_add(dX, k * 2048), id_o, (c > 0 || k > 0) ? 1u : 0u);
                 }
                 tc::tc_commit(bar + B_PEMPTY + pb);
                 tc::tc_commit(bar + B_EMPTY + s);
+                if (c == nch - 1) tc::tc_commit(bar + B_OFULL + ob);
                 return true;
             };
-            bool ok = ctl.wait(B_A, 0);
-            for (int c = 0; ok && c < nch; ++c) {
-                const int s = c % NST, b = c % NSB;
-                if (!ctl.wait(B_FULL + s, (c / NST) & 1)) { ok = false; break; }
-                if (c >= NSB && !ctl.wait(B_SEMPTY + b, ((c / NSB) - 1) & 1)) { ok = false; break; }
-                tc::tc_fence_after();
-                const uint64_t dB = tc::sdesc_add(dStK, s * stage_bytes(MODE));
-#pragma unroll
-                for (int k = 0; k < 4; ++k)
-                    tc::mma_bf16(tS + 128 * b, tc::sdesc_add(dA, 32 * k), tc::sdesc_add(dB, 32 * k),
-                                 id_s, k > 0);
-                if (DS) {
+            bool ok = true;
+            int gc = 0;
+            int pg = -1, pit = 0, pc = 0, pn = 0;  // the chunk whose P X is still to issue
+            for (int it = 0; ok && it < ntl; ++it) {
+                const Tile tl = tile(it);
+                const int ab = it % NAB;
+                if (!ctl.wait(B_AFULL + ab, (it / NAB) & 1)) { ok = false; break; }
+                const uint64_t dA = tc::sdesc_add(dA0, off_a(MODE, ab));
+                for (int c = 0; c < tl.nch; ++c, ++gc) {
+                    const int s = gc % NST, b = gc % NSB;
+                    if (!ctl.wait(B_FULL + s, (gc / NST) & 1)) { ok = false; break; }
+                    if (gc >= NSB && !ctl.wait(B_SEMPTY + b, ((gc / NSB) - 1) & 1)) { ok = false; break; }
+                    tc::tc_fence_after();
+                    const uint64_t dB = tc::sdesc_add(dStK, s * stage_bytes(MODE));
 #pragma unroll
                     for (int k = 0; k < 4; ++k)
-                        tc::mma_bf16(tG, tc::sdesc_add(dA2, 32 * k), tc::sdesc_add(dB, TILE + 32 * k),
+                        tc::mma_bf16(tS + 128 * b, tc::sdesc_add(dA, 32 * k), tc::sdesc_add(dB, 32 * k),
                                      id_s, k > 0);
+                    if (DS) {
+#pragma unroll
+                        for (int k = 0; k < 4; ++k)
+                            tc::mma_bf16(tG, tc::sdesc_add(dA2, 32 * k), tc::sdesc_add(dB, TILE + 32 * k),
+                                         id_s, k > 0);
+                    }
+                    tc::tc_commit(bar + B_SFULL + b);
+                    if (!HASX) tc::tc_commit(bar + B_EMPTY + s);
+                    if (HASX) {
+                        if (pg >= 0 && !issue_pv(pg, pit, pc, pn)) { ok = false; break; }
+                        pg = gc; pit = it; pc = c; pn = tl.nch;
+                    }
                 }
-                tc::tc_commit(bar + B_SFULL + b);
-                if (!HASX) tc::tc_commit(bar + B_EMPTY + s);
-                if (HASX && c >= 1 && !issue_pv(c - 1)) { ok = false; break; }
+                if (!ok) break;
+                tc::tc_commit(bar + B_AEMPTY + ab);  // every score MMA of the tile has read A
             }
-            if (HASX && ok && nch > 0) ok = issue_pv(nch - 1);
-            if (HASX) tc::tc_commit(bar + B_OFULL);
+            if (HASX && ok && pg >= 0) ok = issue_pv(pg, pit, pc, pn);
             // drain: every MMA issued above has completed once this arrives
             tc::tc_commit(bar + B_DRAIN);
             tc::mbar_wait(bar + B_DRAIN, 0, kWaitBudget);
@@ -320,329 +381,356 @@ __global__ void __launch_bounds__(nthreads(MODE), (MODE == LSE || MODE == WSUM) 
     } else {
         // ------------------------------------------------------------ epilogue
         const int qd = warp & 3, pt = warp >> 2;  // part pt: columns PW*pt..PW*pt+PW-1 of a chunk
-        const int lr = qd * 32 + lane;          // local row
-        const int r = r0 + lr;                  // global row
-        const bool rok = r < L && (mk == nullptr || mk[r] != 0);
-        // PV with a row dot: this thread's slice of the Y row, loaded now so that
-        // the load's latency is hidden behind the chunk loop
-        constexpr int OWY = 64 / NPART;
-        uint4 yq[MODE == PV ? OWY / 8 : 1];
-        if (MODE == PV) {
-#pragma unroll
-            for (int q = 0; q < (MODE == PV ? OWY / 8 : 1); ++q) yq[q] = make_uint4(0, 0, 0, 0);
-            if (a.Y && r < L) {
-                const uint4* yp = reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(a.Y) +
-                                                                 ((size_t)bh * L + r) * 64 + OWY * pt);
-#pragma unroll
-                for (int q = 0; q < (MODE == PV ? OWY / 8 : 1); ++q) yq[q] = yp[q];
-            }
-        }
-        const float c2 = a.c2;
-        // row-side values
-        float rd2 = 0.f;
-        if (r < L) {
-            if (MODE == LSE) rd2 = ONLINE ? 0.f : a.rd.at(bh, r) * kLog2e;
-            else if (MODE != DSD) rd2 = a.rd.at(bh, r) * kLog2e;
-        }
-        float rmod[NT > 0 ? NT : 1], rmod2[NT > 0 ? NT : 1];
-#pragma unroll
-        for (int k = 0; k < NT; ++k) {
-            rmod[k] = 0.f;
-            rmod2[k] = 0.f;
-            if (r < L) {
-                if (MODE == DS1) rmod[k] = a.rv[k].p ? a.rv[k].at(bh, r) : 1.f;
-                if (MODE == DSD) {
-                    rmod[k] = a.er[k].at(bh, r) * kLog2e;
-                    rmod2[k] = a.cr[k].p ? a.cr[k].at(bh, r) : 0.f;
-                }
-            }
-        }
-        float m = -INFINITY, acc = 0.f;   // LSE online max / running sum; WSUM sum
-        uint64_t accp[4] = {0, 0, 0, 0};  // packed partial sums (LSE with shift, WSUM)
-        const int rw0 = r0 + qd * 32;       // first row of this warp
+        const int lr = qd * 32 + lane;            // local row
         const uint32_t lanebase = (uint32_t)(qd * 32) << 16;
         uint8_t* Pb = sm + off_p(MODE);
-
-        for (int c = 0; c < nch; ++c) {
-            const int s = c % NST, b = c % NSB, pb = c & 1;
-            if (!ctl.wait(B_FULL + s, (c / NST) & 1)) break;
-            if (!ctl.wait(B_SFULL + b, (c / NSB) & 1)) break;
-            if (HASX && c >= 2 && !ctl.wait(B_PEMPTY + pb, ((c >> 1) - 1) & 1)) break;
-            tc::tc_fence_after();
-            const int c0 = cbeg + 128 * c;
-            const float* cvs = colvec(sm, MODE, s, 0) + PW * pt;
-            // Modes with a matrix output (one CTA per SM, registers to spare) read all
-            // of this warp's scores of the chunk (and the dO V^T tile) with one wait
-            // and free the TMEM buffer at once; the others read a group at a time.
-            constexpr bool UPFRONT = MODE == PV;
-            uint32_t su[UPFRONT ? NG : 1][32], gu[UPFRONT && DS ? NG : 1][32];
-            if (UPFRONT) {
-#pragma unroll
-                for (int g = 0; g < NG; ++g) {
-                    tc::tmem_ld32(tS + 128 * b + lanebase + PW * pt + 32 * g, su[UPFRONT ? g : 0]);
-                    if (DS) tc::tmem_ld32(tG + lanebase + PW * pt + 32 * g, gu[UPFRONT && DS ? g : 0]);
-                }
-                tc::tmem_wait_ld();
-                tc::tc_fence_before();
-                __syncwarp();
-                if (lane == 0) tc::mbar_arrive(bar + B_SEMPTY + b);
+        const float c2 = a.c2;
+        constexpr int OWY = 64 / NPART;
+        int gc = 0;
+        uint32_t eph = 0;
+        bool ok = true;
+        // Row-side values of the tile in progress; the next tile's are loaded as
+        // soon as the chunk loop of the current one no longer needs them.
+        float rd2 = 0.f;
+        bool rok = false;
+        float rmod[NT > 0 ? NT : 1], rmod2[NT > 0 ? NT : 1];
+        auto load_rows = [&](const Tile& tl) {
+            const int r = tl.r0 + lr;
+            rok = r < L && (tl.mk == nullptr || tl.mk[r] != 0);
+            rd2 = 0.f;
+            if (r < L) {
+                if (MODE == LSE) rd2 = ONLINE ? 0.f : a.rd.at(tl.bh, r) * kLog2e;
+                else if (MODE != DSD) rd2 = a.rd.at(tl.bh, r) * kLog2e;
             }
-#pragma unroll 1
-            for (int g = 0; g < NG; ++g) {
-                float sv[32], gv[DS ? 32 : 1], pv[32];
-                if (UPFRONT) {
-                    // select, not index: the loop over g stays rolled and su in registers
 #pragma unroll
-                    for (int j = 0; j < 32; ++j)
-                        sv[j] = __uint_as_float(g ? su[(UPFRONT && NG > 1) ? 1 : 0][j] : su[0][j]);
-                } else {
-                    tc::tmem_ld32(tS + 128 * b + lanebase + PW * pt + 32 * g, su[0]);
-                    if (DS) tc::tmem_ld32(tG + lanebase + PW * pt + 32 * g, gu[0]);
-                    tc::tmem_wait_ld();
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) sv[j] = __uint_as_float(su[0][j]);
-                    if (DS) {
-#pragma unroll
-                        for (int j = 0; j < 32; ++j) gv[j] = __uint_as_float(gu[0][j]);
-                    }
-                    if (g == NG - 1) {  // every TMEM read of this chunk is done
-                        tc::tc_fence_before();
-                        __syncwarp();
-                        if (lane == 0) tc::mbar_arrive(bar + B_SEMPTY + b);
+            for (int k = 0; k < NT; ++k) {
+                rmod[k] = 0.f;
+                rmod2[k] = 0.f;
+                if (r < L) {
+                    if (MODE == DS1) rmod[k] = a.rv[k].p ? a.rv[k].at(tl.bh, r) : 1.f;
+                    if (MODE == DSD) {
+                        rmod[k] = a.er[k].at(tl.bh, r) * kLog2e;
+                        rmod2[k] = a.cr[k].p ? a.cr[k].at(tl.bh, r) : 0.f;
                     }
                 }
-                // band test for this warp's 32 rows x these 32 columns (warp-uniform)
-                const int cg = c0 + PW * pt + 32 * g;
-                const bool all_in = (cg >= rw0 + 31 - W) && (cg + 31 <= rw0 + W);
-                const bool all_out = (cg + 31 < rw0 - W) || (cg > rw0 + 31 + W);
-                const float* ce = cvs + 32 * g;
-                if (MODE == LSE || MODE == WSUM || MODE == PV) {
-                    if (all_out) {
-                        if (MODE == PV) {
+            }
+        };
+        if (ntl >= 1) load_rows(tile(0));
+        for (int it = 0; ok && it < ntl; ++it) {
+            const Tile tl = tile(it);
+            const int bh = tl.bh, r0 = tl.r0, cbeg = tl.cbeg, nch = tl.nch;
+            const int r = r0 + lr;              // global row
+            const int rw0 = r0 + qd * 32;       // first row of this warp
+            // PV with a row dot: this thread's slice of the Y row; WSUM: the output's
+            // base and multiplier.  Loaded now, used after the chunk loop.
+            uint4 yq[MODE == PV ? OWY / 8 : 1];
+            float bb = 0.f, mu = 1.f;
+            if (MODE == PV) {
 #pragma unroll
-                            for (int j = 0; j < 32; ++j) pv[j] = 0.f;
-                        }
+                for (int q = 0; q < (MODE == PV ? OWY / 8 : 1); ++q) yq[q] = make_uint4(0, 0, 0, 0);
+                if (a.Y && r < L) {
+                    const uint4* yp = reinterpret_cast<const uint4*>(
+                        reinterpret_cast<const __nv_bfloat16*>(a.Y) + ((size_t)bh * L + r) * 64 + OWY * pt);
+#pragma unroll
+                    for (int q = 0; q < (MODE == PV ? OWY / 8 : 1); ++q) yq[q] = yp[q];
+                }
+            }
+            if (MODE == WSUM && r < L) {
+                bb = a.base.p ? a.base.at(bh, r) : 0.f;
+                mu = a.mult.p ? a.mult.at(bh, r) : 1.f;
+            }
+            float m = -INFINITY, acc = 0.f;   // LSE online max / running sum; WSUM sum
+            uint64_t accp[4] = {0, 0, 0, 0};  // packed partial sums (LSE with shift, WSUM)
+
+            for (int c = 0; c < nch; ++c, ++gc) {
+                const int s = gc % NST, b = gc % NSB, pb = gc & 1;
+                if (!ctl.wait(B_FULL + s, (gc / NST) & 1)) { ok = false; break; }
+                if (!ctl.wait(B_SFULL + b, (gc / NSB) & 1)) { ok = false; break; }
+                if (HASX && gc >= 2 && !ctl.wait(B_PEMPTY + pb, ((gc >> 1) - 1) & 1)) { ok = false; break; }
+                tc::tc_fence_after();
+                const int c0 = cbeg + 128 * c;
+                const float* cvs = colvec(sm, MODE, s, 0) + PW * pt;
+                // Modes with a matrix output (one CTA per SM, registers to spare) read all
+                // of this warp's scores of the chunk (and the dO V^T tile) with one wait
+                // and free the TMEM buffer at once; the others read a group at a time.
+                constexpr bool UPFRONT = MODE == PV;
+                uint32_t su[UPFRONT ? NG : 1][32], gu[UPFRONT && DS ? NG : 1][32];
+                if (UPFRONT) {
+    #pragma unroll
+                    for (int g = 0; g < NG; ++g) {
+                        tc::tmem_ld32(tS + 128 * b + lanebase + PW * pt + 32 * g, su[UPFRONT ? g : 0]);
+                        if (DS) tc::tmem_ld32(tG + lanebase + PW * pt + 32 * g, gu[UPFRONT && DS ? g : 0]);
+                    }
+                    tc::tmem_wait_ld();
+                    tc::tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) tc::mbar_arrive(bar + B_SEMPTY + b);
+                }
+    #pragma unroll 1
+                for (int g = 0; g < NG; ++g) {
+                    float sv[32], gv[DS ? 32 : 1], pv[32];
+                    if (UPFRONT) {
+                        // select, not index: the loop over g stays rolled and su in registers
+    #pragma unroll
+                        for (int j = 0; j < 32; ++j)
+                            sv[j] = __uint_as_float(g ? su[(UPFRONT && NG > 1) ? 1 : 0][j] : su[0][j]);
                     } else {
+                        tc::tmem_ld32(tS + 128 * b + lanebase + PW * pt + 32 * g, su[0]);
+                        if (DS) tc::tmem_ld32(tG + lanebase + PW * pt + 32 * g, gu[0]);
+                        tc::tmem_wait_ld();
+    #pragma unroll
+                        for (int j = 0; j < 32; ++j) sv[j] = __uint_as_float(su[0][j]);
+                        if (DS) {
+    #pragma unroll
+                            for (int j = 0; j < 32; ++j) gv[j] = __uint_as_float(gu[0][j]);
+                        }
+                        if (g == NG - 1) {  // every TMEM read of this chunk is done
+                            tc::tc_fence_before();
+                            __syncwarp();
+                            if (lane == 0) tc::mbar_arrive(bar + B_SEMPTY + b);
+                        }
+                    }
+                    // band test for this warp's 32 rows x these 32 columns (warp-uniform)
+                    const int cg = c0 + PW * pt + 32 * g;
+                    const bool all_in = (cg >= rw0 + 31 - W) && (cg + 31 <= rw0 + W);
+                    const bool all_out = (cg + 31 < rw0 - W) || (cg > rw0 + 31 + W);
+                    const float* ce = cvs + 32 * g;
+                    if (MODE == LSE || MODE == WSUM || MODE == PV) {
+                        if (all_out) {
+                            if (MODE == PV) {
+    #pragma unroll
+                                for (int j = 0; j < 32; ++j) pv[j] = 0.f;
+                            }
+                        } else {
+                            float x[32];
+                            group_args(sv, ce, rd2, c2, !all_in, r, cg, W, x);
+                            if (MODE == LSE && ONLINE) {
+                                float mloc = -INFINITY;
+    #pragma unroll
+                                for (int j = 0; j < 32; ++j) mloc = fmaxf(mloc, x[j]);
+                                if (mloc > m) {
+                                    acc *= ex2(m - mloc);
+                                    m = mloc;
+                                }
+                                if (m != -INFINITY) {
+    #pragma unroll
+                                    for (int j = 0; j < 32; ++j) acc += ex2(x[j] - m);
+                                }
+                            } else if (MODE == LSE) {
+    #pragma unroll
+                                for (int q = 0; q < 16; ++q)
+                                    accp[q & 3] = tc::add2(accp[q & 3],
+                                                           tc::pk2(ex2(x[2 * q]), ex2(x[2 * q + 1])));
+                            } else if (MODE == WSUM) {
+                                const float4* w4 = reinterpret_cast<const float4*>(
+                                    colvec(sm, MODE, s, 1) + PW * pt + 32 * g);
+    #pragma unroll
+                                for (int q = 0; q < 8; ++q) {
+                                    const float4 wv = w4[q];
+                                    accp[(2 * q) & 3] =
+                                        tc::fma2(tc::pk2(ex2(x[4 * q]), ex2(x[4 * q + 1])),
+                                                 tc::pk2(wv.x, wv.y), accp[(2 * q) & 3]);
+                                    accp[(2 * q + 1) & 3] =
+                                        tc::fma2(tc::pk2(ex2(x[4 * q + 2]), ex2(x[4 * q + 3])),
+                                                 tc::pk2(wv.z, wv.w), accp[(2 * q + 1) & 3]);
+                                }
+                            } else {  // PV
+    #pragma unroll
+                                for (int j = 0; j < 32; ++j) pv[j] = ex2(x[j]);
+                            }
+                        }
+                    } else if (all_out) {
+    #pragma unroll
+                        for (int j = 0; j < 32; ++j) pv[j] = 0.f;
+                    } else if (MODE == DS1) {
+                        // dS = P * M,  M = G + sum_k rv_k[row] cv_k[col]
                         float x[32];
                         group_args(sv, ce, rd2, c2, !all_in, r, cg, W, x);
-                        if (MODE == LSE && ONLINE) {
-                            float mloc = -INFINITY;
-#pragma unroll
-                            for (int j = 0; j < 32; ++j) mloc = fmaxf(mloc, x[j]);
-                            if (mloc > m) {
-                                acc *= ex2(m - mloc);
-                                m = mloc;
+    #pragma unroll
+                        for (int q = 0; q < 8; ++q) {
+                            uint64_t m01 = tc::pk2(gv[4 * q], gv[4 * q + 1]);
+                            uint64_t m23 = tc::pk2(gv[4 * q + 2], gv[4 * q + 3]);
+    #pragma unroll
+                            for (int k = 0; k < NT; ++k) {
+                                const float4 cv = reinterpret_cast<const float4*>(
+                                    colvec(sm, MODE, s, 1 + k) + PW * pt + 32 * g)[q];
+                                const uint64_t rk = tc::pk2(rmod[k], rmod[k]);
+                                m01 = tc::fma2(rk, tc::pk2(cv.x, cv.y), m01);
+                                m23 = tc::fma2(rk, tc::pk2(cv.z, cv.w), m23);
                             }
-                            if (m != -INFINITY) {
-#pragma unroll
-                                for (int j = 0; j < 32; ++j) acc += ex2(x[j] - m);
+                            float M0, M1, M2, M3;
+                            tc::upk2(m01, M0, M1);
+                            tc::upk2(m23, M2, M3);
+                            pv[4 * q] = ex2(x[4 * q]) * M0;
+                            pv[4 * q + 1] = ex2(x[4 * q + 1]) * M1;
+                            pv[4 * q + 2] = ex2(x[4 * q + 2]) * M2;
+                            pv[4 * q + 3] = ex2(x[4 * q + 3]) * M3;
+                        }
+                    } else {
+                        // DSD: dS = sum_k exp(S + er_k[row] + ec_k[col]) (g_k G + cr_k[row] + cc_k[col])
+                        const uint64_t c2p = tc::pk2(c2, c2);
+    #pragma unroll
+                        for (int q = 0; q < 8; ++q) {
+                            float v4[4] = {0.f, 0.f, 0.f, 0.f};
+    #pragma unroll
+                            for (int k = 0; k < NT; ++k) {
+                                const float4 ev = reinterpret_cast<const float4*>(
+                                    colvec(sm, MODE, s, k) + PW * pt + 32 * g)[q];
+                                const float4 cv = reinterpret_cast<const float4*>(
+                                    colvec(sm, MODE, s, MAXT + k) + PW * pt + 32 * g)[q];
+                                const uint64_t rk = tc::pk2(rmod[k], rmod[k]);
+                                float x0, x1, x2, x3;
+                                tc::upk2(tc::fma2(tc::pk2(sv[4 * q], sv[4 * q + 1]), c2p,
+                                                  tc::add2(tc::pk2(ev.x, ev.y), rk)), x0, x1);
+                                tc::upk2(tc::fma2(tc::pk2(sv[4 * q + 2], sv[4 * q + 3]), c2p,
+                                                  tc::add2(tc::pk2(ev.z, ev.w), rk)), x2, x3);
+                                const float gk = a.gk[k], ck = rmod2[k];
+                                v4[0] = fmaf(ex2(x0), fmaf(gk, gv[4 * q], ck + cv.x), v4[0]);
+                                v4[1] = fmaf(ex2(x1), fmaf(gk, gv[4 * q + 1], ck + cv.y), v4[1]);
+                                v4[2] = fmaf(ex2(x2), fmaf(gk, gv[4 * q + 2], ck + cv.z), v4[2]);
+                                v4[3] = fmaf(ex2(x3), fmaf(gk, gv[4 * q + 3], ck + cv.w), v4[3]);
                             }
-                        } else if (MODE == LSE) {
-#pragma unroll
-                            for (int q = 0; q < 16; ++q)
-                                accp[q & 3] = tc::add2(accp[q & 3],
-                                                       tc::pk2(ex2(x[2 * q]), ex2(x[2 * q + 1])));
-                        } else if (MODE == WSUM) {
-                            const float4* w4 = reinterpret_cast<const float4*>(
-                                colvec(sm, MODE, s, 1) + PW * pt + 32 * g);
-#pragma unroll
-                            for (int q = 0; q < 8; ++q) {
-                                const float4 wv = w4[q];
-                                accp[(2 * q) & 3] =
-                                    tc::fma2(tc::pk2(ex2(x[4 * q]), ex2(x[4 * q + 1])),
-                                             tc::pk2(wv.x, wv.y), accp[(2 * q) & 3]);
-                                accp[(2 * q + 1) & 3] =
-                                    tc::fma2(tc::pk2(ex2(x[4 * q + 2]), ex2(x[4 * q + 3])),
-                                             tc::pk2(wv.z, wv.w), accp[(2 * q + 1) & 3]);
+    #pragma unroll
+                            for (int e = 0; e < 4; ++e) pv[4 * q + e] = v4[e];
+                        }
+                        if (!all_in) {
+    #pragma unroll
+                            for (int j = 0; j < 32; ++j) {
+                                const int d = r - (cg + j);
+                                if ((unsigned)(d + W) > (unsigned)(2 * W)) pv[j] = 0.f;
                             }
-                        } else {  // PV
-#pragma unroll
-                            for (int j = 0; j < 32; ++j) pv[j] = ex2(x[j]);
                         }
                     }
-                } else if (all_out) {
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) pv[j] = 0.f;
-                } else if (MODE == DS1) {
-                    // dS = P * M,  M = G + sum_k rv_k[row] cv_k[col]
-                    float x[32];
-                    group_args(sv, ce, rd2, c2, !all_in, r, cg, W, x);
-#pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                        uint64_t m01 = tc::pk2(gv[4 * q], gv[4 * q + 1]);
-                        uint64_t m23 = tc::pk2(gv[4 * q + 2], gv[4 * q + 3]);
-#pragma unroll
-                        for (int k = 0; k < NT; ++k) {
-                            const float4 cv = reinterpret_cast<const float4*>(
-                                colvec(sm, MODE, s, 1 + k) + PW * pt + 32 * g)[q];
-                            const uint64_t rk = tc::pk2(rmod[k], rmod[k]);
-                            m01 = tc::fma2(rk, tc::pk2(cv.x, cv.y), m01);
-                            m23 = tc::fma2(rk, tc::pk2(cv.z, cv.w), m23);
-                        }
-                        float M0, M1, M2, M3;
-                        tc::upk2(m01, M0, M1);
-                        tc::upk2(m23, M2, M3);
-                        pv[4 * q] = ex2(x[4 * q]) * M0;
-                        pv[4 * q + 1] = ex2(x[4 * q + 1]) * M1;
-                        pv[4 * q + 2] = ex2(x[4 * q + 2]) * M2;
-                        pv[4 * q + 3] = ex2(x[4 * q + 3]) * M3;
-                    }
-                } else {
-                    // DSD: dS = sum_k exp(S + er_k[row] + ec_k[col]) (g_k G + cr_k[row] + cc_k[col])
-                    const uint64_t c2p = tc::pk2(c2, c2);
-#pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                        float v4[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-                        for (int k = 0; k < NT; ++k) {
-                            const float4 ev = reinterpret_cast<const float4*>(
-                                colvec(sm, MODE, s, k) + PW * pt + 32 * g)[q];
-                            const float4 cv = reinterpret_cast<const float4*>(
-                                colvec(sm, MODE, s, MAXT + k) + PW * pt + 32 * g)[q];
-                            const uint64_t rk = tc::pk2(rmod[k], rmod[k]);
-                            float x0, x1, x2, x3;
-                            tc::upk2(tc::fma2(tc::pk2(sv[4 * q], sv[4 * q + 1]), c2p,
-                                              tc::add2(tc::pk2(ev.x, ev.y), rk)), x0, x1);
-                            tc::upk2(tc::fma2(tc::pk2(sv[4 * q + 2], sv[4 * q + 3]), c2p,
-                                              tc::add2(tc::pk2(ev.z, ev.w), rk)), x2, x3);
-                            const float gk = a.gk[k], ck = rmod2[k];
-                            v4[0] = fmaf(ex2(x0), fmaf(gk, gv[4 * q], ck + cv.x), v4[0]);
-                            v4[1] = fmaf(ex2(x1), fmaf(gk, gv[4 * q + 1], ck + cv.y), v4[1]);
-                            v4[2] = fmaf(ex2(x2), fmaf(gk, gv[4 * q + 2], ck + cv.z), v4[2]);
-                            v4[3] = fmaf(ex2(x3), fmaf(gk, gv[4 * q + 3], ck + cv.w), v4[3]);
-                        }
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) pv[4 * q + e] = v4[e];
-                    }
-                    if (!all_in) {
-#pragma unroll
-                        for (int j = 0; j < 32; ++j) {
-                            const int d = r - (cg + j);
-                            if ((unsigned)(d + W) > (unsigned)(2 * W)) pv[j] = 0.f;
+                    if (HASX) {
+                        const int jc = PW * pt + 32 * g;  // first column of the group within the chunk
+                        uint8_t* dst = Pb + pb * 2 * TILE + (jc >> 6) * TILE;
+    #pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            uint4 w;
+                            w.x = tc::pack_bf16(pv[8 * q + 0], pv[8 * q + 1]);
+                            w.y = tc::pack_bf16(pv[8 * q + 2], pv[8 * q + 3]);
+                            w.z = tc::pack_bf16(pv[8 * q + 4], pv[8 * q + 5]);
+                            w.w = tc::pack_bf16(pv[8 * q + 6], pv[8 * q + 7]);
+                            *reinterpret_cast<uint4*>(dst + tc::sw128_off(lr, ((jc & 63) >> 3) + q)) = w;
                         }
                     }
                 }
                 if (HASX) {
-                    const int jc = PW * pt + 32 * g;  // first column of the group within the chunk
-                    uint8_t* dst = Pb + pb * 2 * TILE + (jc >> 6) * TILE;
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        uint4 w;
-                        w.x = tc::pack_bf16(pv[8 * q + 0], pv[8 * q + 1]);
-                        w.y = tc::pack_bf16(pv[8 * q + 2], pv[8 * q + 3]);
-                        w.z = tc::pack_bf16(pv[8 * q + 4], pv[8 * q + 5]);
-                        w.w = tc::pack_bf16(pv[8 * q + 6], pv[8 * q + 7]);
-                        *reinterpret_cast<uint4*>(dst + tc::sw128_off(lr, ((jc & 63) >> 3) + q)) = w;
-                    }
+                    tc::fence_async_smem();
+                    __syncwarp();
+                    if (lane == 0) tc::mbar_arrive(bar + B_PFULL + pb);
                 }
-            }
-            if (HASX) {
-                tc::fence_async_smem();
                 __syncwarp();
-                if (lane == 0) tc::mbar_arrive(bar + B_PFULL + pb);
+                if (lane == 0) tc::mbar_arrive(bar + B_EMPTY + s);
             }
-            __syncwarp();
-            if (lane == 0) tc::mbar_arrive(bar + B_EMPTY + s);
-        }
 
-        // ---------------------------------------------------------- finish
-        if ((MODE == LSE && !ONLINE) || MODE == WSUM) {
-            float a0, a1, a2, a3, a4, a5, a6, a7;
-            tc::upk2(accp[0], a0, a1);
-            tc::upk2(accp[1], a2, a3);
-            tc::upk2(accp[2], a4, a5);
-            tc::upk2(accp[3], a6, a7);
-            acc = ((a0 + a1) + (a2 + a3)) + ((a4 + a5) + (a6 + a7));
-        }
-        const float ce_d = a.dustbin ? a.cd.at(bh, L) * kLog2e : 0.f;
-        if (MODE == LSE || MODE == WSUM) {
-            // combine the two column halves of each row
-            if (MODE == LSE && !ONLINE) m = 0.f;  // the sum is relative to the shift
-            red[pt * 256 + lr] = m;
-            red[pt * 256 + 128 + lr] = acc;
-            uint32_t eph = 0;
-            const bool synced = ctl.epi_sync(eph);
-            if (synced && pt == 0 && r < L && !*abort_flag) {
-                float m1 = red[lr], s1 = red[128 + lr];
-                const float m2 = red[256 + lr], s2 = red[384 + lr];
-                float out = 0.f;
-                if (MODE == LSE) {
-                    if (ONLINE) {
-                        lse_merge(m1, s1, m2, s2);
-                        if (a.dustbin) lse_merge(m1, s1, a.sd2 + ce_d, 1.f);
-                        out = -(m1 + lg2(s1)) * kLn2;
+            if (!ok) break;
+            // what the finish still needs of this tile; then the next tile's rows
+            const float rd2f = rd2;
+            const bool rokf = rok;
+            if (it + 1 < ntl) load_rows(tile(it + 1));
+
+            // ---------------------------------------------------------- finish
+            if ((MODE == LSE && !ONLINE) || MODE == WSUM) {
+                float a0, a1, a2, a3, a4, a5, a6, a7;
+                tc::upk2(accp[0], a0, a1);
+                tc::upk2(accp[1], a2, a3);
+                tc::upk2(accp[2], a4, a5);
+                tc::upk2(accp[3], a6, a7);
+                acc = ((a0 + a1) + (a2 + a3)) + ((a4 + a5) + (a6 + a7));
+            }
+            const float ce_d = a.dustbin ? a.cd.at(bh, L) * kLog2e : 0.f;
+            float* rr = red + (it & 1) * 512;  // double-buffered by tile parity
+            if (MODE == LSE || MODE == WSUM) {
+                // combine the two column halves of each row
+                if (MODE == LSE && !ONLINE) m = 0.f;  // the sum is relative to the shift
+                rr[pt * 256 + lr] = m;
+                rr[pt * 256 + 128 + lr] = acc;
+                if (!ctl.epi_sync(eph)) { ok = false; break; }
+                if (pt == 0 && r < L && !*abort_flag) {
+                    float m1 = rr[lr], s1 = rr[128 + lr];
+                    const float m2 = rr[256 + lr], s2 = rr[384 + lr];
+                    float out = 0.f;
+                    if (MODE == LSE) {
+                        if (ONLINE) {
+                            lse_merge(m1, s1, m2, s2);
+                            if (a.dustbin) lse_merge(m1, s1, a.sd2 + ce_d, 1.f);
+                            out = -(m1 + lg2(s1)) * kLn2;
+                        } else {
+                            float tot = s1 + s2;
+                            if (a.dustbin) tot += ex2(a.sd2 + ce_d + rd2f);
+                            out = (rd2f - lg2(tot)) * kLn2;
+                        }
                     } else {
                         float tot = s1 + s2;
-                        if (a.dustbin) tot += ex2(a.sd2 + ce_d + rd2);
-                        out = (rd2 - lg2(tot)) * kLn2;
+                        if (a.dustbin) tot += ex2(a.sd2 + rd2f + ce_d) * a.w.at(bh, L);
+                        out = bb + a.sgn * mu * tot;
                     }
-                } else {
-                    float tot = s1 + s2;
-                    if (a.dustbin) tot += ex2(a.sd2 + rd2 + ce_d) * a.w.at(bh, L);
-                    const float bb = a.base.p ? a.base.at(bh, r) : 0.f;
-                    const float mu = a.mult.p ? a.mult.at(bh, r) : 1.f;
-                    out = bb + a.sgn * mu * tot;
+                    a.out_vec.at(bh, r) = rokf ? out : 0.f;
                 }
-                a.out_vec.at(bh, r) = rok ? out : 0.f;
-            }
-        } else {
-            // O accumulator: this warp reads columns OW*pt..OW*pt+OW-1 of its lanes
-            constexpr int OW = 64 / NPART;
-            const bool okw = ctl.wait(B_OFULL, 0);
-            float o[OW];
-            if (okw) {
-                tc::tc_fence_after();
-                uint32_t u0[OW];
-                if constexpr (OW == 32) tc::tmem_ld32(tO + lanebase + OW * pt, u0);
-                else tc::tmem_ld16(tO + lanebase + OW * pt, u0);
-                tc::tmem_wait_ld();
+            } else {
+                // O accumulator of this tile: this warp reads columns OW*pt..OW*pt+OW-1
+                // of its lanes, then frees the buffer for tile it + 2
+                constexpr int OW = 64 / NPART;
+                const int ob = it & 1;
+                if (!ctl.wait(B_OFULL + ob, (it >> 1) & 1)) { ok = false; break; }
+                float o[OW];
+                {
+                    tc::tc_fence_after();
+                    uint32_t u0[OW];
+                    if constexpr (OW == 32) tc::tmem_ld32(tO + 64 * ob + lanebase + OW * pt, u0);
+                    else tc::tmem_ld16(tO + 64 * ob + lanebase + OW * pt, u0);
+                    tc::tmem_wait_ld();
 #pragma unroll
-                for (int j = 0; j < OW; ++j) o[j] = __uint_as_float(u0[j]);
-            }
-            const float scale = DS ? a.out_scale : 1.f;
-            if (MODE == PV && a.dustbin && a.Xd && rok) {
-                const float p = ex2(a.sd2 + rd2 + ce_d);
-                const float* xd = a.Xd + (size_t)(bh % a.H) * 64 + OW * pt;
-#pragma unroll
-                for (int j = 0; j < OW; ++j) o[j] = fmaf(p, xd[j], o[j]);
-            }
-#pragma unroll
-            for (int j = 0; j < OW; ++j) o[j] = rok ? o[j] * scale : 0.f;
-            float dot = 0.f;
-            if (okw && r < L) {
-                __nv_bfloat16* outp =
-                    reinterpret_cast<__nv_bfloat16*>(a.out_mat) + ((size_t)bh * L + r) * 64 + OW * pt;
-#pragma unroll
-                for (int q = 0; q < OW / 8; ++q) {
-                    uint4 w;
-                    w.x = tc::pack_bf16(o[8 * q + 0], o[8 * q + 1]);
-                    w.y = tc::pack_bf16(o[8 * q + 2], o[8 * q + 3]);
-                    w.z = tc::pack_bf16(o[8 * q + 4], o[8 * q + 5]);
-                    w.w = tc::pack_bf16(o[8 * q + 6], o[8 * q + 7]);
-                    reinterpret_cast<uint4*>(outp)[q] = w;
+                    for (int j = 0; j < OW; ++j) o[j] = __uint_as_float(u0[j]);
+                    tc::tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) tc::mbar_arrive(bar + B_OEMPTY + ob);
                 }
-                if (MODE == PV && a.Y) {
+                const float scale = DS ? a.out_scale : 1.f;
+                if (MODE == PV && a.dustbin && a.Xd && rokf) {
+                    const float p = ex2(a.sd2 + rd2f + ce_d);
+                    const float* xd = a.Xd + (size_t)(bh % a.H) * 64 + OW * pt;
+#pragma unroll
+                    for (int j = 0; j < OW; ++j) o[j] = fmaf(p, xd[j], o[j]);
+                }
+#pragma unroll
+                for (int j = 0; j < OW; ++j) o[j] = rokf ? o[j] * scale : 0.f;
+                float dot = 0.f;
+                if (r < L) {
+                    __nv_bfloat16* outp =
+                        reinterpret_cast<__nv_bfloat16*>(a.out_mat) + ((size_t)bh * L + r) * 64 + OW * pt;
 #pragma unroll
                     for (int q = 0; q < OW / 8; ++q) {
-                        const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&yq[MODE == PV ? q : 0]);
+                        uint4 w;
+                        w.x = tc::pack_bf16(o[8 * q + 0], o[8 * q + 1]);
+                        w.y = tc::pack_bf16(o[8 * q + 2], o[8 * q + 3]);
+                        w.z = tc::pack_bf16(o[8 * q + 4], o[8 * q + 5]);
+                        w.w = tc::pack_bf16(o[8 * q + 6], o[8 * q + 7]);
+                        reinterpret_cast<uint4*>(outp)[q] = w;
+                    }
+                    if (MODE == PV && a.Y) {
 #pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const float2 f = __bfloat1622float2(h[e]);
-                            dot = fmaf(f.x, o[8 * q + 2 * e], dot);
-                            dot = fmaf(f.y, o[8 * q + 2 * e + 1], dot);
+                        for (int q = 0; q < OW / 8; ++q) {
+                            const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&yq[MODE == PV ? q : 0]);
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const float2 f = __bfloat1622float2(h[e]);
+                                dot = fmaf(f.x, o[8 * q + 2 * e], dot);
+                                dot = fmaf(f.y, o[8 * q + 2 * e + 1], dot);
+                            }
                         }
                     }
                 }
-            }
-            if (MODE == PV && a.Y) {
-                red[pt * 128 + lr] = dot;
-                uint32_t eph = 0;
-                const bool synced = ctl.epi_sync(eph);
-                if (synced && pt == 0 && r < L && a.out_vec.p && !*abort_flag) {
-                    float tot = 0.f;
+                if (MODE == PV && a.Y) {
+                    rr[pt * 128 + lr] = dot;
+                    if (!ctl.epi_sync(eph)) { ok = false; break; }
+                    if (pt == 0 && r < L && a.out_vec.p && !*abort_flag) {
+                        float tot = 0.f;
 #pragma unroll
-                    for (int k = 0; k < NPART; ++k) tot += red[k * 128 + lr];
-                    a.out_vec.at(bh, r) = rok ? tot : 0.f;
+                        for (int k = 0; k < NPART; ++k) tot += rr[k * 128 + lr];
+                        a.out_vec.at(bh, r) = rokf ? tot : 0.f;
+                    }
                 }
             }
         }
