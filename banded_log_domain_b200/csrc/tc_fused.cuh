@@ -159,12 +159,13 @@ __device__ __forceinline__ float v_from_partials(const FusedArgs& a, int bh, int
     return a.v_src.at(bh, col) - lg2(partial_sum(a, col, p[0], p[1])) * kLn2;
 }
 
-// E = exp2(c2 * s + cv + rd2) for one thread's 32 columns, written over the
-// scores (as float bits); `CHECK` masks the entries off the band (only the
-// groups that straddle the band's edge).  Row sums go to two packed pairs.
+// E = exp2(c2 * s + cv + rd2) for one thread's 32 columns, packed to fp16
+// pairs in `ep`; `CHECK` masks the entries off the band (only the groups that
+// straddle the band's edge).  The fp32 values are added to four row-sum
+// accumulators (columns 4q + k into acc[k]).
 template <bool CHECK>
-__device__ __forceinline__ void group_exp(uint32_t (&u)[32], const float* cvp, float c2, float rd2,
-                                          int d_first, int W, uint64_t (&accp)[2]) {
+__device__ __forceinline__ void group_exp(const uint32_t (&u)[32], const float* cvp, float c2, float rd2,
+                                          int d_first, int W, uint32_t (&ep)[16], float (&acc)[4]) {
     const float4* c4 = reinterpret_cast<const float4*>(cvp);
     const uint64_t c2p = tc::pk2(c2, c2), rdp = tc::pk2(rd2, rd2);
 #pragma unroll
@@ -183,12 +184,12 @@ __device__ __forceinline__ void group_exp(uint32_t (&u)[32], const float* cvp, f
             if ((unsigned)(d0 - 3 + W) > (unsigned)(2 * W)) x3 = -INFINITY;
         }
         const float e0 = ex2(x0), e1 = ex2(x1), e2 = ex2(x2), e3 = ex2(x3);
-        accp[0] = tc::add2(accp[0], tc::pk2(e0, e1));
-        accp[1] = tc::add2(accp[1], tc::pk2(e2, e3));
-        u[4 * q] = __float_as_uint(e0);
-        u[4 * q + 1] = __float_as_uint(e1);
-        u[4 * q + 2] = __float_as_uint(e2);
-        u[4 * q + 3] = __float_as_uint(e3);
+        acc[0] += e0;
+        acc[1] += e1;
+        acc[2] += e2;
+        acc[3] += e3;
+        ep[2 * q] = pack_f16(e0, e1);
+        ep[2 * q + 1] = pack_f16(e2, e3);
     }
 }
 
@@ -454,7 +455,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fused_iter(const FusedArgs a,
             // invalid rows carry -inf: all their E are 0
             const float rd2 = rowring[(it & 1) * 128 + lr];
             const bool rok = rd2 != -INFINITY;
-            uint64_t accp[2] = {0ull, 0ull};  // packed partial row sums
+            float acc4[4] = {0.f, 0.f, 0.f, 0.f};  // partial row sums
             for (int c = 0; c < nch; ++c) {
                 const int g = it * nch + c, b = g & 1;
                 if (b != grp) continue;  // the other group's chunk
@@ -476,26 +477,22 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fused_iter(const FusedArgs a,
                     const int cg = r0 - W + 128 * c + jc;
                     const bool all_in = (cg >= rw0 + 31 - W) && (cg + 31 <= rw0 + W);
                     const bool all_out = (cg + 31 < rw0 - W) || (cg > rw0 + 31 + W);
+                    uint32_t ep[16];
                     if (all_out) {
 #pragma unroll
-                        for (int j = 0; j < 32; ++j) u[j] = 0u;
+                        for (int j = 0; j < 16; ++j) ep[j] = 0u;
                     } else if (all_in) {
-                        group_exp<false>(u, cvc + jc, c2, rd2, r - cg, W, accp);
+                        group_exp<false>(u, cvc + jc, c2, rd2, r - cg, W, ep, acc4);
                     } else {
-                        group_exp<true>(u, cvc + jc, c2, rd2, r - cg, W, accp);
+                        group_exp<true>(u, cvc + jc, c2, rd2, r - cg, W, ep, acc4);
                     }
                     // the previous tile's column sums must have read E chunk c
                     if (q2 == 0 && it >= 1 && !ctl.wait(B_CS + c, (it - 1) & 1)) { ok = false; break; }
                     // E of these 32 columns: 16-byte chunks 4 q2 + q of the half tile
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        uint4 w4;
-                        w4.x = pack_f16(__uint_as_float(u[8 * q + 0]), __uint_as_float(u[8 * q + 1]));
-                        w4.y = pack_f16(__uint_as_float(u[8 * q + 2]), __uint_as_float(u[8 * q + 3]));
-                        w4.z = pack_f16(__uint_as_float(u[8 * q + 4]), __uint_as_float(u[8 * q + 5]));
-                        w4.w = pack_f16(__uint_as_float(u[8 * q + 6]), __uint_as_float(u[8 * q + 7]));
-                        *reinterpret_cast<uint4*>(et + tc::sw128_off(lr, 4 * q2 + q)) = w4;
-                    }
+                    for (int q = 0; q < 4; ++q)
+                        *reinterpret_cast<uint4*>(et + tc::sw128_off(lr, 4 * q2 + q)) =
+                            make_uint4(ep[4 * q], ep[4 * q + 1], ep[4 * q + 2], ep[4 * q + 3]);
                 }
                 if (!ok) break;
                 // the previous tile's column sums of chunk c (complete: waited above)
@@ -512,10 +509,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fused_iter(const FusedArgs a,
             // on to the next tile; part 0 forms u, 1/r and the quadrant's scale.
             tc::fence_async_smem();  // this warp's E stores, for the column MMAs
             float* rq = red + (it & 1) * 512 + qd * 128;
-            float a0, a1, a2, a3;
-            tc::upk2(accp[0], a0, a1);
-            tc::upk2(accp[1], a2, a3);
-            const float rpart = (a0 + a1) + (a2 + a3);
+            const float rpart = (acc4[0] + acc4[1]) + (acc4[2] + acc4[3]);
             if (pt != 0) {
                 // part 0 has read this buffer's previous contents (and arrived on
                 // WFULL for the previous tile) once it released tile it - 1
