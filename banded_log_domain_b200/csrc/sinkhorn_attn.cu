@@ -151,23 +151,30 @@ BwdLayout bwd_layout(const Dims& d) {
 // ---------------------------------------------------------------------------
 
 // out[bh][t] = <X_t, Y_t> over d for valid tokens, 0 for masked ones and for
-// the dustbin slot t = L.  One warp per token.
+// the dustbin slot t = L.  A token's row is read by kD / (16 / sizeof(T)) lanes,
+// one 16-byte load per tensor each (coalesced), and summed with shuffles.
 template <typename T>
 __global__ void k_rowdot(const T* X, const T* Y, const uint8_t* mask, int L, int H, int ld,
                          int BH, float* out) {
-    const long long gw = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-    const int lane = threadIdx.x & 31;
-    if (gw >= (long long)BH * ld) return;
-    const int bh = (int)(gw / ld), t = (int)(gw % ld);
+    constexpr int VE = 16 / (int)sizeof(T), LPT = kD / VE;  // elements per load, lanes per token
+    static_assert(32 % LPT == 0, "a token's lanes share a warp");
+    const long long g = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    const long long tok = g / LPT;
+    const int sub = (int)(g % LPT);
+    const bool in = tok < (long long)BH * ld;
+    const int bh = in ? (int)(tok / ld) : 0, t = in ? (int)(tok % ld) : 0;
     float s = 0.f;
-    const bool ok = t < L && (mask == nullptr || mask[(size_t)(bh / H) * L + t]);
-    if (ok) {
-        const size_t o = ((size_t)bh * L + t) * kD;
-        for (int e = lane; e < kD; e += 32) s = fmaf(to_f32(X[o + e]), to_f32(Y[o + e]), s);
+    if (in && t < L && (mask == nullptr || mask[(size_t)(bh / H) * L + t])) {
+        const size_t o = ((size_t)bh * L + t) * kD + (size_t)sub * VE;
+        float x[8], y[8];
+        load_vec(X + o, x, VE);
+        load_vec(Y + o, y, VE);
+#pragma unroll
+        for (int e = 0; e < VE; ++e) s = fmaf(x[e], y[e], s);
     }
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
-    if (lane == 0) out[(size_t)bh * ld + t] = s;
+    for (int off = LPT / 2; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off, LPT);
+    if (in && sub == 0) out[(size_t)bh * ld + t] = s;
 }
 
 // eu[a][bh][t] = exp(u^(a) - u^(R)), ev[a][bh][t] = exp(v^(a) - v^(R)), a = 0..R;
@@ -589,7 +596,7 @@ sa_status bwd_impl(const Ctx& x, const T* q, const T* k, const T* v, const uint8
 
     // a = rowdot(dO, O); orbit factors
     {
-        const long long thr = nvec * 32;
+        const long long thr = nvec * (kD / (16 / (long long)sizeof(T)));
         SA_AUX(x.tr, k_rowdot<T><<<(unsigned)((thr + 255) / 256), 256, 0, x.st>>>(
                          dO, o, mask, d.L, d.H, d.ld, d.BH, A_));
         SA_AUX(x.tr, k_orbit<<<egrid, eb, 0, x.st>>>(x.state, R, d.L, d.H, d.ld, d.BH, mask,
