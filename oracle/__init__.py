@@ -215,3 +215,76 @@ def support_size(L, W, mask_row=None, dustbin=False):
     p = _params(L, 1, W, 0, 1, 1.0, dustbin, 0.0)
     m = None if mask_row is None else np.ascontiguousarray(mask_row, dtype=np.uint8)
     return int(lib.orc_support_size(ctypes.byref(p), None if m is None else _up(m)))
+
+
+# ---------------------------------------------------------------------------
+# Full backpropagation, the tail-depth-0 gradient and the bias certificate
+# (Block-Wise Differentiable Sinkhorn Attention, gist.science/de technical
+# summary: section 3 states the a posteriori bias certificate, section 4.1 the
+# bias-decay comparison of tail gradients with full backpropagation through time)
+# ---------------------------------------------------------------------------
+
+def full_bptt(q, k, v, dO, *, N, W, eps, mask=None, schedule="direct"):
+    """Gradients of <dO, O> with backpropagation through the whole N-iteration
+    solve (nothing stopped).  The solve from v = 0 is a stopped base of zero
+    iterations (a constant) followed by an N-iteration tail, so these are the
+    surrogate's exact gradients with T = 0, R = N.  Returns (o, state, (dq, dk, dv))."""
+    o, st = forward(q, k, v, W=W, eps=eps, T=0, R=N, mask=mask)
+    dq, dk, dv, _ = backward(q, k, v, st, dO, W=W, eps=eps, R=N, mask=mask, schedule=schedule)
+    return o, st, (dq, dk, dv)
+
+
+def stopped_gradients(q, k, v, dO, *, N, W, eps, mask=None):
+    """Gradients with every one of the N iterations stopped (tail depth 0):
+    O = P V with P = exp(S + u + v) from the stopped duals, so on the support
+    dS = P * (dO V^T), dQ = c dS K, dK = c dS^T Q, dV = P^T dO (c = 1/(sqrt(d) eps)).
+    Band layout: offset t of row i is column i - W + t.  No dustbin."""
+    q, k, v, dO = _f64(q), _f64(k), _f64(v), _f64(dO)
+    B, H, L, d = q.shape
+    c = 1.0 / (np.sqrt(d) * eps)
+    _, st = forward(q, k, v, W=W, eps=eps, T=N, R=1, mask=mask)
+    P, _, _ = plan(q, k, st, 0, 0, W=W, eps=eps, R=1, mask=mask)  # [B,H,L,2W+1], 0 off the support
+    dq = np.zeros_like(q)
+    dk = np.zeros_like(k)
+    dv = np.zeros_like(v)
+    for t in range(2 * W + 1):
+        off = t - W  # column j = i + off
+        i0, i1 = max(0, -off), min(L, L - off)  # rows whose column is inside [0, L)
+        if i1 <= i0:
+            continue
+        rows = slice(i0, i1)
+        cols = slice(i0 + off, i1 + off)
+        p = P[:, :, rows, t]                                           # [B,H,n]
+        g = np.einsum("bhnd,bhnd->bhn", dO[:, :, rows], v[:, :, cols])  # <dO_i, V_j>
+        ds = p * g
+        dq[:, :, rows] += c * ds[..., None] * k[:, :, cols]
+        dk[:, :, cols] += c * ds[..., None] * q[:, :, rows]
+        dv[:, :, cols] += p[..., None] * dO[:, :, rows]
+    return dq, dk, dv
+
+
+def tail_gradients(q, k, v, dO, *, N, R, W, eps, mask=None, schedule="direct"):
+    """The surrogate's gradients for a solve of N iterations with tail depth R
+    (T = N - R stopped base iterations); R = 0 stops every iteration."""
+    if R == 0:
+        return stopped_gradients(q, k, v, dO, N=N, W=W, eps=eps, mask=mask)
+    _, st = forward(q, k, v, W=W, eps=eps, T=N - R, R=R, mask=mask)
+    dq, dk, dv, _ = backward(q, k, v, st, dO, W=W, eps=eps, R=R, mask=mask, schedule=schedule)
+    return dq, dk, dv
+
+
+def bias_certificate(q, k, v, dO, *, N, Rs=(0, 1, 2, 4), tau=1e-5, W, eps, mask=None):
+    """For a solve of N iterations, eta_R = ||g_R - g_full|| / ||g_full|| over
+    (dQ, dK, dV): the relative size of the gradient that the stopped base omits
+    at tail depth R (g_R as in ``tail_gradients``, g_full = ``full_bptt``).
+    Returns ({R: eta_R}, R*), R* the smallest R in Rs with eta_R <= tau (None if
+    none does)."""
+    _, _, gf = full_bptt(q, k, v, dO, N=N, W=W, eps=eps, mask=mask)
+    ref = np.sqrt(sum(float(np.sum(x * x)) for x in gf))
+    eta = {}
+    for R in sorted(Rs):
+        g = tail_gradients(q, k, v, dO, N=N, R=R, W=W, eps=eps, mask=mask)
+        num = np.sqrt(sum(float(np.sum((a - b) ** 2)) for a, b in zip(g, gf)))
+        eta[R] = num / ref if ref > 0 else num
+    ok = [R for R in sorted(Rs) if eta[R] <= tau]
+    return eta, (ok[0] if ok else None)

@@ -19,11 +19,13 @@ import torch
 
 
 def surrogate(q, k, v, *, W, eps, T, R, mask=None, dustbin=False, dustbin_score=-2.0,
-              v_dust=None, base=None):
+              v_dust=None, base=None, stop_base=True):
     """One problem: ``q, k, v`` are ``[L,d]`` float64 (may require grad).
 
     Returns ``o [L,d]`` and ``state [2R+2, L+db]`` (rows u0, v0, u1, v1, ...),
     with zeros on masked tokens.  ``base``: optional frozen ``[2, L+db]``.
+    ``stop_base=False`` lets the gradient run through the T base iterations too
+    (full backpropagation through the whole T+R-iteration solve).
     """
     L, d = q.shape
     c = 1.0 / (math.sqrt(d) * eps)
@@ -58,7 +60,7 @@ def surrogate(q, k, v, *, W, eps, T, R, mask=None, dustbin=False, dustbin_score=
         return out.index_put((full_idx,), x)
 
     if base is None:
-        with torch.no_grad():
+        with torch.set_grad_enabled(not stop_base and torch.is_grad_enabled()):
             uu = torch.zeros(m, dtype=q.dtype)
             vv = torch.zeros(m, dtype=q.dtype)
             for _ in range(T):
@@ -67,8 +69,10 @@ def surrogate(q, k, v, *, W, eps, T, R, mask=None, dustbin=False, dustbin_score=
     else:
         b = torch.as_tensor(base, dtype=q.dtype)
         uu, vv = b[0][full_idx], b[1][full_idx]
-    us, vs = [uu.detach()], [vv.detach()]
-    vprev = vv.detach()
+    if stop_base:
+        uu, vv = uu.detach(), vv.detach()
+    us, vs = [uu], [vv]
+    vprev = vv
     for _ in range(R):
         uu = row_upd(vprev)
         vv = col_upd(uu)
