@@ -102,11 +102,12 @@ def _L():
                                              vp, vp, vp]
     lib.sinkhorn_attn_poll.argtypes = [vp, vp]
     lib.sinkhorn_attn_debug_timeout.argtypes = [vp, ctypes.c_longlong, vp]
+    lib.sinkhorn_attn_sq_dist.argtypes = [vp, vp, ctypes.c_longlong, ctypes.c_int, vp, vp]
     lib.sinkhorn_attn_strerror.argtypes = [ctypes.c_int]
     lib.sinkhorn_attn_strerror.restype = ctypes.c_char_p
     for f in ("sinkhorn_attn_state_size", "sinkhorn_attn_workspace_size", "sinkhorn_attn_fwd",
               "sinkhorn_attn_bwd", "sinkhorn_attn_debug_plan", "sinkhorn_attn_poll",
-              "sinkhorn_attn_debug_timeout"):
+              "sinkhorn_attn_debug_timeout", "sinkhorn_attn_sq_dist"):
         getattr(lib, f).restype = ctypes.c_int
     _lib = lib
     return lib
@@ -119,7 +120,8 @@ def load():
 
 EXPORTS = ("sinkhorn_attn_state_size", "sinkhorn_attn_workspace_size", "sinkhorn_attn_fwd",
            "sinkhorn_attn_bwd", "sinkhorn_attn_bwd_static_ws", "sinkhorn_attn_debug_plan",
-           "sinkhorn_attn_poll", "sinkhorn_attn_strerror", "sinkhorn_attn_debug_timeout")
+           "sinkhorn_attn_poll", "sinkhorn_attn_strerror", "sinkhorn_attn_debug_timeout",
+           "sinkhorn_attn_sq_dist")
 
 
 def strerror(status: int) -> str:
@@ -285,6 +287,53 @@ def sinkhorn_attn_debug_timeout(ws, budget_cycles: int = 1_000_000) -> int:
     for the failure path); the timeout lands in the status word of ``ws`` (a
     CUDA tensor of at least 256 bytes) and is read by :func:`sinkhorn_attn_poll`."""
     return int(_L().sinkhorn_attn_debug_timeout(_ptr(ws), int(budget_cycles), _stream(ws.device)))
+
+
+def sinkhorn_attn_sq_dist(x, y):
+    """``(sum (x - y)^2, sum y^2)`` in double for two contiguous CUDA tensors of
+    one shape and dtype (float32 or bfloat16)."""
+    _contig(x, y)
+    if x.shape != y.shape or x.dtype != y.dtype:
+        raise ValueError("x and y must have one shape and dtype")
+    dt = {torch.float32: SA_F32, torch.bfloat16: SA_BF16}[x.dtype]
+    out = torch.empty(2, dtype=torch.float64, device=x.device)
+    _check(_L().sinkhorn_attn_sq_dist(_ptr(x), _ptr(y), x.numel(), dt, _ptr(out),
+                                      _stream(x.device)), "sinkhorn_attn_sq_dist")
+    s = out.cpu()
+    return float(s[0]), float(s[1])
+
+
+def bias_certificate(q, k, v, dO, *, N, Rs=(0, 1, 2, 4), tau=1e-5, W, eps, mask=None,
+                     schedule="one_reference"):
+    """A-posteriori bias certificate of the stopped base for a solve of N
+    iterations (gist.science/de section 3, section 4.1).  For each tail depth R in
+    ``Rs`` (0 <= R <= N) the gradients g_R of <dO, O> come from
+    :func:`sinkhorn_attn_fwd` / :func:`sinkhorn_attn_bwd` with T = N - R stopped
+    iterations; g_full, full backpropagation, from T = 0 and R = N.  Then
+    eta_R = ||g_R - g_full|| / ||g_full|| over (dQ, dK, dV), the norms from
+    :func:`sinkhorn_attn_sq_dist`.  Returns ``({R: eta_R}, R*)``, R* the smallest
+    R in ``Rs`` with eta_R <= tau (None if none is).  No dustbin."""
+    if any(not 0 <= R <= N for R in Rs):
+        raise ValueError("every R must lie in [0, N]")
+
+    def grads(T, R):
+        o, st = sinkhorn_attn_fwd(q, k, v, W=W, eps=eps, T=T, R=R, mask=mask)
+        g = sinkhorn_attn_bwd(q, k, v, o, dO, st, W=W, eps=eps, R=R, mask=mask,
+                              schedule=schedule)[:3]
+        return g
+
+    full = grads(0, N)
+    eta = {}
+    for R in sorted(set(Rs)):
+        g = full if R == N else grads(N - R, R)
+        num = den = 0.0
+        for a, b in zip(g, full):
+            d2, n2 = sinkhorn_attn_sq_dist(a, b)
+            num += d2
+            den += n2
+        eta[R] = math.sqrt(num / den) if den > 0 else math.sqrt(num)
+    ok = [R for R in sorted(eta) if eta[R] <= tau]
+    return eta, (ok[0] if ok else None)
 
 
 def score_scale(d: int, eps: float) -> float:

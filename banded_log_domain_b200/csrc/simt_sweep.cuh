@@ -68,6 +68,13 @@ struct SweepArgs {
     Vec er[MAXT], ec[MAXT], cr[MAXT], cc[MAXT];  // DSD (cr/cc p null = 0)
     float gk[MAXT];                          // DSD: weight of G in term k
     float* dvd_part;        // PV dustbin row: [BH][D] sum_c P_(dust,c) X_c (or null)
+    // DS with more than MAXT terms runs one launch per block of terms; the
+    // launches sum their results in fp32 (plain read-add-write: every output row
+    // has one writer per launch and launches are stream ordered)
+    float* acc;             // fp32 running sum [BH][L][D]
+    int acc_in;             // 1: add acc's contents to this launch's result
+    int acc_out;            // 1: write the sum to acc instead of out_mat
+    int g_off;              // DS1: leave G out of M (every block but the first)
     int online;             // LSE on tensor cores: 1 = no previous dual, use a running max
 };
 
@@ -368,7 +375,7 @@ __global__ void __launch_bounds__(NT) band_sweep(const SweepArgs a) {
                         if (MODE == PV) {
                             val = ex2(fmaf(a.c2, acc[i][j], rd2[i] + ce[cj]));
                         } else if (MODE == DS1) {
-                            float M = g[i][j];
+                            float M = a.g_off ? 0.f : g[i][j];
 #pragma unroll
                             for (int k = 0; k < MAXT; ++k)
                                 if (k < a.nterms) M = fmaf(rmod[k][i], cmod[k * BN + cj], M);
@@ -448,7 +455,15 @@ __global__ void __launch_bounds__(NT) band_sweep(const SweepArgs a) {
 #pragma unroll
             for (int j = 0; j < 4; ++j) o4[j] = rv_ok[i] ? oacc[i][j] * scale : 0.f;
             if (r < L) {
-                store4(outb + (size_t)r * D + tx * 4, o4[0], o4[1], o4[2], o4[3]);
+                float* accr = (DS && a.acc) ? a.acc + off + (size_t)r * D + tx * 4 : nullptr;
+                if (DS && accr && a.acc_in) {
+                    const float4 p = *reinterpret_cast<const float4*>(accr);
+                    o4[0] += p.x; o4[1] += p.y; o4[2] += p.z; o4[3] += p.w;
+                }
+                if (DS && accr && a.acc_out)
+                    *reinterpret_cast<float4*>(accr) = make_float4(o4[0], o4[1], o4[2], o4[3]);
+                else
+                    store4(outb + (size_t)r * D + tx * 4, o4[0], o4[1], o4[2], o4[3]);
                 if (Yb) {
 #pragma unroll
                     for (int j = 0; j < 4; ++j) dot = fmaf(to_f32(Yb[(size_t)r * D + tx * 4 + j]), o4[j], dot);

@@ -21,6 +21,7 @@
 // P^(r,r) formed by its own exponential.
 #include <cmath>
 #include <algorithm>
+#include <vector>
 #include <cstring>
 #include <mutex>
 
@@ -38,6 +39,7 @@ namespace {
 
 constexpr size_t kHeader = 256;   // status word + padding at the start of every workspace
 constexpr int kD = simt::D;
+constexpr int kMaxR = 256;  // tail length limit (host term lists, workspace)
 
 size_t align_up(size_t x) { return (x + 255) & ~size_t(255); }
 
@@ -48,7 +50,7 @@ struct Dims {
 
 sa_status check_params(const sa_params* p, Dims* dd) {
     if (!p) return SA_ERR_INVALID_ARG;
-    if (p->B < 0 || p->H < 0 || p->L < 0 || p->d <= 0 || p->W < 0 || p->T < 0 || p->R < 1)
+    if (p->B < 0 || p->H < 0 || p->L < 0 || p->d <= 0 || p->W < 0 || p->T < 0 || p->R < 0)
         return SA_ERR_INVALID_ARG;
     if (!(p->eps > 0.f) || !std::isfinite(p->eps)) return SA_ERR_INVALID_ARG;
     if (p->dtype != SA_F32 && p->dtype != SA_BF16) return SA_ERR_INVALID_ARG;
@@ -57,7 +59,7 @@ sa_status check_params(const sa_params* p, Dims* dd) {
     if (p->bwd != SA_BWD_ONE_REFERENCE && p->bwd != SA_BWD_DIRECT) return SA_ERR_INVALID_ARG;
     if (p->check_finite != 0 && p->check_finite != 1) return SA_ERR_INVALID_ARG;
     if (p->d != kD) return SA_ERR_UNSUPPORTED;
-    if (p->R > 4) return SA_ERR_UNSUPPORTED;
+    if (p->R > kMaxR) return SA_ERR_UNSUPPORTED;
     const long long BH = (long long)p->B * p->H;
     if (BH > 65535) return SA_ERR_UNSUPPORTED;
     if ((long long)p->L * kD > (1LL << 40)) return SA_ERR_UNSUPPORTED;
@@ -126,7 +128,7 @@ FwdLayout fwd_layout(const Dims& d, const sa_params* p) {
 
 // Backward workspace layout (float32 vectors of BH * ld elements each).
 struct BwdLayout {
-    size_t a, ubar, vbar, eu, ev, w, rv, cv, dvd, total;
+    size_t a, ubar, vbar, eu, ev, w, rv, cv, dvd, acc, total;
     size_t vec;  // bytes of one [BH][ld] vector, 256-aligned
 };
 BwdLayout bwd_layout(const Dims& d) {
@@ -142,6 +144,8 @@ BwdLayout bwd_layout(const Dims& d) {
     l.rv = o;   o += l.vec * 2 * d.R;
     l.cv = o;   o += l.vec * 2 * d.R;
     l.dvd = o;  o += align_up((size_t)d.BH * kD * sizeof(float));
+    l.acc = o;  // fp32 sum of the dS sweeps' term blocks, when 2R > MAXT
+    if (2 * d.R > simt::MAXT) o += align_up((size_t)d.BH * d.L * kD * sizeof(float));
     l.total = o;
     return l;
 }
@@ -212,6 +216,27 @@ __global__ void k_dvd_reduce(const float* part, int B, int H, float* out) {
     float s = 0.f;
     for (int b = 0; b < B; ++b) s += part[((size_t)b * H + h) * kD + e];
     out[g] = s;
+}
+
+// out[0] += sum_i (x_i - y_i)^2, out[1] += sum_i y_i^2 in double: grid-stride
+// loop, warp shuffles, one atomic pair per warp.
+template <typename T>
+__global__ void k_sq_dist(const T* x, const T* y, long long n, double* out) {
+    double s0 = 0.0, s1 = 0.0;
+    const long long stride = (long long)gridDim.x * blockDim.x;
+    for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += stride) {
+        const double a = to_f32(x[i]), b = to_f32(y[i]);
+        s0 += (a - b) * (a - b);
+        s1 += b * b;
+    }
+    for (int o = 16; o > 0; o >>= 1) {
+        s0 += __shfl_xor_sync(0xffffffffu, s0, o);
+        s1 += __shfl_xor_sync(0xffffffffu, s1, o);
+    }
+    if ((threadIdx.x & 31) == 0) {
+        atomicAdd(out, s0);
+        atomicAdd(out + 1, s1);
+    }
 }
 
 // A wait that nothing completes: thread 0 waits on a fresh mbarrier (one
@@ -375,7 +400,9 @@ cudaError_t launch_sweep(const simt::SweepArgs& a, int BH, cudaStream_t st, Trac
                 if (a.online) return launch_tc<MODE, true, 0>(a, BH, st, tr, status);
                 return launch_tc<MODE, false, 0>(a, BH, st, tr, status);
             } else if constexpr (MODE == simt::DS1 || MODE == simt::DSD) {
-                switch (a.nterms) {  // 2R terms, R = 1..4
+                if (MODE == simt::DS1 && a.nterms == 0)  // R = 0: dS = P * G
+                    return launch_tc<MODE, false, 0>(a, BH, st, tr, status);
+                switch (a.nterms) {  // a block of the 2R terms: 2, 4, 6 or MAXT
                     case 2: return launch_tc<MODE, false, 2>(a, BH, st, tr, status);
                     case 4: return launch_tc<MODE, false, 4>(a, BH, st, tr, status);
                     case 6: return launch_tc<MODE, false, 6>(a, BH, st, tr, status);
@@ -622,8 +649,8 @@ sa_status bwd_impl(const Ctx& x, const T* q, const T* k, const T* v, const uint8
         a.dvd_part = dvd;
         SA_CUDA((launch_sweep<T, simt::PV>(a, d.BH, x.st, x.tr, x.status)));
     }
-    // ubar^R = a - P vbar^R  (query sweep)
-    {
+    // ubar^R = a - P vbar^R  (query sweep; R = 0 has no dual cotangents)
+    if (R > 0) {
         simt::SweepArgs a = base_args(x);
         a.mask = mask;
         a.A = q; a.Bo = k;
@@ -675,13 +702,12 @@ sa_status bwd_impl(const Ctx& x, const T* q, const T* k, const T* v, const uint8
     //   direct: dS = sum_k exp(S + eq_k[i] + ek_k[j]) (g_k G + cq_k[i] + ck_k[j])
     //     k=0: (u^R, v^R; G - vbar^R);  r: (u^r, v^(r-1); -ubar^r);  r<R: (u^r, v^r; -vbar^r)
     int nt = 0;
-    Vec rq[simt::MAXT], rk[simt::MAXT];
-    Vec eq[simt::MAXT], ek[simt::MAXT], cq[simt::MAXT], ck[simt::MAXT];
-    float gk[simt::MAXT];
+    std::vector<Vec> rq(2 * R), rk(2 * R), eq(2 * R), ek(2 * R), cq(2 * R), ck(2 * R);
+    std::vector<float> gk(2 * R);
     const Vec none{nullptr, 0};
     auto slot_q = [&](int i) { return (float*)(ws + l.rv + (size_t)i * l.vec); };
     auto slot_k = [&](int i) { return (float*)(ws + l.cv + (size_t)i * l.vec); };
-    {
+    if (R > 0) {  // R = 0: every dual is a constant and dS = P * G (no terms)
         // k = 0
         SA_AUX(x.tr, k_vmul<<<egrid, eb, 0, x.st>>>(vb(R), nullptr, -1.f, slot_k(0), nvec));
         rq[nt] = none; rk[nt] = vec(slot_k(0), vs);
@@ -711,33 +737,45 @@ sa_status bwd_impl(const Ctx& x, const T* q, const T* k, const T* v, const uint8
             ++nt;
         }
     }
-    // dQ (query sweep) and dK (key sweep)
+    // dQ (query sweep) and dK (key sweep).  A sweep takes at most MAXT terms;
+    // longer tails (R > MAXT / 2) run one sweep per block of MAXT terms (the
+    // first block carrying G), summed in fp32 in the workspace and rounded once.
+    const int nblk_t = std::max(1, (nt + simt::MAXT - 1) / simt::MAXT);
     for (int side = 0; side < 2; ++side) {
-        simt::SweepArgs a = base_args(x);
-        a.mask = mask;
-        a.dust_cta = 0;
-        a.nterms = nt;
-        if (side == 0) {
-            a.A = q; a.Bo = k; a.A2 = dO; a.B2 = v; a.X = k;
-            a.rd = uR; a.cd = vR;
-            a.out_mat = dq;
-            for (int t = 0; t < nt; ++t) {
-                a.rv[t] = rq[t]; a.cv[t] = rk[t];
-                a.er[t] = eq[t]; a.ec[t] = ek[t]; a.cr[t] = cq[t]; a.cc[t] = ck[t];
-                a.gk[t] = gk[t];
+        for (int tb = 0; tb < nblk_t; ++tb) {
+            const int k0 = tb * simt::MAXT, kn = std::min(simt::MAXT, nt - k0);
+            simt::SweepArgs a = base_args(x);
+            a.mask = mask;
+            a.dust_cta = 0;
+            a.nterms = kn;
+            if (nblk_t > 1) {
+                a.acc = (float*)(ws + l.acc);
+                a.acc_in = tb > 0;
+                a.acc_out = tb + 1 < nblk_t;
+                a.g_off = tb > 0;
             }
-        } else {
-            a.A = k; a.Bo = q; a.A2 = v; a.B2 = dO; a.X = q;
-            a.rd = vR; a.cd = uR;
-            a.out_mat = dk;
-            for (int t = 0; t < nt; ++t) {
-                a.rv[t] = rk[t]; a.cv[t] = rq[t];
-                a.er[t] = ek[t]; a.ec[t] = eq[t]; a.cr[t] = ck[t]; a.cc[t] = cq[t];
-                a.gk[t] = gk[t];
+            if (side == 0) {
+                a.A = q; a.Bo = k; a.A2 = dO; a.B2 = v; a.X = k;
+                a.rd = uR; a.cd = vR;
+                a.out_mat = dq;
+                for (int t = 0; t < kn; ++t) {
+                    a.rv[t] = rq[k0 + t]; a.cv[t] = rk[k0 + t];
+                    a.er[t] = eq[k0 + t]; a.ec[t] = ek[k0 + t]; a.cr[t] = cq[k0 + t]; a.cc[t] = ck[k0 + t];
+                    a.gk[t] = gk[k0 + t];
+                }
+            } else {
+                a.A = k; a.Bo = q; a.A2 = v; a.B2 = dO; a.X = q;
+                a.rd = vR; a.cd = uR;
+                a.out_mat = dk;
+                for (int t = 0; t < kn; ++t) {
+                    a.rv[t] = rk[k0 + t]; a.cv[t] = rq[k0 + t];
+                    a.er[t] = ek[k0 + t]; a.ec[t] = eq[k0 + t]; a.cr[t] = ck[k0 + t]; a.cc[t] = cq[k0 + t];
+                    a.gk[t] = gk[k0 + t];
+                }
             }
+            if (direct && R > 0) SA_CUDA((launch_sweep<T, simt::DSD>(a, d.BH, x.st, x.tr, x.status)));
+            else SA_CUDA((launch_sweep<T, simt::DS1>(a, d.BH, x.st, x.tr, x.status)));
         }
-        if (direct) SA_CUDA((launch_sweep<T, simt::DSD>(a, d.BH, x.st, x.tr, x.status)));
-        else SA_CUDA((launch_sweep<T, simt::DS1>(a, d.BH, x.st, x.tr, x.status)));
     }
     if (x.p->dustbin && dv_dust) {
         SA_AUX(x.tr, k_dvd_reduce<<<(d.H * kD + 255) / 256, 256, 0, x.st>>>(dvd, d.B, d.H,
@@ -786,6 +824,7 @@ sa_status sinkhorn_attn_fwd(const sa_params* p, const void* q, const void* k, co
     Dims d;
     sa_status s = check_params(p, &d);
     if (s != SA_OK) return s;
+    if (p->T + p->R < 1) return SA_ERR_INVALID_ARG;  // the solve needs an iteration
     if (ws_bytes < fwd_layout(d, p).total) return SA_ERR_WORKSPACE;
     if (d.BH == 0 || d.L == 0) return SA_OK;
     if (!device_ok(q) || !device_ok(k) || !device_ok(v) || !device_ok(o) || !device_ok(state) ||
@@ -1001,6 +1040,23 @@ sa_status sinkhorn_attn_debug_timeout(void* ws, long long budget_cycles, void* s
     if (!ws || ((uintptr_t)ws & 15)) return SA_ERR_INVALID_ARG;
     const long long b = budget_cycles < 1 ? 1 : (budget_cycles > 100000000LL ? 100000000LL : budget_cycles);
     sa::k_stall<<<1, 32, 0, (cudaStream_t)stream>>>((int*)ws, b);
+    return cudaGetLastError() == cudaSuccess ? SA_OK : SA_ERR_CUDA;
+}
+
+sa_status sinkhorn_attn_sq_dist(const void* x, const void* y, long long n, sa_dtype dtype,
+                               double* out, void* stream) {
+    if (n < 0 || (dtype != SA_F32 && dtype != SA_BF16)) return SA_ERR_INVALID_ARG;
+    if (!sa::device_ok(out) || (n > 0 && (!sa::device_ok(x) || !sa::device_ok(y))))
+        return SA_ERR_INVALID_ARG;
+    cudaStream_t st = (cudaStream_t)stream;
+    if (cudaMemsetAsync(out, 0, 2 * sizeof(double), st) != cudaSuccess) return SA_ERR_CUDA;
+    if (n == 0) return SA_OK;
+    const long long blocks = std::min<long long>((n + 255) / 256, 148LL * 8);
+    if (dtype == SA_F32)
+        sa::k_sq_dist<float><<<(unsigned)blocks, 256, 0, st>>>((const float*)x, (const float*)y, n, out);
+    else
+        sa::k_sq_dist<__nv_bfloat16><<<(unsigned)blocks, 256, 0, st>>>(
+            (const __nv_bfloat16*)x, (const __nv_bfloat16*)y, n, out);
     return cudaGetLastError() == cudaSuccess ? SA_OK : SA_ERR_CUDA;
 }
 

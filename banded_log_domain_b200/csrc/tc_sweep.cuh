@@ -482,7 +482,8 @@ __global__ void __launch_bounds__(nthreads(MODE), ctas_per_sm(MODE)) tc_band_swe
                         for (int j = 0; j < 32; ++j) sv[j] = __uint_as_float(su[0][j]);
                         if (DS) {
     #pragma unroll
-                            for (int j = 0; j < 32; ++j) gv[j] = __uint_as_float(gu[0][j]);
+                            for (int j = 0; j < 32; ++j)
+                                gv[j] = (MODE == DS1 && a.g_off) ? 0.f : __uint_as_float(gu[0][j]);
                         }
                         if (g == NG - 1) {  // every TMEM read of this chunk is done
                             tc::tc_fence_before();
@@ -697,7 +698,20 @@ __global__ void __launch_bounds__(nthreads(MODE), ctas_per_sm(MODE)) tc_band_swe
 #pragma unroll
                 for (int j = 0; j < OW; ++j) o[j] = rokf ? o[j] * scale : 0.f;
                 float dot = 0.f;
-                if (r < L) {
+                float* accr = (DS && a.acc && r < L) ? a.acc + ((size_t)bh * L + r) * 64 + OW * pt : nullptr;
+                if (DS && accr && a.acc_in) {
+#pragma unroll
+                    for (int q = 0; q < OW / 4; ++q) {
+                        const float4 p = reinterpret_cast<const float4*>(accr)[q];
+                        o[4 * q] += p.x; o[4 * q + 1] += p.y; o[4 * q + 2] += p.z; o[4 * q + 3] += p.w;
+                    }
+                }
+                if (DS && accr && a.acc_out) {
+#pragma unroll
+                    for (int q = 0; q < OW / 4; ++q)
+                        reinterpret_cast<float4*>(accr)[q] =
+                            make_float4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
+                } else if (r < L) {
                     __nv_bfloat16* outp =
                         reinterpret_cast<__nv_bfloat16*>(a.out_mat) + ((size_t)bh * L + r) * 64 + OW * pt;
 #pragma unroll

@@ -70,7 +70,11 @@ typedef struct {
     int W;                 /* band half-width, W >= 0 (W >= L-1 is dense) */
     float eps;             /* entropic temperature, > 0 */
     int T;                 /* stopped base iterations, T >= 0 */
-    int R;                 /* tail iterations, 1 <= R <= 4 (2 in the pages) */
+    int R;                 /* differentiable tail iterations, 0 <= R <= 256 (2 in the
+                              pages); the forward needs T + R >= 1 (the backward does
+                              not read T).  T = 0, R = N backpropagates through
+                              the whole N-iteration solve; R = 0 holds every dual
+                              constant (dS = P * dO V^T, dV = P^T dO) */
     sa_dtype dtype;        /* element type of Q, K, V, O, dO, dQ, dK, dV */
     int dustbin;           /* 0 or 1: add the dustbin row and column */
     float dustbin_score;   /* score on every dustbin entry, used as given */
@@ -106,7 +110,10 @@ sa_status sinkhorn_attn_state_size(const sa_params* p, size_t* n_floats);
 
 /* Workspace bytes needed by sinkhorn_attn_fwd and sinkhorn_attn_bwd (either
  * pointer may be NULL).  Both are O(B*H*L) and include a 256-byte status
- * header at offset 0. */
+ * header at offset 0.  The backward's grows with R (a few float32 vectors of
+ * B*H*(L+dustbin) per tail step); for R > 4 it also holds a float32
+ * [B][H][L][d] sum of the dQ / dK sweeps over blocks of at most 8 modifier
+ * terms. */
 sa_status sinkhorn_attn_workspace_size(const sa_params* p, size_t* fwd_bytes, size_t* bwd_bytes);
 
 /*
@@ -190,6 +197,22 @@ sa_status sinkhorn_attn_poll(void* ws, void* stream);
 
 /* Static English description of a status code. */
 const char* sinkhorn_attn_strerror(sa_status s);
+
+/* Squared distance for the a-posteriori bias certificate (gist.science/de
+ * section 3, section 4.1): the certificate of tail depth R compares the
+ * gradients with T = N - R stopped iterations against full backpropagation
+ * (T = 0, R = N) as ||g_R - g_full|| / ||g_full||.  This call supplies the two
+ * sums for one gradient tensor:
+ *   out[0] = sum_i (x_i - y_i)^2,  out[1] = sum_i y_i^2,
+ * accumulated in double over n elements of type dtype (SA_F32 or SA_BF16).
+ *   x, y : n elements each, device, 16-byte aligned (may be NULL when n == 0).
+ *   out  : 2 doubles, device, 16-byte aligned; zeroed on `stream`, then
+ *          written by the kernel (summation order is not fixed, so the last
+ *          bits may differ between calls).
+ * Returns SA_ERR_INVALID_ARG for n < 0, another dtype, or a bad pointer;
+ * SA_ERR_CUDA on a launch error; else SA_OK. */
+sa_status sinkhorn_attn_sq_dist(const void* x, const void* y, long long n, sa_dtype dtype,
+                               double* out, void* stream);
 
 /* Test hook for the failure path; no counterpart in the pages.  Launches on
  * `stream` one CTA whose thread waits, through the same bounded mbarrier wait

@@ -47,9 +47,21 @@ def test_state_and_workspace_sizes():
     assert b1 == b2 and 1.9 < b3 / b1 < 2.1
 
 
+def test_workspace_holds_the_term_block_sum_beyond_four_tail_steps():
+    # R <= 4: 2R modifier terms fit one dS sweep; R = 5 adds an fp32 [B][H][L][d]
+    # sum of the term blocks plus the per-step vectors
+    _, b4 = sa.sinkhorn_attn_workspace_size(P(R=4))
+    _, b5 = sa.sinkhorn_attn_workspace_size(P(R=5))
+    acc = 2 * 3 * 100 * 64 * 4
+    per_step = 8 * 2560  # four [B][H][L] vectors and two term slots per side, 256-aligned
+    assert b5 - b4 == acc + per_step
+    _, b6 = sa.sinkhorn_attn_workspace_size(P(R=6))
+    assert b6 - b5 == per_step
+
+
 @pytest.mark.parametrize("kw,status", [
     (dict(W=-1), -1), (dict(eps=0.0), -1), (dict(eps=float("nan")), -1), (dict(T=-1), -1),
-    (dict(R=0), -1), (dict(L=-5), -1), (dict(d=32), -2), (dict(R=5), -2),
+    (dict(R=-1), -1), (dict(L=-5), -1), (dict(d=32), -2), (dict(R=257), -2),
     (dict(dustbin=True, dustbin_score=float("inf")), -1),
 ])
 def test_invalid_params_rejected(kw, status):
@@ -88,6 +100,29 @@ def test_null_and_host_pointers_rejected_before_launch():
     rc = lib.sinkhorn_attn_fwd(ctypes.byref(p), addr + 4, addr, addr, None, None, addr, addr,
                                ctypes.addressof(ws), 4096, None)
     assert rc == -1
+
+
+def test_sq_dist_rejects_bad_arguments_on_the_host():
+    lib = sa._L()
+    buf = ctypes.create_string_buffer(1024)
+    addr = (ctypes.addressof(buf) + 15) & ~15
+    assert lib.sinkhorn_attn_sq_dist(None, None, -1, sa.SA_F32, None, None) == -1
+    assert lib.sinkhorn_attn_sq_dist(None, None, 0, 7, None, None) == -1
+    assert lib.sinkhorn_attn_sq_dist(None, None, 0, sa.SA_F32, None, None) == -1  # no output
+    # plain host memory is not a device pointer
+    assert lib.sinkhorn_attn_sq_dist(addr, addr, 16, sa.SA_BF16, addr, None) == -1
+
+
+def test_forward_needs_an_iteration():
+    # T = R = 0 is rejected before any pointer is looked at (the backward, which
+    # does not read T, accepts it)
+    lib = sa._L()
+    # B = 0: an empty batch is a no-op that succeeds once the parameters pass
+    assert lib.sinkhorn_attn_fwd(ctypes.byref(P(B=0, T=1, R=0)), *([None] * 8), 1 << 30, None) == 0
+    assert lib.sinkhorn_attn_fwd(ctypes.byref(P(B=0, T=0, R=0)), *([None] * 8), 1 << 30, None) == -1
+    p = P(T=0, R=0)
+    _, b = sa.sinkhorn_attn_workspace_size(p)
+    assert lib.sinkhorn_attn_bwd(ctypes.byref(p), *([None] * 13), b - 1, None) == -3
 
 
 def test_workspace_too_small():

@@ -1,7 +1,7 @@
 """GPU (C ABI, CUDA kernels) vs the CPU oracle on the same seeded inputs.
 
 Small cases cover several row blocks and a ragged tail, the edge cases of the
-method (L = 1, W = 0, dense W >= L, T = 0, R = 1..4, masks with holes, fully
+method (L = 1, W = 0, dense W >= L, T = 0, R = 1..20, masks with holes, fully
 padded sequences, the dustbin), both storage types and both backward
 schedules.  The named workloads run at their full sizes; the two largest are
 compared on a subset of heads (every (batch, head) problem is independent).
@@ -41,6 +41,13 @@ SMALL = [
     (520, 64, 0.6, 4, 3, "bf16", "holes", False),
     (700, 256, 1.0, 2, 4, "bf16", None, False),
     (1000, 37, 0.9, 5, 2, "bf16", (600, 1000), False),
+    # tails longer than one dS sweep's 8 modifier terms: 2, 3 and 5 blocks of
+    # terms summed in fp32; T = 0 with R = N is full backpropagation
+    (150, 9, 0.9, 0, 5, "f32", None, False),
+    (130, 7, 1.0, 1, 9, "f32", "holes", True),
+    (520, 64, 0.6, 0, 5, "bf16", "holes", False),
+    (300, 100, 1.0, 2, 9, "bf16", (180, 300), False),
+    (384, 64, 1.0, 0, 20, "bf16", None, False),
 ]
 
 
