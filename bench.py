@@ -278,6 +278,39 @@ def run_reference(args, w):
     print(json.dumps(line), flush=True)
 
 
+def run_certificate(args, w):
+    """One JSON line: eta_R for the workload's N = T + R iteration solve (full
+    backpropagation as the reference), R*, and the device time it took."""
+    if w.dustbin:
+        raise SystemExit("the bias certificate is defined here without a dustbin")
+    if int(os.environ.get("WORLD_SIZE", "1")) > 1:
+        raise SystemExit("--bias-certificate runs on one GPU")
+    import banded_log_domain_b200 as sa
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    sa.load()
+    _, x = workloads.make(w)
+    dt = torch.float32 if args.cert_dtype == "f32" else torch.bfloat16
+    d = {k: (None if v is None else (v.to(dev) if k == "mask" else v.to(dev).to(dt)))
+         for k, v in x.items() if k in ("q", "k", "v", "dO", "mask")}
+    N = w.T + w.R
+    Rs = tuple(sorted({int(r) for r in args.cert_rs.split(",") if int(r) <= N}))
+    stream = torch.cuda.current_stream(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    eta, sel = sa.bias_certificate(d["q"], d["k"], d["v"], d["dO"], N=N, Rs=Rs, tau=args.cert_tau,
+                                   W=w.W, eps=w.eps, mask=d["mask"], schedule=args.schedule)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    print(json.dumps({
+        "mode": "bias_certificate", "workload": w.name, "N": N, "storage": args.cert_dtype,
+        "schedule": args.schedule, "eta": {str(r): eta[r] for r in Rs}, "tau": args.cert_tau,
+        "R_star": sel, "seconds": round(e0.elapsed_time(e1) / 1e3, 3),
+        "solves": len(Rs) + (0 if N in Rs else 1)}))
+
+
 def config_of(w, args):
     return {"workload": w.name, "B": w.B, "H": w.H, "L": w.L, "d": w.d, "W": w.W, "eps": w.eps,
             "T": w.T, "R": w.R, "storage": w.dtype, "dustbin": w.dustbin,
@@ -299,11 +332,21 @@ def main():
     ap.add_argument("--schedule", default="one_reference", choices=["one_reference", "direct"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--bias-certificate", action="store_true",
+                    help="instead of timing steps, print the bias certificate eta_R of the "
+                         "workload's solve (N = T + R iterations) on one GPU")
+    ap.add_argument("--cert-dtype", default="f32", choices=["f32", "bf16"],
+                    help="storage type for the certificate (f32: the inputs upcast exactly)")
+    ap.add_argument("--cert-rs", default="0,1,2,4,8")
+    ap.add_argument("--cert-tau", type=float, default=1e-5)
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     w = workloads.WORKLOADS[args.workload]
     if args.impl == "reference":
         run_reference(args, w)
+        return
+    if args.bias_certificate:
+        run_certificate(args, w)
         return
 
     ws, rank, local = dist_setup()
