@@ -64,7 +64,7 @@ def _load():
             lib.orc_forward.argtypes = [pp, dp, dp, dp, up, dp, dp, dp, dp, lp]
             lib.orc_forward.restype = ctypes.c_int
             lib.orc_backward.argtypes = [pp, ctypes.c_int, dp, dp, dp, up, dp, dp, dp, dp, dp, dp,
-                                         dp, lp]
+                                         dp, dp, lp]
             lib.orc_backward.restype = ctypes.c_int
             lib.orc_plan.argtypes = [pp, ctypes.c_int, ctypes.c_int, dp, dp, up, dp, dp, dp, dp]
             lib.orc_plan.restype = ctypes.c_int
@@ -151,10 +151,13 @@ def forward(q, k, v, *, W, eps, T, R=2, mask=None, dustbin=False, dustbin_score=
 
 
 def backward(q, k, v, state, dO, *, W, eps, R=2, mask=None, dustbin=False, dustbin_score=-2.0,
-             v_dust=None, schedule="direct", count=False):
+             v_dust=None, schedule="direct", count=False, score_grad=False):
     """Exact surrogate backward.  ``schedule`` is ``"direct"`` (every staircase
     plan by its own exponential) or ``"one_reference"``.  Returns
-    ``(dq, dk, dv, dv_dust)``; ``dv_dust`` is ``[H,d]`` summed over the batch."""
+    ``(dq, dk, dv, dv_dust)``; ``dv_dust`` is ``[H,d]`` summed over the batch.
+    With ``score_grad`` a fifth element follows: the cotangent of the dustbin
+    score (one scalar shared by every problem, so summed over batch and heads;
+    section 2.3 of the gist.science/de summary, one learned dustbin token)."""
     lib = _load()
     q, k, v, dO = _f64(q), _f64(k), _f64(v), _f64(dO)
     st = _f64(state)
@@ -167,22 +170,26 @@ def backward(q, k, v, state, dO, *, W, eps, R=2, mask=None, dustbin=False, dustb
     dv = np.zeros((B, H, L, d))
     dvd = np.zeros((H, d))
     visits = np.zeros((B, H), dtype=np.int64)
+    dsc = 0.0
     p = _params(L, d, W, 0, R, eps, dustbin, dustbin_score)
     for b in range(B):
         for h in range(H):
             cnt = ctypes.c_longlong(0)
             part = np.zeros(d)
+            gs = np.zeros(1)
             rc = lib.orc_backward(
                 ctypes.byref(p), sched, _dp(q[b, h]), _dp(k[b, h]), _dp(v[b, h]),
                 None if m is None else _up(m[b]),
                 None if vd is None else _dp(np.ascontiguousarray(vd[h])),
                 _dp(np.ascontiguousarray(st[b, h])), _dp(dO[b, h]),
-                _dp(dq[b, h]), _dp(dk[b, h]), _dp(dv[b, h]), _dp(part), ctypes.byref(cnt))
+                _dp(dq[b, h]), _dp(dk[b, h]), _dp(dv[b, h]), _dp(part), _dp(gs),
+                ctypes.byref(cnt))
             if rc != 0:
                 raise ValueError("oracle backward rejected its arguments")
             dvd[h] += part
+            dsc += float(gs[0])
             visits[b, h] = cnt.value
-    out = (dq, dk, dv, dvd)
+    out = (dq, dk, dv, dvd) + ((dsc,) if score_grad else ())
     return (out, visits) if count else out
 
 

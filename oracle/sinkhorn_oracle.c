@@ -379,11 +379,16 @@ static void score_vjp(const orc_params* p, const double* q, const double* k, con
  *   dS = A - P^(R,R)*(1 vbar^R^T) - sum_{r=1..R} P^(r,r-1)*(ubar^r 1^T)
  *          - sum_{r=1..R-1} P^(r,r)*(1 vbar^r^T)
  *   dQ = c dS K;  dK = c dS^T Q.
+ * With a dustbin, d_score (if not NULL) receives the cotangent of the dustbin
+ * score (section 2.3: one learned dustbin token): the score enters every
+ * dustbin entry -- column (i, dustbin), row (dustbin, j) and the corner -- with
+ * weight 1, so its cotangent is the sum of dS over those entries, dS as above
+ * (A is zero on the dustbin row, which has no output).
  */
 int orc_backward(const orc_params* p, int schedule, const double* q, const double* k,
                  const double* v, const unsigned char* mask, const double* v_dust,
                  const double* state_in, const double* dO, double* dq, double* dk, double* dv,
-                 double* dv_dust, long long* visits) {
+                 double* dv_dust, double* d_score, long long* visits) {
     if (p->L < 0 || p->d <= 0 || p->W < 0 || p->R < 1 || !(p->eps > 0)) return -1;
     const int L = p->L, d = p->d, W = p->W, bw = band_w(p), n = nd(p), R = p->R;
     double* state = (double*)state_in; /* read only */
@@ -531,6 +536,49 @@ int orc_backward(const orc_params* p, int schedule, const double* q, const doubl
     }
     cnt += support_size(p, mask);
     score_vjp(p, q, k, dS, dq, dk);
+
+    /* the dustbin score's cotangent: dS summed over the dustbin entries.  An
+     * entry is (row i, column j) with i or j equal to L; pref its P^(R,R) value
+     * and a its A value. */
+    if (d_score) {
+        double g = 0.0;
+        if (p->dustbin) {
+            for (int e = 0; e < 2 * L + 1; ++e) {
+                int i, j;
+                double pref, a;
+                if (e < L) {            /* column entry (e, dustbin) */
+                    if (!valid(mask, e)) continue;
+                    i = e; j = L; pref = P.dcol[e]; a = A.dcol[e];
+                } else if (e < 2 * L) { /* row entry (dustbin, e - L) */
+                    if (!valid(mask, e - L)) continue;
+                    i = L; j = e - L; pref = P.drow[j]; a = 0.0;
+                } else {                /* the corner */
+                    i = L; j = L; pref = P.drow[L]; a = 0.0;
+                }
+                double ds;
+                if (schedule == 1) {
+                    ds = a - pref * vbR[j];
+                    for (int r = 1; r <= R; ++r) {
+                        const double pr = (i == L) ? Prr1[r].drow[j] : Prr1[r].dcol[i];
+                        ds -= pr * ub[(size_t)r * n + i];
+                    }
+                    for (int r = 1; r < R; ++r) {
+                        const double pr = (i == L) ? Prr[r].drow[j] : Prr[r].dcol[i];
+                        ds -= pr * vb[(size_t)r * n + j];
+                    }
+                } else {
+                    double M = -vbR[j];
+                    for (int r = 1; r <= R; ++r)
+                        M -= eu[(size_t)r * n + i] * ev[(size_t)(r - 1) * n + j] * ub[(size_t)r * n + i];
+                    for (int r = 1; r < R; ++r)
+                        M -= eu[(size_t)r * n + i] * ev[(size_t)r * n + j] * vb[(size_t)r * n + j];
+                    ds = a + pref * M;
+                }
+                g += ds;
+            }
+        }
+        *d_score = g;
+    }
 
     if (visits) *visits += cnt;
     if (schedule == 1) {

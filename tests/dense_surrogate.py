@@ -36,9 +36,9 @@ def surrogate(q, k, v, *, W, eps, T, R, mask=None, dustbin=False, dustbin_score=
     S = c * (qc @ kc.T)
     sup = (pos[:, None] - pos[None, :]).abs() <= W
     if dustbin:
-        sd = torch.full((n, 1), float(dustbin_score), dtype=q.dtype)
-        S = torch.cat([torch.cat([S, sd], 1),
-                       torch.full((1, n + 1), float(dustbin_score), dtype=q.dtype)], 0)
+        # the score may be a 0-d tensor that requires grad
+        sdt = torch.as_tensor(dustbin_score, dtype=q.dtype)
+        S = torch.cat([torch.cat([S, sdt.expand(n, 1)], 1), sdt.expand(1, n + 1)], 0)
         sup = torch.cat([torch.cat([sup, torch.ones(n, 1, dtype=torch.bool)], 1),
                          torch.ones(1, n + 1, dtype=torch.bool)], 0)
         vd = torch.zeros(1, d, dtype=q.dtype) if v_dust is None else v_dust.reshape(1, d)
@@ -101,3 +101,15 @@ def surrogate_and_grads(q, k, v, dO, *, v_dust=None, **kw):
     dvd = None if vdt is None else vdt.grad.numpy()
     return (o.detach().numpy(), st.detach().numpy(), qt.grad.numpy(), kt.grad.numpy(),
             vt.grad.numpy(), dvd)
+
+
+def dustbin_score_grad(q, k, v, dO, *, dustbin_score, v_dust=None, **kw):
+    """d<dO, O> / d(dustbin score) for one problem by autograd (the stopped base
+    is a constant, as in the surrogate); float64 numpy in, float out."""
+    st = torch.tensor(float(dustbin_score), dtype=torch.float64, requires_grad=True)
+    vd = None if v_dust is None else torch.tensor(v_dust, dtype=torch.float64)
+    o, _ = surrogate(torch.tensor(q, dtype=torch.float64), torch.tensor(k, dtype=torch.float64),
+                     torch.tensor(v, dtype=torch.float64), dustbin=True, dustbin_score=st,
+                     v_dust=vd, **kw)
+    (o * torch.tensor(dO, dtype=torch.float64)).sum().backward()
+    return float(st.grad)

@@ -296,6 +296,66 @@ def test_frozen_base_finite_differences(oracle_mod, d, dustbin):
         assert abs(fd - an) <= 1e-7 * max(1.0, abs(an)), (fd, an)
 
 
+# --------------------------------------------------------------------------
+# the dustbin score's cotangent (one learned dustbin token, gist.science/de
+# section 2.3): the sum of dS over the dustbin column, row and corner
+# --------------------------------------------------------------------------
+
+DSCORE_CASES = [
+    # (L, d, W, eps, T, R, mask_kind)
+    (18, 4, 3, 0.7, 3, 2, None),
+    (26, 8, 4, 0.6, 4, 2, "holes"),
+    (15, 4, 20, 1.0, 2, 1, None),     # W >= L: dense
+    (21, 4, 3, 0.8, 2, 3, "holes"),
+    (16, 4, 2, 0.9, 0, 2, None),      # T = 0
+]
+
+
+@pytest.mark.parametrize("case", DSCORE_CASES)
+def test_dustbin_score_cotangent_matches_autograd(oracle_mod, case):
+    L, d, W, eps, T, R, mk = case
+    q, k, v, dO, mask = _rand(1, 2, L, d, seed=3 * L + W, mask_kind=mk)
+    vd = np.random.default_rng(L + 1).normal(size=(2, d))
+    sc = -0.9
+    kw = dict(W=W, eps=eps, R=R, dustbin=True, dustbin_score=sc)
+    o, st = oracle_mod.forward(q, k, v, T=T, mask=mask, v_dust=vd, **kw)
+    m = None if mask is None else mask[0].numpy()
+    ref = sum(ds.dustbin_score_grad(q[0, h], k[0, h], v[0, h], dO[0, h], v_dust=vd[h], W=W,
+                                    eps=eps, T=T, R=R, mask=m, dustbin_score=sc)
+              for h in range(2))
+    assert abs(ref) > 1e-3  # the pin has something to check
+    for s in ("direct", "one_reference"):
+        g = oracle_mod.backward(q, k, v, st, dO, mask=mask, v_dust=vd, schedule=s,
+                                score_grad=True, **kw)[4]
+        assert abs(g - ref) <= 1e-10 * max(1.0, abs(ref)), (s, g, ref)
+
+
+def test_dustbin_score_cotangent_finite_differences(oracle_mod):
+    """Central difference of F = <dO, O> in the dustbin score, the stopped base
+    held at its unperturbed value."""
+    L, d, W, eps, T, R = 22, 8, 3, 0.8, 4, 2
+    q, k, v, dO, mask = _rand(2, 2, L, d, seed=77, mask_kind="holes")
+    vd = np.random.default_rng(5).normal(size=(2, d))
+    sc, h = -1.1, 1e-5
+    kw = dict(W=W, eps=eps, R=R, mask=mask, dustbin=True, v_dust=vd)
+    o, st = oracle_mod.forward(q, k, v, T=T, dustbin_score=sc, **kw)
+    base = st[:, :, 0:2].copy()
+    g = oracle_mod.backward(q, k, v, st, dO, dustbin_score=sc, score_grad=True, **kw)[4]
+
+    def F(s):
+        oo, _ = oracle_mod.forward(q, k, v, T=T, base=base, dustbin_score=s, **kw)
+        return float((oo * dO).sum())
+
+    fd = (F(sc + h) - F(sc - h)) / (2 * h)
+    assert abs(fd - g) <= 1e-7 * max(1.0, abs(g)), (fd, g)
+
+
+def test_dustbin_score_cotangent_is_zero_without_a_dustbin(oracle_mod):
+    q, k, v, dO, mask = _rand(1, 1, 12, 4, seed=2)
+    o, st = oracle_mod.forward(q, k, v, W=2, eps=1.0, T=2, R=2)
+    assert oracle_mod.backward(q, k, v, st, dO, W=2, eps=1.0, R=2, score_grad=True)[4] == 0.0
+
+
 def test_one_reference_equals_direct(oracle_mod):
     q, k, v, dO, mask = _rand(2, 2, 90, 16, seed=31, valid_len=(60, 90))
     kw = dict(W=9, eps=0.5, R=2, mask=mask)
