@@ -93,10 +93,10 @@ def _L():
     lib.sinkhorn_attn_state_size.argtypes = [P, ctypes.POINTER(sz)]
     lib.sinkhorn_attn_workspace_size.argtypes = [P, ctypes.POINTER(sz), ctypes.POINTER(sz)]
     lib.sinkhorn_attn_fwd.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
-    lib.sinkhorn_attn_bwd.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz,
-                                      vp]
+    lib.sinkhorn_attn_bwd.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp,
+                                      sz, vp]
     lib.sinkhorn_attn_bwd_static_ws.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp,
-                                                vp, vp]
+                                                vp, vp, vp]
     lib.sinkhorn_attn_bwd_static_ws.restype = ctypes.c_int
     lib.sinkhorn_attn_debug_plan.argtypes = [P, ctypes.c_int, ctypes.c_int, vp, vp, vp, vp, vp,
                                              vp, vp, vp]
@@ -201,10 +201,13 @@ def sinkhorn_attn_fwd(q, k, v, *, W, eps, T, R=2, mask=None, dustbin=False, dust
 
 def sinkhorn_attn_bwd(q, k, v, o, dO, state, *, W, eps, R=2, mask=None, dustbin=False,
                       dustbin_score=-2.0, v_dust=None, schedule="one_reference", dq=None, dk=None,
-                      dv=None, dv_dust=None, ws=None, check_finite=False, trace=None):
+                      dv=None, dv_dust=None, d_dust_score=None, ws=None, check_finite=False,
+                      trace=None):
     """Backward of <dO, O> through the tail.  Returns ``(dq, dk, dv, dv_dust)``
-    (``dv_dust`` is ``[H,64]`` float32 when ``dustbin``, else None)."""
-    _contig(q, k, v, o, dO, state, mask, v_dust, dq, dk, dv, dv_dust, ws)
+    (``dv_dust`` is ``[H,64]`` float32 when ``dustbin``, else None).  With a
+    dustbin, a one-element float32 CUDA tensor ``d_dust_score`` receives the
+    cotangent of ``dustbin_score`` (summed over batch and heads)."""
+    _contig(q, k, v, o, dO, state, mask, v_dust, dq, dk, dv, dv_dust, d_dust_score, ws)
     p = _params_for(q, W, eps, 0, R, dustbin, dustbin_score, schedule, check_finite)
     if trace is not None:
         trace.attach(p)
@@ -218,8 +221,9 @@ def sinkhorn_attn_bwd(q, k, v, o, dO, state, *, W, eps, R=2, mask=None, dustbin=
         ws = torch.zeros(sinkhorn_attn_workspace_size(p)[1], dtype=torch.uint8, device=dev)
     rc = _L().sinkhorn_attn_bwd(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(mask),
                                 _ptr(v_dust), _ptr(o), _ptr(dO), _ptr(state), _ptr(dq), _ptr(dk),
-                                _ptr(dv), _ptr(dv_dust if dustbin else None), _ptr(ws),
-                                ws.numel(), _stream(dev))
+                                _ptr(dv), _ptr(dv_dust if dustbin else None),
+                                _ptr(d_dust_score if dustbin else None), _ptr(ws), ws.numel(),
+                                _stream(dev))
     _check(rc, "sinkhorn_attn_bwd")
     return dq, dk, dv, (dv_dust if dustbin else None)
 
@@ -230,14 +234,15 @@ STATIC_SCRATCH_BYTES = 32 << 20
 def sinkhorn_attn_bwd_static_ws(q, k, v, o, dO, state, *, W, eps, R=2, mask=None,
                                 dustbin=False, dustbin_score=-2.0, v_dust=None,
                                 schedule="one_reference", dq=None, dk=None, dv=None,
-                                dv_dust=None, trace=None):
+                                dv_dust=None, d_dust_score=None, trace=None):
     """Backward that takes no workspace: for callers that cannot allocate
     device memory where they run it (see ``sinkhorn_attn_bwd_static_ws`` in
     the C header).  The library's fixed scratch array (``STATIC_SCRATCH_BYTES``
     per GPU) is used instead; calls that overlap on the GPU race.  Pass
     preallocated ``dq, dk, dv`` (and ``dv_dust``) to keep the call free of
-    allocations on the Python side too."""
-    _contig(q, k, v, o, dO, state, mask, v_dust, dq, dk, dv, dv_dust)
+    allocations on the Python side too.  ``d_dust_score`` as in
+    :func:`sinkhorn_attn_bwd`."""
+    _contig(q, k, v, o, dO, state, mask, v_dust, dq, dk, dv, dv_dust, d_dust_score)
     p = _params_for(q, W, eps, 0, R, dustbin, dustbin_score, schedule, False)
     if trace is not None:
         trace.attach(p)
@@ -250,7 +255,7 @@ def sinkhorn_attn_bwd_static_ws(q, k, v, o, dO, state, *, W, eps, R=2, mask=None
     rc = _L().sinkhorn_attn_bwd_static_ws(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(mask),
                                           _ptr(v_dust), _ptr(o), _ptr(dO), _ptr(state), _ptr(dq),
                                           _ptr(dk), _ptr(dv), _ptr(dv_dust if dustbin else None),
-                                          _stream(dev))
+                                          _ptr(d_dust_score if dustbin else None), _stream(dev))
     _check(rc, "sinkhorn_attn_bwd_static_ws")
     return dq, dk, dv, (dv_dust if dustbin else None)
 

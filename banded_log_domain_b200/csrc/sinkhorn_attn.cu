@@ -86,6 +86,17 @@ bool device_ok(const void* x) {
     return at.type == cudaMemoryTypeDevice || at.type == cudaMemoryTypeManaged ||
            at.type == cudaMemoryTypeHost;
 }
+// A device float that may sit anywhere a float may (4-byte alignment).
+bool device_f32_ok(const void* x) {
+    if (!x || ((uintptr_t)x & 3u)) return false;
+    cudaPointerAttributes at;
+    if (cudaPointerGetAttributes(&at, x) != cudaSuccess) {
+        cudaGetLastError();
+        return false;
+    }
+    return at.type == cudaMemoryTypeDevice || at.type == cudaMemoryTypeManaged ||
+           at.type == cudaMemoryTypeHost;
+}
 bool mask_ok(const void* x) {
     if (!x) return true;
     cudaPointerAttributes at;
@@ -128,7 +139,7 @@ FwdLayout fwd_layout(const Dims& d, const sa_params* p) {
 
 // Backward workspace layout (float32 vectors of BH * ld elements each).
 struct BwdLayout {
-    size_t a, ubar, vbar, eu, ev, w, rv, cv, dvd, acc, total;
+    size_t a, ubar, vbar, eu, ev, w, rv, cv, dvd, dsc, acc, total;
     size_t vec;  // bytes of one [BH][ld] vector, 256-aligned
 };
 BwdLayout bwd_layout(const Dims& d) {
@@ -144,6 +155,7 @@ BwdLayout bwd_layout(const Dims& d) {
     l.rv = o;   o += l.vec * 2 * d.R;
     l.cv = o;   o += l.vec * 2 * d.R;
     l.dvd = o;  o += align_up((size_t)d.BH * kD * sizeof(float));
+    l.dsc = o;  o += align_up((size_t)d.BH * sizeof(double));  // dustbin score, per problem
     l.acc = o;  // fp32 sum of the dS sweeps' term blocks, when 2R > MAXT
     if (2 * d.R > simt::MAXT) o += align_up((size_t)d.BH * d.L * kD * sizeof(float));
     l.total = o;
@@ -216,6 +228,72 @@ __global__ void k_dvd_reduce(const float* part, int B, int H, float* out) {
     float s = 0.f;
     for (int b = 0; b < B; ++b) s += part[((size_t)b * H + h) * kD + e];
     out[g] = s;
+}
+
+// Cotangent of the dustbin score (one learned dustbin token): the score enters
+// every dustbin entry -- column (i, L), row (L, j) and the corner (L, L) -- so
+// its cotangent is the sum of dS over them, each entry's staircase plans formed
+// by their own exponential:
+//   dS_e = P^(R,R)_e (G_e - vbar^R_col) - sum_{r=1..R} P^(r,r-1)_e ubar^r_row
+//          - sum_{r=1..R-1} P^(r,r)_e vbar^r_col,   P^(a,b)_e = exp(s + u^(a)_row + v^(b)_col)
+// with G_(i,L) = <dO_i, v_dust> and G = 0 on the dustbin row (it has no
+// output).  R = 0 keeps every dual constant: dS_e = P_e G_e.  The entries
+// cancel to a remainder far smaller than their sizes, so the sums run in
+// double.  One block per problem writes its sum to part[bh]; ubar/vbar hold
+// index r at r * rs floats.
+template <typename T>
+__global__ void k_dscore(const T* dO, const float* v_dust, const uint8_t* mask,
+                         const float* state, const float* ubar, const float* vbar, size_t rs,
+                         int R, int L, int H, int ld, float sd, double* part) {
+    const int bh = blockIdx.x, b = bh / H, h = bh % H;
+    const float* st = state + (size_t)bh * (2 * R + 2) * ld;
+    auto U = [&](int a, int t) { return st[(size_t)(2 * a) * ld + t]; };
+    auto V = [&](int a, int t) { return st[(size_t)(2 * a + 1) * ld + t]; };
+    auto UB = [&](int r, int t) { return ubar[(size_t)r * rs + (size_t)bh * ld + t]; };
+    auto VB = [&](int r, int t) { return vbar[(size_t)r * rs + (size_t)bh * ld + t]; };
+    // dS at (row i, column j) without the A term
+    auto ds_tail = [&](int i, int j) {
+        if (R == 0) return 0.0;
+        double g = -(double)expf(sd + U(R, i) + V(R, j)) * VB(R, j);
+        for (int r = 1; r <= R; ++r) g -= (double)expf(sd + U(r, i) + V(r - 1, j)) * UB(r, i);
+        for (int r = 1; r < R; ++r) g -= (double)expf(sd + U(r, i) + V(r, j)) * VB(r, j);
+        return g;
+    };
+    double acc = 0.0;
+    for (int t = threadIdx.x; t < L; t += blockDim.x) {
+        if (mask && !mask[(size_t)b * L + t]) continue;
+        float gi = 0.f;  // <dO_t, v_dust>
+        if (v_dust) {
+            const T* row = dO + ((size_t)bh * L + t) * kD;
+            const float* vd = v_dust + (size_t)h * kD;
+            for (int e = 0; e < kD; ++e) gi = fmaf(to_f32(row[e]), vd[e], gi);
+        }
+        acc += (double)expf(sd + U(R, t) + V(R, L)) * gi + ds_tail(t, L) + ds_tail(L, t);
+    }
+    if (threadIdx.x == 0) acc += ds_tail(L, L);
+    __shared__ double red[32];
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = acc;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        double sum = 0.0;
+        for (int w = 0; w < (int)(blockDim.x >> 5); ++w) sum += red[w];
+        part[bh] = sum;
+    }
+}
+
+// out[0] = sum of part[0..n) in a fixed order (one block of 256 threads).
+__global__ void k_sum_parts(const double* part, int n, float* out) {
+    __shared__ double red[256];
+    double s = 0.0;
+    for (int i = threadIdx.x; i < n; i += blockDim.x) s += part[i];
+    red[threadIdx.x] = s;
+    __syncthreads();
+    for (int w = blockDim.x / 2; w > 0; w >>= 1) {
+        if ((int)threadIdx.x < w) red[threadIdx.x] += red[threadIdx.x + w];
+        __syncthreads();
+    }
+    if (threadIdx.x == 0) out[0] = (float)red[0];
 }
 
 // out[0] += sum_i (x_i - y_i)^2, out[1] += sum_i y_i^2 in double: grid-stride
@@ -607,7 +685,7 @@ sa_status fwd_fused(const Ctx& x, const __nv_bfloat16* q, const __nv_bfloat16* k
 template <typename T>
 sa_status bwd_impl(const Ctx& x, const T* q, const T* k, const T* v, const uint8_t* mask,
                    const float* v_dust, const T* o, const T* dO, T* dq, T* dk, T* dv,
-                   float* dv_dust, char* ws) {
+                   float* dv_dust, float* d_score, char* ws) {
     const Dims& d = x.d;
     const int R = d.R;
     const BwdLayout l = bwd_layout(d);
@@ -781,6 +859,13 @@ sa_status bwd_impl(const Ctx& x, const T* q, const T* k, const T* v, const uint8
         SA_AUX(x.tr, k_dvd_reduce<<<(d.H * kD + 255) / 256, 256, 0, x.st>>>(dvd, d.B, d.H,
                                                                             dv_dust));
     }
+    if (x.p->dustbin && d_score) {
+        double* part = (double*)(ws + l.dsc);
+        SA_AUX(x.tr, k_dscore<T><<<d.BH, 256, 0, x.st>>>(dO, v_dust, mask, x.state, W_(l.ubar, 0),
+                                                         W_(l.vbar, 0), vstride, R, d.L, d.H,
+                                                         d.ld, x.p->dustbin_score, part));
+        SA_AUX(x.tr, k_sum_parts<<<1, 256, 0, x.st>>>(part, d.BH, d_score));
+    }
     return SA_OK;
 }
 
@@ -869,7 +954,8 @@ sa_status sinkhorn_attn_fwd(const sa_params* p, const void* q, const void* k, co
 sa_status sinkhorn_attn_bwd(const sa_params* p, const void* q, const void* k, const void* v,
                             const uint8_t* mask, const float* v_dust, const void* o,
                             const void* dO, const float* state, void* dq, void* dk, void* dv,
-                            float* dv_dust, void* ws, size_t ws_bytes, void* stream) {
+                            float* dv_dust, float* d_dust_score, void* ws, size_t ws_bytes,
+                            void* stream) {
     Dims d;
     sa_status s = check_params(p, &d);
     if (s != SA_OK) return s;
@@ -881,6 +967,7 @@ sa_status sinkhorn_attn_bwd(const sa_params* p, const void* q, const void* k, co
         return SA_ERR_INVALID_ARG;
     if (p->dustbin && v_dust && !device_ok(v_dust)) return SA_ERR_INVALID_ARG;
     if (p->dustbin && dv_dust && !device_ok(dv_dust)) return SA_ERR_INVALID_ARG;
+    if (p->dustbin && d_dust_score && !device_f32_ok(d_dust_score)) return SA_ERR_INVALID_ARG;
     Ctx x;
     x.p = p;
     x.d = d;
@@ -893,15 +980,16 @@ sa_status sinkhorn_attn_bwd(const sa_params* p, const void* q, const void* k, co
     x.tr.st = x.st;
     const float* vd = p->dustbin ? v_dust : nullptr;
     float* dvd = p->dustbin ? dv_dust : nullptr;
+    float* dsc = p->dustbin ? d_dust_score : nullptr;
     if (p->dtype == SA_F32)
         s = bwd_impl<float>(x, (const float*)q, (const float*)k, (const float*)v, mask, vd,
                             (const float*)o, (const float*)dO, (float*)dq, (float*)dk, (float*)dv,
-                            dvd, (char*)ws);
+                            dvd, dsc, (char*)ws);
     else
         s = bwd_impl<__nv_bfloat16>(
             x, (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v, mask, vd,
             (const __nv_bfloat16*)o, (const __nv_bfloat16*)dO, (__nv_bfloat16*)dq,
-            (__nv_bfloat16*)dk, (__nv_bfloat16*)dv, dvd, (char*)ws);
+            (__nv_bfloat16*)dk, (__nv_bfloat16*)dv, dvd, dsc, (char*)ws);
     if (s != SA_OK) return s;
     if (p->check_finite) {
         int* status = (int*)ws;
@@ -955,7 +1043,7 @@ sa_status sinkhorn_attn_bwd_static_ws(const sa_params* p, const void* q, const v
                                       const void* v, const uint8_t* mask, const float* v_dust,
                                       const void* o, const void* dO, const float* state,
                                       void* dq, void* dk, void* dv, float* dv_dust,
-                                      void* stream) {
+                                      float* d_dust_score, void* stream) {
     Dims d;
     sa_status s = check_params(p, &d);
     if (s != SA_OK) return s;
@@ -969,6 +1057,7 @@ sa_status sinkhorn_attn_bwd_static_ws(const sa_params* p, const void* q, const v
         return SA_ERR_INVALID_ARG;
     if (p->dustbin && v_dust && !device_ok(v_dust)) return SA_ERR_INVALID_ARG;
     if (p->dustbin && dv_dust && !device_ok(dv_dust)) return SA_ERR_INVALID_ARG;
+    if (p->dustbin && d_dust_score && !device_f32_ok(d_dust_score)) return SA_ERR_INVALID_ARG;
     void* ws = nullptr;
     s = bwd_scratch_current_device(&ws);
     if (s != SA_OK) return s;
@@ -987,14 +1076,15 @@ sa_status sinkhorn_attn_bwd_static_ws(const sa_params* p, const void* q, const v
     x.tr.st = st;
     const float* vd = p->dustbin ? v_dust : nullptr;
     float* dvd = p->dustbin ? dv_dust : nullptr;
+    float* dsc = p->dustbin ? d_dust_score : nullptr;
     if (p->dtype == SA_F32)
         return bwd_impl<float>(x, (const float*)q, (const float*)k, (const float*)v, mask, vd,
                                (const float*)o, (const float*)dO, (float*)dq, (float*)dk,
-                               (float*)dv, dvd, (char*)ws);
+                               (float*)dv, dvd, dsc, (char*)ws);
     return bwd_impl<__nv_bfloat16>(
         x, (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v, mask, vd,
         (const __nv_bfloat16*)o, (const __nv_bfloat16*)dO, (__nv_bfloat16*)dq,
-        (__nv_bfloat16*)dk, (__nv_bfloat16*)dv, dvd, (char*)ws);
+        (__nv_bfloat16*)dk, (__nv_bfloat16*)dv, dvd, dsc, (char*)ws);
 }
 
 sa_status sinkhorn_attn_debug_plan(const sa_params* p, int a, int b, const void* q,

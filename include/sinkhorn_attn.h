@@ -132,21 +132,31 @@ sa_status sinkhorn_attn_fwd(const sa_params* p, const void* q, const void* k, co
                             void* ws, size_t ws_bytes, void* stream);
 
 /*
- * Backward: dQ, dK, dV (and the dustbin value gradient) of <dO, O> through the
- * R-step tail, the stopped base held constant (section 2.2).
+ * Backward: dQ, dK, dV (and the dustbin's value and score gradients) of
+ * <dO, O> through the R-step tail, the stopped base held constant (section 2.2;
+ * the dustbin token of section 2.3 is learned: its value vector and its score).
  *   q, k, v, mask, v_dust : as given to the forward.
  *   o, state              : the forward's outputs.
  *   dO                    : [B][H][L][d] dtype, device.
  *   dq, dk, dv            : [B][H][L][d] dtype, device, written.
  *   dv_dust               : [H][d] float32, device, written (summed over the
  *                           batch), or NULL; used only when p->dustbin.
+ *   d_dust_score          : one float32, device (4-byte aligned), written with
+ *                           the cotangent of p->dustbin_score summed over every
+ *                           (batch, head) problem, or NULL; used only when
+ *                           p->dustbin.  The score enters every dustbin entry
+ *                           (column, row, corner), so this is the sum of the
+ *                           score cotangent over them, each staircase plan on
+ *                           those O(L) entries formed by its own exponential
+ *                           whatever the schedule.
  *   ws                    : workspace of ws_bytes >= bwd_bytes, device.
  * The schedule is p->bwd.
  */
 sa_status sinkhorn_attn_bwd(const sa_params* p, const void* q, const void* k, const void* v,
                             const uint8_t* mask, const float* v_dust, const void* o,
                             const void* dO, const float* state, void* dq, void* dk, void* dv,
-                            float* dv_dust, void* ws, size_t ws_bytes, void* stream);
+                            float* dv_dust, float* d_dust_score, void* ws, size_t ws_bytes,
+                            void* stream);
 
 /*
  * Test hook: the plan P^(a,b) (0 <= a, b <= R) from a finished forward state.
@@ -188,7 +198,7 @@ sa_status sinkhorn_attn_bwd_static_ws(const sa_params* p, const void* q, const v
                                       const void* v, const uint8_t* mask, const float* v_dust,
                                       const void* o, const void* dO, const float* state,
                                       void* dq, void* dk, void* dv, float* dv_dust,
-                                      void* stream);
+                                      float* d_dust_score, void* stream);
 
 /* Synchronises `stream`, then returns the status word recorded in `ws` by the
  * last forward/backward that used it (SA_OK, SA_ERR_NONFINITE or

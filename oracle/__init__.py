@@ -151,13 +151,15 @@ def forward(q, k, v, *, W, eps, T, R=2, mask=None, dustbin=False, dustbin_score=
 
 
 def backward(q, k, v, state, dO, *, W, eps, R=2, mask=None, dustbin=False, dustbin_score=-2.0,
-             v_dust=None, schedule="direct", count=False, score_grad=False):
+             v_dust=None, schedule="direct", count=False, score_grad=False, score_scale=False):
     """Exact surrogate backward.  ``schedule`` is ``"direct"`` (every staircase
     plan by its own exponential) or ``"one_reference"``.  Returns
     ``(dq, dk, dv, dv_dust)``; ``dv_dust`` is ``[H,d]`` summed over the batch.
     With ``score_grad`` a fifth element follows: the cotangent of the dustbin
     score (one scalar shared by every problem, so summed over batch and heads;
-    section 2.3 of the gist.science/de summary, one learned dustbin token)."""
+    section 2.3 of the gist.science/de summary, one learned dustbin token);
+    with ``score_scale`` also a sixth, the sum of |dS| over the dustbin entries
+    (the size of what cancels in the fifth: an error scale for comparisons)."""
     lib = _load()
     q, k, v, dO = _f64(q), _f64(k), _f64(v), _f64(dO)
     st = _f64(state)
@@ -170,13 +172,13 @@ def backward(q, k, v, state, dO, *, W, eps, R=2, mask=None, dustbin=False, dustb
     dv = np.zeros((B, H, L, d))
     dvd = np.zeros((H, d))
     visits = np.zeros((B, H), dtype=np.int64)
-    dsc = 0.0
+    dsc = dabs = 0.0
     p = _params(L, d, W, 0, R, eps, dustbin, dustbin_score)
     for b in range(B):
         for h in range(H):
             cnt = ctypes.c_longlong(0)
             part = np.zeros(d)
-            gs = np.zeros(1)
+            gs = np.zeros(2)
             rc = lib.orc_backward(
                 ctypes.byref(p), sched, _dp(q[b, h]), _dp(k[b, h]), _dp(v[b, h]),
                 None if m is None else _up(m[b]),
@@ -188,8 +190,9 @@ def backward(q, k, v, state, dO, *, W, eps, R=2, mask=None, dustbin=False, dustb
                 raise ValueError("oracle backward rejected its arguments")
             dvd[h] += part
             dsc += float(gs[0])
+            dabs += float(gs[1])
             visits[b, h] = cnt.value
-    out = (dq, dk, dv, dvd) + ((dsc,) if score_grad else ())
+    out = (dq, dk, dv, dvd) + ((dsc,) if score_grad else ()) + ((dabs,) if score_scale else ())
     return (out, visits) if count else out
 
 

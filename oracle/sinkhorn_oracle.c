@@ -379,11 +379,13 @@ static void score_vjp(const orc_params* p, const double* q, const double* k, con
  *   dS = A - P^(R,R)*(1 vbar^R^T) - sum_{r=1..R} P^(r,r-1)*(ubar^r 1^T)
  *          - sum_{r=1..R-1} P^(r,r)*(1 vbar^r^T)
  *   dQ = c dS K;  dK = c dS^T Q.
- * With a dustbin, d_score (if not NULL) receives the cotangent of the dustbin
- * score (section 2.3: one learned dustbin token): the score enters every
- * dustbin entry -- column (i, dustbin), row (dustbin, j) and the corner -- with
- * weight 1, so its cotangent is the sum of dS over those entries, dS as above
- * (A is zero on the dustbin row, which has no output).
+ * With a dustbin, d_score (if not NULL, two doubles) receives in d_score[0]
+ * the cotangent of the dustbin score (section 2.3: one learned dustbin token):
+ * the score enters every dustbin entry -- column (i, dustbin), row
+ * (dustbin, j) and the corner -- with weight 1, so its cotangent is the sum of
+ * dS over those entries, dS as above (A is zero on the dustbin row, which has
+ * no output).  d_score[1] = the sum of |dS| over the same entries, the size
+ * of what cancels in d_score[0] (an error scale for comparisons).
  */
 int orc_backward(const orc_params* p, int schedule, const double* q, const double* k,
                  const double* v, const unsigned char* mask, const double* v_dust,
@@ -541,7 +543,7 @@ int orc_backward(const orc_params* p, int schedule, const double* q, const doubl
      * entry is (row i, column j) with i or j equal to L; pref its P^(R,R) value
      * and a its A value. */
     if (d_score) {
-        double g = 0.0;
+        double g = 0.0, gabs = 0.0;
         if (p->dustbin) {
             for (int e = 0; e < 2 * L + 1; ++e) {
                 int i, j;
@@ -575,9 +577,11 @@ int orc_backward(const orc_params* p, int schedule, const double* q, const doubl
                     ds = a + pref * M;
                 }
                 g += ds;
+                gabs += fabs(ds);
             }
         }
-        *d_score = g;
+        d_score[0] = g;
+        d_score[1] = gabs;
     }
 
     if (visits) *visits += cnt;

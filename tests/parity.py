@@ -12,6 +12,10 @@ Tolerances (the stated contract of this library):
   * O, dQ, dK, dV, dv_dust: relative l2 (||x - y|| / ||y|| over the compared
     elements) 1e-4 for fp32 storage, 2e-2 for bf16 storage (the outputs are
     rounded to bf16, whose unit roundoff is 2^-8);
+  * the dustbin score's cotangent (a scalar): the larger of the relative bound
+    above and SCORE_ROUND times sum |dS_e|, the total size of the
+    dustbin-entry cotangents it sums; they cancel down to a remainder 10^3 to
+    10^4 times smaller on these random inputs, so its error follows their size;
   * the support (which plan entries are non-zero) and the zeros of masked
     tokens: exact.
 """
@@ -25,6 +29,10 @@ import workloads
 
 DUAL_ATOL = {"f32": 1e-5, "bf16": 2e-3}
 REL_L2 = {"f32": 1e-4, "bf16": 2e-2}
+# relative accuracy of the inputs of the dustbin-entry cotangents: fp32 duals
+# and vector cotangents (about 1e-6); with bf16 storage the row dot <dO, O>
+# reads O rounded to 2^-9, averaged over 64 dimensions
+SCORE_ROUND = {"f32": 2.0 ** -20, "bf16": 2.0 ** -12}
 
 
 def rel_l2(x, y):
@@ -50,11 +58,12 @@ def gpu_run(x, *, W, eps, T, R, dustbin=False, dustbin_score=-2.0, schedules=("o
                                  v_dust=d["v_dust"])
     out = {"o": o, "state": st}
     for s in schedules:
+        dsc = torch.full((1,), float("nan"), dtype=torch.float32, device="cuda") if dustbin else None
         dq, dk, dv, dvd = sa.sinkhorn_attn_bwd(d["q"], d["k"], d["v"], o, d["dO"], st, W=W,
                                                eps=eps, R=R, mask=d["mask"], dustbin=dustbin,
                                                dustbin_score=dustbin_score, v_dust=d["v_dust"],
-                                               schedule=s)
-        out[s] = (dq, dk, dv, dvd)
+                                               schedule=s, d_dust_score=dsc)
+        out[s] = (dq, dk, dv, dvd, dsc)
     for (a, b) in plans:
         out[("plan", a, b)] = sa.sinkhorn_attn_debug_plan(d["q"], d["k"], st, a, b, W=W, eps=eps,
                                                           R=R, mask=d["mask"], dustbin=dustbin,
@@ -80,7 +89,8 @@ def oracle_run(x, *, W, eps, T, R, dustbin=False, dustbin_score=-2.0, plans=(), 
         vd = vd[heads]
     kw = dict(W=W, eps=eps, R=R, mask=x["mask"], dustbin=dustbin, dustbin_score=dustbin_score)
     o, st = oracle.forward(q, k, v, T=T, v_dust=vd, **kw)
-    g = oracle.backward(q, k, v, st, dO, v_dust=vd, schedule="direct", **kw)
+    g = oracle.backward(q, k, v, st, dO, v_dust=vd, schedule="direct", score_grad=True,
+                        score_scale=True, **kw)
     out = {"o": o, "state": st, "grads": g}
     for (a, b) in plans:
         out[("plan", a, b)] = oracle.plan(q, k, st, a, b, **kw)
@@ -121,9 +131,9 @@ def compare(x, g, r, *, dtype, dustbin, schedules=("one_reference",), heads=None
     e = rel_l2(go[mo], ro[mo])
     assert e <= tol, f"{label} O rel-l2 {e}"
     assert np.all(go[~mo] == 0), f"{label} masked O not zero"
-    rdq, rdk, rdv, rdvd = r["grads"]
+    rdq, rdk, rdv, rdvd, rdsc, rdabs = r["grads"]
     for s in schedules:
-        gdq, gdk, gdv, gdvd = g[s]
+        gdq, gdk, gdv, gdvd, gdsc = g[s]
         for name, gt, rt in (("dQ", gdq, rdq), ("dK", gdk, rdk), ("dV", gdv, rdv)):
             gt = gt[:, hs][:, :, rs]
             rt = rt[:, :, rs]
@@ -133,6 +143,13 @@ def compare(x, g, r, *, dtype, dustbin, schedules=("one_reference",), heads=None
         if dustbin and rows is None and heads is None:
             e = rel_l2(gdvd, rdvd)
             assert e <= max(tol, 1e-4) or np.abs(rdvd).max() == 0, f"{label} dv_dust rel-l2 {e}"
+            # the dustbin score's cotangent: one scalar summed over every problem,
+            # the small remainder of dustbin-entry cotangents that cancel, so its
+            # error scales with their total size sum |dS_e| (with bf16 storage
+            # the row dot <dO, O> also reads the rounded O)
+            gs, rs_ = float(gdsc[0]), float(rdsc)
+            bound = max(tol * abs(rs_), SCORE_ROUND[dtype] * rdabs)
+            assert abs(gs - rs_) <= bound, f"{label} {s} d_score {gs} vs {rs_} (bound {bound})"
 
 
 def compare_plans(g, r, plans, *, dtype="f32", heads=None, label=""):

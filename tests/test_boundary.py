@@ -122,14 +122,14 @@ def test_forward_needs_an_iteration():
     assert lib.sinkhorn_attn_fwd(ctypes.byref(P(B=0, T=0, R=0)), *([None] * 8), 1 << 30, None) == -1
     p = P(T=0, R=0)
     _, b = sa.sinkhorn_attn_workspace_size(p)
-    assert lib.sinkhorn_attn_bwd(ctypes.byref(p), *([None] * 13), b - 1, None) == -3
+    assert lib.sinkhorn_attn_bwd(ctypes.byref(p), *([None] * 14), b - 1, None) == -3
 
 
 def test_workspace_too_small():
     lib = sa._L()
     p = P()
     _, b = sa.sinkhorn_attn_workspace_size(p)
-    rc = lib.sinkhorn_attn_bwd(ctypes.byref(p), *([None] * 13), b - 1, None)
+    rc = lib.sinkhorn_attn_bwd(ctypes.byref(p), *([None] * 14), b - 1, None)
     assert rc == -3
     rc = lib.sinkhorn_attn_fwd(ctypes.byref(p), *([None] * 8), 16, None)
     assert rc == -3

@@ -64,6 +64,33 @@ def test_tail_depth_zero(case):
             assert np.all(np_(gt)[~mo] == 0), f"{s} masked {name} not zero"
 
 
+def test_tail_depth_zero_dustbin_gradients():
+    # every dual constant: dv_dust = sum_i P_(i,dustbin) dO_i and the score's
+    # cotangent sum_i P_(i,dustbin) <dO_i, v_dust> (G is zero on the dustbin row)
+    import banded_log_domain_b200 as sa
+
+    L, W, eps, N, B, H = 150, 9, 0.8, 4, 2, 2
+    x = parity.draw_case(B, H, L, dtype="f32", seed=19, mask_kind="holes", dustbin=True,
+                         v_dust_random=True)
+    d = parity.to_dev(x)
+    kw = dict(W=W, eps=eps, dustbin=True, dustbin_score=-1.4)
+    o, st = sa.sinkhorn_attn_fwd(d["q"], d["k"], d["v"], T=N, R=0, mask=d["mask"],
+                                 v_dust=d["v_dust"], **kw)
+    dsc = torch.zeros(1, dtype=torch.float32, device="cuda")
+    _, _, _, dvd = sa.sinkhorn_attn_bwd(d["q"], d["k"], d["v"], o, d["dO"], st, R=0,
+                                        mask=d["mask"], v_dust=d["v_dust"], d_dust_score=dsc, **kw)
+    torch.cuda.synchronize()
+    _, rst = oracle.forward(x["q"], x["k"], x["v"], T=N - 1, R=1, mask=x["mask"],
+                            v_dust=x["v_dust"], **kw)
+    _, dcol, _ = oracle.plan(x["q"], x["k"], rst, 1, 1, R=1, mask=x["mask"], **kw)
+    dO = x["dO"].double().numpy()
+    vd = x["v_dust"].double().numpy()
+    r_dvd = np.einsum("bhl,bhld->hd", dcol, dO)
+    r_dsc = float(np.einsum("bhl,bhld,hd->", dcol, dO, vd))
+    assert parity.rel_l2(dvd.double().cpu().numpy(), r_dvd) <= 1e-4
+    assert abs(float(dsc[0]) - r_dsc) <= 1e-4 * max(abs(r_dsc), 1e-3)
+
+
 def test_full_backpropagation_matches_oracle():
     # T = 0, R = N = 12: 24 modifier terms, three blocks of the dS sweep
     L, W, eps, N = 260, 30, 0.7, 12
