@@ -24,7 +24,7 @@ SA_F32, SA_BF16 = 0, 1
 SA_BWD_ONE_REFERENCE, SA_BWD_DIRECT = 0, 1
 _STATUS = {0: "SA_OK", -1: "SA_ERR_INVALID_ARG", -2: "SA_ERR_UNSUPPORTED",
            -3: "SA_ERR_WORKSPACE", -4: "SA_ERR_CUDA", -5: "SA_ERR_NONFINITE",
-           -6: "SA_ERR_TIMEOUT"}
+           -6: "SA_ERR_TIMEOUT", -7: "SA_ERR_EXCHANGE"}
 SCHEDULES = {"one_reference": SA_BWD_ONE_REFERENCE, "direct": SA_BWD_DIRECT}
 
 
@@ -46,6 +46,15 @@ class sa_params(ctypes.Structure):
 
 
 KERNEL_KINDS = {1: "lse_sweep", 2: "pv", 3: "wsum", 4: "ds", 5: "aux", 6: "fused_sweep"}
+
+# int exchange(float* vec, long long row_stride, int rows, void* user, void* stream)
+EXCHANGE_FN = ctypes.CFUNCTYPE(ctypes.c_int, ctypes.c_void_p, ctypes.c_longlong, ctypes.c_int,
+                               ctypes.c_void_p, ctypes.c_void_p)
+
+
+class sa_shard(ctypes.Structure):
+    _fields_ = [("halo_lo", ctypes.c_int), ("halo_hi", ctypes.c_int),
+                ("exchange", EXCHANGE_FN), ("user", ctypes.c_void_p)]
 
 
 class LaunchTrace:
@@ -103,11 +112,16 @@ def _L():
     lib.sinkhorn_attn_poll.argtypes = [vp, vp]
     lib.sinkhorn_attn_debug_timeout.argtypes = [vp, ctypes.c_longlong, vp]
     lib.sinkhorn_attn_sq_dist.argtypes = [vp, vp, ctypes.c_longlong, ctypes.c_int, vp, vp]
+    SP = ctypes.POINTER(sa_shard)
+    lib.sinkhorn_attn_fwd_sharded.argtypes = [P, SP, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.sinkhorn_attn_bwd_sharded.argtypes = [P, SP, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp,
+                                              sz, vp]
     lib.sinkhorn_attn_strerror.argtypes = [ctypes.c_int]
     lib.sinkhorn_attn_strerror.restype = ctypes.c_char_p
     for f in ("sinkhorn_attn_state_size", "sinkhorn_attn_workspace_size", "sinkhorn_attn_fwd",
               "sinkhorn_attn_bwd", "sinkhorn_attn_debug_plan", "sinkhorn_attn_poll",
-              "sinkhorn_attn_debug_timeout", "sinkhorn_attn_sq_dist"):
+              "sinkhorn_attn_debug_timeout", "sinkhorn_attn_sq_dist", "sinkhorn_attn_fwd_sharded",
+              "sinkhorn_attn_bwd_sharded"):
         getattr(lib, f).restype = ctypes.c_int
     _lib = lib
     return lib
@@ -121,7 +135,7 @@ def load():
 EXPORTS = ("sinkhorn_attn_state_size", "sinkhorn_attn_workspace_size", "sinkhorn_attn_fwd",
            "sinkhorn_attn_bwd", "sinkhorn_attn_bwd_static_ws", "sinkhorn_attn_debug_plan",
            "sinkhorn_attn_poll", "sinkhorn_attn_strerror", "sinkhorn_attn_debug_timeout",
-           "sinkhorn_attn_sq_dist")
+           "sinkhorn_attn_sq_dist", "sinkhorn_attn_fwd_sharded", "sinkhorn_attn_bwd_sharded")
 
 
 def strerror(status: int) -> str:
@@ -258,6 +272,159 @@ def sinkhorn_attn_bwd_static_ws(q, k, v, o, dO, state, *, W, eps, R=2, mask=None
                                           _ptr(d_dust_score if dustbin else None), _stream(dev))
     _check(rc, "sinkhorn_attn_bwd_static_ws")
     return dq, dk, dv, (dv_dust if dustbin else None)
+
+
+# ---------------------------------------------------------------------------
+# sequence sharding (see sa_shard in the C header)
+# ---------------------------------------------------------------------------
+
+
+class _DeviceRows:
+    """``rows`` float32 rows of ``L`` entries, ``row_stride`` elements apart,
+    at a raw device address, for ``torch.as_tensor``."""
+
+    def __init__(self, ptr, rows, L, row_stride):
+        self.__cuda_array_interface__ = {
+            "shape": (rows, L), "typestr": "<f4", "data": (int(ptr), False),
+            "strides": (int(row_stride) * 4, 4), "version": 3}
+
+
+def _shard_for(halo_lo, halo_hi, exchange, L, device):
+    """The sa_shard of a sharded call: ``exchange(view)`` gets the vector as a
+    ``[rows, L]`` float32 tensor view.  Returns (shard, errors, keep-alive)."""
+    errors = []
+
+    def cb(ptr, row_stride, rows, user, stream):
+        try:
+            view = torch.as_tensor(_DeviceRows(ptr, rows, L, row_stride), device=device)
+            exchange(view)
+            return 0
+        except BaseException as e:  # reported by the caller after the C call returns
+            errors.append(e)
+            return 1
+
+    fn = EXCHANGE_FN(cb)
+    return sa_shard(int(halo_lo), int(halo_hi), fn, None), errors, fn
+
+
+def _check_sharded(rc, what, errors):
+    if rc != SA_OK:
+        err = SinkhornAttnError(rc, what)
+        if errors:
+            raise err from errors[0]
+        raise err
+
+
+def sinkhorn_attn_fwd_sharded(q, k, v, *, W, eps, T, R=2, mask=None, halo_lo, halo_hi, exchange,
+                              o=None, state=None, ws=None, trace=None):
+    """Forward on one shard of a sequence-sharded problem.  ``q, k, v``:
+    ``[B,H,L,64]`` for the local sequence (halo tokens included); ``mask``:
+    ``[B,L]``; ``exchange(view)`` fills the halo entries of the ``[B*H, L]``
+    float32 view from the neighbours (:class:`HaloExchange` over
+    torch.distributed).  Returns ``(o, state)`` like :func:`sinkhorn_attn_fwd`;
+    only the own tokens' entries are final."""
+    _contig(q, k, v, mask, o, state, ws)
+    p = _params_for(q, W, eps, T, R, False, -2.0, "one_reference", False)
+    if trace is not None:
+        trace.attach(p)
+    dev = q.device
+    B, H, L, _ = q.shape
+    o = torch.empty_like(q) if o is None else o
+    if state is None:
+        state = torch.empty(sinkhorn_attn_state_size(p), dtype=torch.float32, device=dev)
+    if ws is None:
+        ws = torch.zeros(sinkhorn_attn_workspace_size(p)[0], dtype=torch.uint8, device=dev)
+    sh, errors, _keep = _shard_for(halo_lo, halo_hi, exchange, L, dev)
+    rc = _L().sinkhorn_attn_fwd_sharded(ctypes.byref(p), ctypes.byref(sh), _ptr(q), _ptr(k),
+                                        _ptr(v), _ptr(mask), _ptr(o), _ptr(state), _ptr(ws),
+                                        ws.numel(), _stream(dev))
+    _check_sharded(rc, "sinkhorn_attn_fwd_sharded", errors)
+    return o, state.view(B, H, 2 * R + 2, L)
+
+
+def sinkhorn_attn_bwd_sharded(q, k, v, o, dO, state, *, W, eps, R=2, mask=None, halo_lo,
+                              halo_hi, exchange, schedule="one_reference", dq=None, dk=None,
+                              dv=None, ws=None, trace=None):
+    """Backward on one shard of a sequence-sharded problem (arguments as in
+    :func:`sinkhorn_attn_fwd_sharded` and :func:`sinkhorn_attn_bwd`).  Returns
+    ``(dq, dk, dv)``; only the own tokens' rows are final."""
+    _contig(q, k, v, o, dO, state, mask, dq, dk, dv, ws)
+    p = _params_for(q, W, eps, 0, R, False, -2.0, schedule, False)
+    if trace is not None:
+        trace.attach(p)
+    dev = q.device
+    L = q.shape[2]
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(q) if dk is None else dk
+    dv = torch.empty_like(q) if dv is None else dv
+    if ws is None:
+        ws = torch.zeros(sinkhorn_attn_workspace_size(p)[1], dtype=torch.uint8, device=dev)
+    sh, errors, _keep = _shard_for(halo_lo, halo_hi, exchange, L, dev)
+    rc = _L().sinkhorn_attn_bwd_sharded(ctypes.byref(p), ctypes.byref(sh), _ptr(q), _ptr(k),
+                                        _ptr(v), _ptr(mask), _ptr(o), _ptr(dO), _ptr(state),
+                                        _ptr(dq), _ptr(dk), _ptr(dv), _ptr(ws), ws.numel(),
+                                        _stream(dev))
+    _check_sharded(rc, "sinkhorn_attn_bwd_sharded", errors)
+    return dq, dk, dv
+
+
+def shard_bounds(L_total, W, rank, world):
+    """Contiguous shards of a sequence of ``L_total`` tokens over ``world``
+    ranks: ``(own_lo, own_hi, lo, hi)`` with own tokens [own_lo, own_hi) and the
+    local sequence [lo, hi) = own tokens plus up to W halo tokens each side.
+    Every shard must own at least W tokens."""
+    base, extra = divmod(L_total, world)
+    own_lo = rank * base + min(rank, extra)
+    own_hi = own_lo + base + (1 if rank < extra else 0)
+    if world > 1 and base < max(W, 1):
+        raise ValueError(f"{L_total} tokens over {world} ranks leave fewer than W = {W} per rank")
+    return own_lo, own_hi, max(0, own_lo - W), min(L_total, own_hi + W)
+
+
+class HaloExchange:
+    """The exchange of a sequence-sharded call over torch.distributed (NCCL on
+    GPUs, gloo on CPUs): rank r's local vector is [left halo | own | right
+    halo]; it sends its first and last own entries (as many as the
+    neighbour's halo holds: the halos on the two sides of a boundary are equal,
+    W tokens, as ``shard_bounds`` makes them) and receives its halos.  Ranks are
+    in sequence order within ``group``."""
+
+    def __init__(self, halo_lo, halo_hi, group=None):
+        import torch.distributed as dist
+
+        self.dist = dist
+        self.group = group
+        self.rank = dist.get_rank(group)
+        self.world = dist.get_world_size(group)
+        self.halo_lo, self.halo_hi = int(halo_lo), int(halo_hi)
+        if (self.halo_lo > 0 and self.rank == 0) or (self.halo_hi > 0 and self.rank == self.world - 1):
+            raise ValueError("a halo on a side without a neighbour")
+
+    def _peer(self, r):
+        return r if self.group is None else self.dist.get_global_rank(self.group, r)
+
+    def __call__(self, view):
+        dist, L = self.dist, view.shape[1]
+        hl, hh = self.halo_lo, self.halo_hi
+        ops, recvs = [], []
+        if hl > 0:
+            left = self._peer(self.rank - 1)
+            ops.append(dist.P2POp(dist.isend, view[:, hl:2 * hl].contiguous(), left, self.group))
+            buf = torch.empty(view.shape[0], hl, dtype=view.dtype, device=view.device)
+            ops.append(dist.P2POp(dist.irecv, buf, left, self.group))
+            recvs.append((slice(0, hl), buf))
+        if hh > 0:
+            right = self._peer(self.rank + 1)
+            ops.append(dist.P2POp(dist.isend, view[:, L - 2 * hh:L - hh].contiguous(), right,
+                                  self.group))
+            buf = torch.empty(view.shape[0], hh, dtype=view.dtype, device=view.device)
+            ops.append(dist.P2POp(dist.irecv, buf, right, self.group))
+            recvs.append((slice(L - hh, L), buf))
+        if ops:
+            for w in dist.batch_isend_irecv(ops):
+                w.wait()
+        for sl, buf in recvs:
+            view[:, sl].copy_(buf)
 
 
 def sinkhorn_attn_debug_plan(q, k, state, a, b, *, W, eps, R=2, mask=None, dustbin=False,

@@ -524,9 +524,24 @@ struct Ctx {
     const float* state;
     int* status;   // device status word (workspace header)
     mutable Tracer tr;
+    const sa_shard* shard = nullptr;  // sequence-sharded call, else null
     // state row r (0..2R+1) as a Vec
     Vec srow(int r) const { return vec(state + (size_t)r * d.ld, sst); }
+    // sharded calls: the neighbours' values into the halo entries of a vector
+    // just produced (rows of d.L entries, row_stride apart)
+    sa_status halo(const float* v, long long row_stride) const {
+        if (!shard) return SA_OK;
+        return shard->exchange(const_cast<float*>(v), row_stride, d.BH, shard->user, st) == 0
+                   ? SA_OK
+                   : SA_ERR_EXCHANGE;
+    }
 };
+
+#define SA_HALO(x, v, stride)                      \
+    do {                                           \
+        sa_status h_ = (x).halo((v), (stride));    \
+        if (h_ != SA_OK) return h_;                \
+    } while (0)
 
 simt::SweepArgs base_args(const Ctx& x) {
     simt::SweepArgs a;
@@ -570,6 +585,7 @@ sa_status fwd_impl(const Ctx& x, const T* q, const T* k, const T* v, const uint8
         a.online = (it == 0);
         a.out_vec = mvec(state + (size_t)(2 * rout) * d.ld, x.sst);
         SA_CUDA((launch_sweep<T, simt::LSE>(a, d.BH, x.st, x.tr, x.status)));
+        SA_HALO(x, a.out_vec.p, x.sst);
         // columns: v^(rout) = -LSE_i(S + u^(rout)), shifted by the previous v
         a.A = k; a.Bo = q;
         a.cd = x.srow(2 * rout);
@@ -577,6 +593,7 @@ sa_status fwd_impl(const Ctx& x, const T* q, const T* k, const T* v, const uint8
         a.online = 0;
         a.out_vec = mvec(state + (size_t)(2 * rout + 1) * d.ld, x.sst);
         SA_CUDA((launch_sweep<T, simt::LSE>(a, d.BH, x.st, x.tr, x.status)));
+        SA_HALO(x, a.out_vec.p, x.sst);
     }
     // O = P^(R,R) V (+ dustbin column times v_dust)
     simt::SweepArgs b = base_args(x);
@@ -726,6 +743,7 @@ sa_status bwd_impl(const Ctx& x, const T* q, const T* k, const T* v, const uint8
         a.out_vec = mvec(vb(R), vs);
         a.dvd_part = dvd;
         SA_CUDA((launch_sweep<T, simt::PV>(a, d.BH, x.st, x.tr, x.status)));
+        if (R > 0) SA_HALO(x, vb(R), vs);
     }
     // ubar^R = a - P vbar^R  (query sweep; R = 0 has no dual cotangents)
     if (R > 0) {
@@ -738,6 +756,7 @@ sa_status bwd_impl(const Ctx& x, const T* q, const T* k, const T* v, const uint8
         a.sgn = -1.f;
         a.out_vec = mvec(ub(R), vs);
         SA_CUDA((launch_sweep<T, simt::WSUM>(a, d.BH, x.st, x.tr, x.status)));
+        SA_HALO(x, ub(R), vs);
     }
     for (int r = R; r >= 2; --r) {
         // vbar^(r-1) = -P^(r,r-1)^T ubar^r
@@ -756,6 +775,7 @@ sa_status bwd_impl(const Ctx& x, const T* q, const T* k, const T* v, const uint8
             a.mult = vec(ev(r - 1), vs);
         }
         SA_CUDA((launch_sweep<T, simt::WSUM>(a, d.BH, x.st, x.tr, x.status)));
+        SA_HALO(x, vb(r - 1), vs);
         // ubar^(r-1) = -P^(r-1,r-1) vbar^(r-1)
         simt::SweepArgs b = base_args(x);
         b.mask = mask;
@@ -772,6 +792,7 @@ sa_status bwd_impl(const Ctx& x, const T* q, const T* k, const T* v, const uint8
             b.mult = vec(eu(r - 1), vs);
         }
         SA_CUDA((launch_sweep<T, simt::WSUM>(b, d.BH, x.st, x.tr, x.status)));
+        SA_HALO(x, ub(r - 1), vs);
     }
 
     // modifier / staircase terms, query side (rq) and key side (rk)
@@ -903,9 +924,21 @@ sa_status sinkhorn_attn_workspace_size(const sa_params* p, size_t* fwd_bytes, si
     return SA_OK;
 }
 
-sa_status sinkhorn_attn_fwd(const sa_params* p, const void* q, const void* k, const void* v,
-                            const uint8_t* mask, const float* v_dust, void* o, float* state,
-                            void* ws, size_t ws_bytes, void* stream) {
+}  // extern "C"
+
+namespace {
+// A shard description a sharded call can use (see sa_shard).
+sa_status check_shard(const sa_params* p, const sa_shard* sh) {
+    if (!sh || !sh->exchange) return SA_ERR_INVALID_ARG;
+    if (sh->halo_lo < 0 || sh->halo_hi < 0 || (long long)sh->halo_lo + sh->halo_hi > p->L)
+        return SA_ERR_INVALID_ARG;
+    if (p->dustbin) return SA_ERR_UNSUPPORTED;
+    return SA_OK;
+}
+
+sa_status fwd_call(const sa_params* p, const sa_shard* shard, const void* q, const void* k,
+                   const void* v, const uint8_t* mask, const float* v_dust, void* o, float* state,
+                   void* ws, size_t ws_bytes, void* stream) {
     Dims d;
     sa_status s = check_params(p, &d);
     if (s != SA_OK) return s;
@@ -926,11 +959,12 @@ sa_status sinkhorn_attn_fwd(const sa_params* p, const void* q, const void* k, co
     x.status = (int*)ws;
     x.tr.p = p;
     x.tr.st = x.st;
+    x.shard = shard;
     const float* vd = p->dustbin ? v_dust : nullptr;
     if (p->dtype == SA_F32)
         s = fwd_impl<float>(x, (const float*)q, (const float*)k, (const float*)v, mask, vd,
                             (float*)o, state);
-    else if (fused_fwd(p))
+    else if (fused_fwd(p) && !shard)
         s = fwd_fused(x, (const __nv_bfloat16*)q, (const __nv_bfloat16*)k,
                       (const __nv_bfloat16*)v, mask, (__nv_bfloat16*)o, state, (char*)ws);
     else
@@ -951,11 +985,10 @@ sa_status sinkhorn_attn_fwd(const sa_params* p, const void* q, const void* k, co
     return SA_OK;
 }
 
-sa_status sinkhorn_attn_bwd(const sa_params* p, const void* q, const void* k, const void* v,
-                            const uint8_t* mask, const float* v_dust, const void* o,
-                            const void* dO, const float* state, void* dq, void* dk, void* dv,
-                            float* dv_dust, float* d_dust_score, void* ws, size_t ws_bytes,
-                            void* stream) {
+sa_status bwd_call(const sa_params* p, const sa_shard* shard, const void* q, const void* k,
+                   const void* v, const uint8_t* mask, const float* v_dust, const void* o,
+                   const void* dO, const float* state, void* dq, void* dk, void* dv,
+                   float* dv_dust, float* d_dust_score, void* ws, size_t ws_bytes, void* stream) {
     Dims d;
     sa_status s = check_params(p, &d);
     if (s != SA_OK) return s;
@@ -978,6 +1011,7 @@ sa_status sinkhorn_attn_bwd(const sa_params* p, const void* q, const void* k, co
     x.status = (int*)ws;
     x.tr.p = p;
     x.tr.st = x.st;
+    x.shard = shard;
     const float* vd = p->dustbin ? v_dust : nullptr;
     float* dvd = p->dustbin ? dv_dust : nullptr;
     float* dsc = p->dustbin ? d_dust_score : nullptr;
@@ -1003,6 +1037,44 @@ sa_status sinkhorn_attn_bwd(const sa_params* p, const void* q, const void* k, co
         }
     }
     return SA_OK;
+}
+}  // namespace
+
+extern "C" {
+
+sa_status sinkhorn_attn_fwd(const sa_params* p, const void* q, const void* k, const void* v,
+                            const uint8_t* mask, const float* v_dust, void* o, float* state,
+                            void* ws, size_t ws_bytes, void* stream) {
+    return fwd_call(p, nullptr, q, k, v, mask, v_dust, o, state, ws, ws_bytes, stream);
+}
+
+sa_status sinkhorn_attn_bwd(const sa_params* p, const void* q, const void* k, const void* v,
+                            const uint8_t* mask, const float* v_dust, const void* o,
+                            const void* dO, const float* state, void* dq, void* dk, void* dv,
+                            float* dv_dust, float* d_dust_score, void* ws, size_t ws_bytes,
+                            void* stream) {
+    return bwd_call(p, nullptr, q, k, v, mask, v_dust, o, dO, state, dq, dk, dv, dv_dust,
+                    d_dust_score, ws, ws_bytes, stream);
+}
+
+sa_status sinkhorn_attn_fwd_sharded(const sa_params* p, const sa_shard* shard, const void* q,
+                                    const void* k, const void* v, const uint8_t* mask, void* o,
+                                    float* state, void* ws, size_t ws_bytes, void* stream) {
+    if (!p) return SA_ERR_INVALID_ARG;
+    const sa_status s = check_shard(p, shard);
+    if (s != SA_OK) return s;
+    return fwd_call(p, shard, q, k, v, mask, nullptr, o, state, ws, ws_bytes, stream);
+}
+
+sa_status sinkhorn_attn_bwd_sharded(const sa_params* p, const sa_shard* shard, const void* q,
+                                    const void* k, const void* v, const uint8_t* mask,
+                                    const void* o, const void* dO, const float* state, void* dq,
+                                    void* dk, void* dv, void* ws, size_t ws_bytes, void* stream) {
+    if (!p) return SA_ERR_INVALID_ARG;
+    const sa_status s = check_shard(p, shard);
+    if (s != SA_OK) return s;
+    return bwd_call(p, shard, q, k, v, mask, nullptr, o, dO, state, dq, dk, dv, nullptr, nullptr,
+                    ws, ws_bytes, stream);
 }
 
 }  // extern "C"
@@ -1159,6 +1231,7 @@ const char* sinkhorn_attn_strerror(sa_status s) {
         case SA_ERR_CUDA: return "CUDA runtime or launch error";
         case SA_ERR_NONFINITE: return "non-finite value in duals or outputs";
         case SA_ERR_TIMEOUT: return "bounded device wait gave up";
+        case SA_ERR_EXCHANGE: return "halo exchange callback failed (sequence-sharded call)";
     }
     return "unknown status";
 }

@@ -55,7 +55,8 @@ typedef enum {
     SA_ERR_WORKSPACE = -3,    /* workspace smaller than sinkhorn_attn_workspace_size() */
     SA_ERR_CUDA = -4,         /* a CUDA runtime call or kernel launch failed */
     SA_ERR_NONFINITE = -5,    /* device found a NaN/Inf (only with check_finite) */
-    SA_ERR_TIMEOUT = -6       /* a bounded device-side wait gave up */
+    SA_ERR_TIMEOUT = -6,      /* a bounded device-side wait gave up */
+    SA_ERR_EXCHANGE = -7      /* a sharded call's halo exchange callback failed */
 } sa_status;
 
 typedef enum { SA_F32 = 0, SA_BF16 = 1 } sa_dtype;
@@ -157,6 +158,53 @@ sa_status sinkhorn_attn_bwd(const sa_params* p, const void* q, const void* k, co
                             const void* dO, const float* state, void* dq, void* dk, void* dv,
                             float* dv_dust, float* d_dust_score, void* ws, size_t ws_bytes,
                             void* stream);
+
+/*
+ * Sequence sharding (no counterpart in the pages, which shard by batch): one
+ * problem's tokens split into contiguous shards, one per rank, each rank
+ * holding its own tokens plus halos of its neighbours' tokens.  The local
+ * sequence of p->L tokens is
+ *     [0, halo_lo)                 the left neighbour's last halo_lo tokens,
+ *     [halo_lo, L - halo_hi)       this rank's own tokens,
+ *     [L - halo_hi, L)             the right neighbour's first halo_hi tokens,
+ * with halo_lo = 0 on the shard that starts the sequence and halo_hi = 0 on
+ * the one that ends it; an interior halo must hold at least W tokens (every
+ * band neighbour of an own token is then local) and every shard at least W
+ * own tokens (a halo then comes from one neighbour).  The sharded calls run the
+ * same path with one iteration as a row sweep and a column sweep (the fused
+ * single-pass iteration needs both halves of an iteration on one device), and
+ * after every sweep that produces a dual or vector cotangent they call
+ *     exchange(vec, row_stride, rows, user, stream)
+ * on the host, in stream order (the sweep has been launched on `stream`, not
+ * necessarily finished): vec + r * row_stride (r < rows = B*H) is row r's p->L
+ * float32 entries in device memory, and the callback must, before returning
+ * or in work it enqueues on `stream`, overwrite each row's halo entries with
+ * the values its neighbours hold for those tokens (and hand them this rank's
+ * edge values).  Every rank makes the same sequence of calls.  A non-zero
+ * return ends the call with SA_ERR_EXCHANGE.  Results are exact for own
+ * tokens; halo rows of o, dq, dk, dv hold partial values to be discarded.
+ * The dustbin couples every token and is not supported (SA_ERR_UNSUPPORTED).
+ */
+typedef int (*sa_exchange_fn)(float* vec, long long row_stride, int rows, void* user,
+                              void* stream);
+typedef struct {
+    int halo_lo, halo_hi;      /* halo tokens at the start and end of the local sequence */
+    sa_exchange_fn exchange;   /* not NULL */
+    void* user;                /* passed through to exchange */
+} sa_shard;
+
+/* sinkhorn_attn_fwd / sinkhorn_attn_bwd on one shard of a sequence-sharded
+ * problem (see sa_shard); the other arguments, sizes and the workspace are
+ * those of the unsharded calls for the local sequence length p->L.
+ * SA_ERR_INVALID_ARG for a NULL shard or exchange, or halos outside [0, L]
+ * that overlap; SA_ERR_UNSUPPORTED with a dustbin. */
+sa_status sinkhorn_attn_fwd_sharded(const sa_params* p, const sa_shard* shard, const void* q,
+                                    const void* k, const void* v, const uint8_t* mask, void* o,
+                                    float* state, void* ws, size_t ws_bytes, void* stream);
+sa_status sinkhorn_attn_bwd_sharded(const sa_params* p, const sa_shard* shard, const void* q,
+                                    const void* k, const void* v, const uint8_t* mask,
+                                    const void* o, const void* dO, const float* state, void* dq,
+                                    void* dk, void* dv, void* ws, size_t ws_bytes, void* stream);
 
 /*
  * Test hook: the plan P^(a,b) (0 <= a, b <= R) from a finished forward state.

@@ -146,3 +146,20 @@ def test_strerror_covers_every_status():
     for s in range(0, -7, -1):
         assert sa.strerror(s) and "unknown" not in sa.strerror(s)
     assert "unknown" in sa.strerror(42)
+
+
+def test_sharded_calls_validate_the_shard_on_the_host():
+    lib = sa._L()
+    p = P(B=1, H=1, L=50, W=4, dtype=torch.bfloat16)
+    noop = sa.EXCHANGE_FN(lambda *a: 0)
+    fwd = lambda sh: lib.sinkhorn_attn_fwd_sharded(ctypes.byref(p), sh, *([None] * 7), 1 << 30, None)
+    bwd = lambda sh: lib.sinkhorn_attn_bwd_sharded(ctypes.byref(p), sh, *([None] * 11), 1 << 30,
+                                                   None)
+    for call in (fwd, bwd):
+        assert call(None) == -1                                                  # no shard
+        assert call(ctypes.byref(sa.sa_shard(4, 4, sa.EXCHANGE_FN(), None))) == -1  # no callback
+        assert call(ctypes.byref(sa.sa_shard(30, 30, noop, None))) == -1          # halos overlap
+        assert call(ctypes.byref(sa.sa_shard(-1, 0, noop, None))) == -1
+    pd = P(B=1, H=1, L=50, W=4, dustbin=True)
+    assert lib.sinkhorn_attn_fwd_sharded(ctypes.byref(pd), ctypes.byref(sa.sa_shard(4, 4, noop, None)),
+                                         *([None] * 7), 1 << 30, None) == -2      # dustbin

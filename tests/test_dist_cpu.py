@@ -110,3 +110,58 @@ def test_reference_arm_prints_on_rank_zero_only(capsys, monkeypatch):
 
     bench.run_reference(A(), bench.workloads.WORKLOADS["small512"])
     assert capsys.readouterr().out == ""
+
+
+def _worker_halo(rank, ws, port, q):
+    """One rank of a sequence-sharded vector: own entries filled with their
+    global values, halos empty; after the exchange the local vector must equal
+    the global one over [lo, hi), and the row padding must be untouched."""
+    _env(rank, ws, port)
+    from datetime import timedelta
+
+    import torch
+    import torch.distributed as dist
+
+    import banded_log_domain_b200 as sa
+
+    try:
+        dist.init_process_group("gloo", rank=rank, world_size=ws, timeout=timedelta(seconds=30))
+        Lt, W, rows = 23, 3, 4
+        own_lo, own_hi, lo, hi = sa.shard_bounds(Lt, W, rank, ws)
+        glob = torch.arange(Lt, dtype=torch.float32)[None, :] * 10 + torch.arange(rows)[:, None]
+        buf = torch.full((rows, hi - lo + 5), -1.0)  # rows wider than L, like the state's
+        view = buf[:, :hi - lo]
+        view[:, own_lo - lo:own_hi - lo] = glob[:, own_lo:own_hi]
+        ex = sa.HaloExchange(own_lo - lo, hi - own_hi)
+        ex(view)
+        ok = torch.equal(view, glob[:, lo:hi]) and bool((buf[:, hi - lo:] == -1).all())
+        # a second exchange (the next sweep) with new values
+        view[:, own_lo - lo:own_hi - lo] += 1000.0
+        ex(view)
+        ok = ok and torch.equal(view, glob[:, lo:hi] + 1000.0)
+        q.put((rank, ok, (own_lo, own_hi, lo, hi)))
+    finally:
+        if dist.is_initialized():
+            dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("ws", [2, 3])
+def test_halo_exchange_fills_every_halo(ws):
+    ps, out = _run(_worker_halo, ws=ws)
+    assert all(p.exitcode == 0 for p in ps)
+    assert sorted(o[0] for o in out) == list(range(ws))
+    assert all(o[1] for o in out), out
+    bounds = sorted(o[2] for o in out)
+    assert bounds[0][0] == 0 and bounds[-1][1] == 23           # shards cover the sequence
+    assert all(a[1] == b[0] for a, b in zip(bounds, bounds[1:]))  # contiguously
+
+
+def test_shard_bounds():
+    import banded_log_domain_b200 as sa
+
+    assert sa.shard_bounds(10, 2, 0, 1) == (0, 10, 0, 10)
+    assert sa.shard_bounds(10, 2, 0, 3) == (0, 4, 0, 6)
+    assert sa.shard_bounds(10, 2, 1, 3) == (4, 7, 2, 9)
+    assert sa.shard_bounds(10, 2, 2, 3) == (7, 10, 5, 10)
+    with pytest.raises(ValueError):
+        sa.shard_bounds(10, 4, 0, 3)  # 3 own tokens < W
