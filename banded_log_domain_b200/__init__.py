@@ -47,6 +47,14 @@ class sa_params(ctypes.Structure):
 
 KERNEL_KINDS = {1: "lse_sweep", 2: "pv", 3: "wsum", 4: "ds", 5: "aux", 6: "fused_sweep"}
 
+class sa_host_step(ctypes.Structure):
+    _fields_ = [("q", ctypes.c_void_p), ("k", ctypes.c_void_p), ("v", ctypes.c_void_p),
+                ("dO", ctypes.c_void_p), ("mask", ctypes.c_void_p), ("v_dust", ctypes.c_void_p),
+                ("o", ctypes.c_void_p), ("dq", ctypes.c_void_p), ("dk", ctypes.c_void_p),
+                ("dv", ctypes.c_void_p), ("state", ctypes.c_void_p), ("dv_dust", ctypes.c_void_p),
+                ("d_dust_score", ctypes.c_void_p), ("groups", ctypes.c_int)]
+
+
 # int exchange(float* vec, long long row_stride, int rows, void* user, void* stream)
 EXCHANGE_FN = ctypes.CFUNCTYPE(ctypes.c_int, ctypes.c_void_p, ctypes.c_longlong, ctypes.c_int,
                                ctypes.c_void_p, ctypes.c_void_p)
@@ -112,6 +120,8 @@ def _L():
     lib.sinkhorn_attn_poll.argtypes = [vp, vp]
     lib.sinkhorn_attn_debug_timeout.argtypes = [vp, ctypes.c_longlong, vp]
     lib.sinkhorn_attn_sq_dist.argtypes = [vp, vp, ctypes.c_longlong, ctypes.c_int, vp, vp]
+    lib.sinkhorn_attn_step_host_workspace_size.argtypes = [P, ctypes.c_int, ctypes.POINTER(sz)]
+    lib.sinkhorn_attn_step_host.argtypes = [P, ctypes.POINTER(sa_host_step), vp, sz, vp]
     SP = ctypes.POINTER(sa_shard)
     lib.sinkhorn_attn_fwd_sharded.argtypes = [P, SP, vp, vp, vp, vp, vp, vp, vp, sz, vp]
     lib.sinkhorn_attn_bwd_sharded.argtypes = [P, SP, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp,
@@ -121,7 +131,8 @@ def _L():
     for f in ("sinkhorn_attn_state_size", "sinkhorn_attn_workspace_size", "sinkhorn_attn_fwd",
               "sinkhorn_attn_bwd", "sinkhorn_attn_debug_plan", "sinkhorn_attn_poll",
               "sinkhorn_attn_debug_timeout", "sinkhorn_attn_sq_dist", "sinkhorn_attn_fwd_sharded",
-              "sinkhorn_attn_bwd_sharded"):
+              "sinkhorn_attn_bwd_sharded", "sinkhorn_attn_step_host_workspace_size",
+              "sinkhorn_attn_step_host"):
         getattr(lib, f).restype = ctypes.c_int
     _lib = lib
     return lib
@@ -135,7 +146,8 @@ def load():
 EXPORTS = ("sinkhorn_attn_state_size", "sinkhorn_attn_workspace_size", "sinkhorn_attn_fwd",
            "sinkhorn_attn_bwd", "sinkhorn_attn_bwd_static_ws", "sinkhorn_attn_debug_plan",
            "sinkhorn_attn_poll", "sinkhorn_attn_strerror", "sinkhorn_attn_debug_timeout",
-           "sinkhorn_attn_sq_dist", "sinkhorn_attn_fwd_sharded", "sinkhorn_attn_bwd_sharded")
+           "sinkhorn_attn_sq_dist", "sinkhorn_attn_fwd_sharded", "sinkhorn_attn_bwd_sharded",
+           "sinkhorn_attn_step_host_workspace_size", "sinkhorn_attn_step_host")
 
 
 def strerror(status: int) -> str:
@@ -272,6 +284,52 @@ def sinkhorn_attn_bwd_static_ws(q, k, v, o, dO, state, *, W, eps, R=2, mask=None
                                           _ptr(d_dust_score if dustbin else None), _stream(dev))
     _check(rc, "sinkhorn_attn_bwd_static_ws")
     return dq, dk, dv, (dv_dust if dustbin else None)
+
+
+def sinkhorn_attn_step_host_workspace_size(p: sa_params, groups: int) -> int:
+    n = ctypes.c_size_t()
+    _check(_L().sinkhorn_attn_step_host_workspace_size(ctypes.byref(p), int(groups),
+                                                       ctypes.byref(n)),
+           "sinkhorn_attn_step_host_workspace_size")
+    return n.value
+
+
+def sinkhorn_attn_step_host(q, k, v, dO, *, W, eps, T, R=2, mask=None, dustbin=False,
+                            dustbin_score=-2.0, v_dust=None, schedule="one_reference", groups=4,
+                            o=None, dq=None, dk=None, dv=None, state=None, dv_dust=None,
+                            d_dust_score=None, ws=None, device=None):
+    """Forward + backward with inputs and results in host memory: ``q, k, v,
+    dO`` are CPU tensors ``[B,H,L,64]`` (page-locked for the copies to overlap
+    the compute), ``mask`` ``[B,L]`` uint8 and ``v_dust`` ``[H,64]`` CPU tensors or
+    None.  The library copies ``groups`` groups of problems in and results out
+    while other groups compute.  Returns CPU tensors ``(o, dq, dk, dv)`` (and
+    fills ``state``, ``dv_dust``, ``d_dust_score`` when given); they are final once
+    the device's current stream has been synchronised (this function does not
+    synchronise).  ``ws``: optional device workspace of
+    :func:`sinkhorn_attn_step_host_workspace_size` bytes."""
+    for t in (q, k, v, dO, mask, v_dust, o, dq, dk, dv, state, dv_dust, d_dust_score):
+        if t is not None and t.is_cuda:
+            raise ValueError("sinkhorn_attn_step_host takes host (CPU) tensors")
+    _contig(q, k, v, dO, mask, v_dust, o, dq, dk, dv, state, dv_dust, d_dust_score)
+    p = _params_for(q, W, eps, T, R, dustbin, dustbin_score, schedule, False)
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    pin = q.is_pinned()
+    mk = lambda: torch.empty(q.shape, dtype=q.dtype, pin_memory=pin)
+    o = mk() if o is None else o
+    dq = mk() if dq is None else dq
+    dk = mk() if dk is None else dk
+    dv = mk() if dv is None else dv
+    if ws is None:
+        ws = torch.empty(sinkhorn_attn_step_host_workspace_size(p, groups), dtype=torch.uint8,
+                         device=dev)
+    io = sa_host_step(_ptr(q), _ptr(k), _ptr(v), _ptr(dO), _ptr(mask),
+                      _ptr(v_dust if dustbin else None), _ptr(o), _ptr(dq), _ptr(dk), _ptr(dv),
+                      _ptr(state), _ptr(dv_dust if dustbin else None),
+                      _ptr(d_dust_score if dustbin else None), int(groups))
+    rc = _L().sinkhorn_attn_step_host(ctypes.byref(p), ctypes.byref(io), _ptr(ws), ws.numel(),
+                                      _stream(dev))
+    _check(rc, "sinkhorn_attn_step_host")
+    return o, dq, dk, dv
 
 
 # ---------------------------------------------------------------------------

@@ -40,6 +40,7 @@ namespace {
 constexpr size_t kHeader = 256;   // status word + padding at the start of every workspace
 constexpr int kD = simt::D;
 constexpr int kMaxR = 256;  // tail length limit (host term lists, workspace)
+constexpr int kMaxDevicesHS = 64;  // devices with copy streams for the host-buffer step
 
 size_t align_up(size_t x) { return (x + 255) & ~size_t(255); }
 
@@ -280,6 +281,12 @@ __global__ void k_dscore(const T* dO, const float* v_dust, const uint8_t* mask,
         for (int w = 0; w < (int)(blockDim.x >> 5); ++w) sum += red[w];
         part[bh] = sum;
     }
+}
+
+// out[i] += in[i], i < n.
+__global__ void k_add(float* out, const float* in, int n) {
+    const int i = blockIdx.x * blockDim.x + threadIdx.x;
+    if (i < n) out[i] += in[i];
 }
 
 // out[0] = sum of part[0..n) in a fixed order (one block of 256 threads).
@@ -1075,6 +1082,271 @@ sa_status sinkhorn_attn_bwd_sharded(const sa_params* p, const sa_shard* shard, c
     if (s != SA_OK) return s;
     return bwd_call(p, shard, q, k, v, mask, nullptr, o, dO, state, dq, dk, dv, nullptr, nullptr,
                     ws, ws_bytes, stream);
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// One step with host-memory inputs and results, pipelined over problem groups
+// ---------------------------------------------------------------------------
+namespace {
+
+struct Group {
+    int b0, nb, h0, nh;  // batches [b0, b0 + nb), heads [h0, h0 + nh)
+};
+
+// Boundaries of n items in `parts` runs; with three or more runs the first and
+// last are half as large as the others (the pipeline fills with the first
+// group's copies and drains with the last one's), every run at least one item.
+std::vector<int> split_runs(int n, int parts) {
+    parts = std::max(1, std::min(parts, n));
+    std::vector<int> cut(parts + 1, 0);
+    const double total = parts >= 3 ? parts - 1.0 : parts;
+    double acc = 0.0;
+    for (int i = 0; i < parts; ++i) {
+        acc += (parts >= 3 && (i == 0 || i == parts - 1)) ? 0.5 : 1.0;
+        cut[i + 1] = (int)std::lround(acc / total * n);
+    }
+    cut[parts] = n;
+    for (int i = 1; i <= parts; ++i) cut[i] = std::max(cut[i], cut[i - 1] + 1);  // non-empty
+    for (int i = parts - 1; i >= 1; --i) cut[i] = std::min(cut[i], cut[i + 1] - 1);
+    return cut;
+}
+
+// Contiguous groups of (batch, head) problems: whole batches, or runs of heads
+// within each batch when there are fewer batches than groups (never with a
+// dustbin, whose value and score gradients sum over every head of a batch).
+std::vector<Group> plan_groups(const sa_params* p, int groups) {
+    std::vector<Group> g;
+    const int B = p->B, H = p->H;
+    if (B <= 0 || H <= 0) return g;
+    if (groups <= B || p->dustbin || H == 1) {
+        const std::vector<int> cut = split_runs(B, groups);
+        for (size_t i = 0; i + 1 < cut.size(); ++i) g.push_back({cut[i], cut[i + 1] - cut[i], 0, H});
+    } else {
+        const int per = std::min(H, (groups + B - 1) / B);
+        const std::vector<int> cut = split_runs(H, per);
+        for (int b = 0; b < B; ++b)
+            for (size_t i = 0; i + 1 < cut.size(); ++i) g.push_back({b, 1, cut[i], cut[i + 1] - cut[i]});
+    }
+    return g;
+}
+
+sa_params group_params(const sa_params* p, const Group& g) {
+    sa_params q = *p;
+    q.B = g.nb;
+    q.H = g.nh;
+    q.trace_events = nullptr;
+    q.trace_kinds = nullptr;
+    q.trace_count = nullptr;
+    q.trace_cap = 0;
+    return q;
+}
+
+// Two slots (groups in flight), each with device copies of a group's inputs,
+// results, dual state and fwd/bwd workspaces; then the whole mask, v_dust and
+// the dustbin gradient sums.
+struct HostLayout {
+    size_t mat, st, fws, bws;        // bytes of one matrix, the state, the workspaces (largest group)
+    size_t slot;                     // bytes of one slot
+    size_t mat_off[8], st_off, fws_off, bws_off, dvd_off, dsc_off;  // within a slot
+    size_t mask_off, vd_off, acc_dvd_off, acc_dsc_off, total;
+};
+
+HostLayout host_layout(const sa_params* p, const std::vector<Group>& gs) {
+    HostLayout l{};
+    int maxp = 0;
+    Group big{0, 0, 0, 0};
+    for (const Group& g : gs)
+        if (g.nb * g.nh > maxp) { maxp = g.nb * g.nh; big = g; }
+    const size_t es = p->dtype == SA_F32 ? 4 : 2;
+    const long long ld = (long long)p->L + (p->dustbin ? 1 : 0);
+    l.mat = align_up((size_t)maxp * p->L * kD * es);
+    l.st = align_up((size_t)maxp * (2 * p->R + 2) * ld * sizeof(float));
+    if (maxp > 0) {
+        const sa_params q = group_params(p, big);
+        Dims d;
+        check_params(&q, &d);
+        l.fws = align_up(fwd_layout(d, &q).total);
+        l.bws = align_up(bwd_layout(d).total);
+    }
+    size_t o = 0;
+    for (int i = 0; i < 8; ++i) { l.mat_off[i] = o; o += l.mat; }
+    l.st_off = o;  o += l.st;
+    l.fws_off = o; o += l.fws;
+    l.bws_off = o; o += l.bws;
+    l.dvd_off = o; o += align_up((size_t)p->H * kD * sizeof(float));
+    l.dsc_off = o; o += 256;
+    l.slot = o;
+    o = 2 * l.slot;
+    l.mask_off = o;    o += align_up((size_t)p->B * p->L);
+    l.vd_off = o;      o += align_up((size_t)p->H * kD * sizeof(float));
+    l.acc_dvd_off = o; o += align_up((size_t)p->H * kD * sizeof(float));
+    l.acc_dsc_off = o; o += 256;
+    l.total = o;
+    return l;
+}
+
+// Host memory, page-locked or pageable (not device memory).
+bool host_ok(const void* x) {
+    if (!x) return false;
+    cudaPointerAttributes at;
+    if (cudaPointerGetAttributes(&at, x) != cudaSuccess) {
+        cudaGetLastError();
+        return true;  // unknown to CUDA: pageable host memory
+    }
+    return at.type == cudaMemoryTypeHost || at.type == cudaMemoryTypeUnregistered;
+}
+
+// The library's two copy streams on the current device (created on first use).
+sa_status copy_streams(cudaStream_t* h2d, cudaStream_t* d2h) {
+    static cudaStream_t s_h2d[kMaxDevicesHS], s_d2h[kMaxDevicesHS];
+    static std::mutex mu;
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) return SA_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevicesHS) return SA_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!s_h2d[dev]) {
+        if (cudaStreamCreateWithFlags(&s_h2d[dev], cudaStreamNonBlocking) != cudaSuccess ||
+            cudaStreamCreateWithFlags(&s_d2h[dev], cudaStreamNonBlocking) != cudaSuccess)
+            return SA_ERR_CUDA;
+    }
+    *h2d = s_h2d[dev];
+    *d2h = s_d2h[dev];
+    return SA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+sa_status sinkhorn_attn_step_host_workspace_size(const sa_params* p, int groups, size_t* bytes) {
+    Dims d;
+    sa_status s = check_params(p, &d);
+    if (s != SA_OK) return s;
+    if (groups < 1 || !bytes) return SA_ERR_INVALID_ARG;
+    *bytes = host_layout(p, plan_groups(p, groups)).total;
+    return SA_OK;
+}
+
+sa_status sinkhorn_attn_step_host(const sa_params* p, const sa_host_step* io, void* ws,
+                                  size_t ws_bytes, void* stream) {
+    Dims d;
+    sa_status s = check_params(p, &d);
+    if (s != SA_OK) return s;
+    if (!io || io->groups < 1) return SA_ERR_INVALID_ARG;
+    if (p->check_finite) return SA_ERR_UNSUPPORTED;
+    if (p->T + p->R < 1) return SA_ERR_INVALID_ARG;
+    const std::vector<Group> gs = plan_groups(p, io->groups);
+    const HostLayout l = host_layout(p, gs);
+    if (ws_bytes < l.total) return SA_ERR_WORKSPACE;
+    if (d.BH == 0 || d.L == 0) return SA_OK;
+    for (const void* h : {io->q, io->k, io->v, io->dO, (const void*)io->o, (const void*)io->dq,
+                          (const void*)io->dk, (const void*)io->dv})
+        if (!host_ok(h)) return SA_ERR_INVALID_ARG;
+    for (const void* h : {(const void*)io->mask, (const void*)io->v_dust, (const void*)io->state,
+                          (const void*)io->dv_dust, (const void*)io->d_dust_score})
+        if (h && !host_ok(h)) return SA_ERR_INVALID_ARG;
+    if (!device_ok(ws)) return SA_ERR_INVALID_ARG;
+    cudaStream_t cs = (cudaStream_t)stream, h2d = nullptr, d2h = nullptr;
+    s = copy_streams(&h2d, &d2h);
+    if (s != SA_OK) return s;
+
+    char* w = (char*)ws;
+    const size_t es = p->dtype == SA_F32 ? 4 : 2;
+    const size_t row = (size_t)d.L * kD * es;                          // one problem's matrix
+    const size_t strow = (size_t)(2 * d.R + 2) * d.ld * sizeof(float);  // one problem's state
+    const bool db = p->dustbin != 0;
+    uint8_t* mask_d = io->mask ? (uint8_t*)(w + l.mask_off) : nullptr;
+    float* vd_d = (db && io->v_dust) ? (float*)(w + l.vd_off) : nullptr;
+    float* acc_dvd = (float*)(w + l.acc_dvd_off);
+    float* acc_dsc = (float*)(w + l.acc_dsc_off);
+
+    cudaEvent_t ev_start, ev_const, ev_end, ev_in[2], ev_comp[2], ev_out[2];
+    cudaEvent_t* all[] = {&ev_start, &ev_const, &ev_end, &ev_in[0], &ev_in[1],
+                          &ev_comp[0], &ev_comp[1], &ev_out[0], &ev_out[1]};
+    for (cudaEvent_t* e : all)
+        if (cudaEventCreateWithFlags(e, cudaEventDisableTiming) != cudaSuccess) return SA_ERR_CUDA;
+    auto fail = [&](sa_status st) {
+        for (cudaEvent_t* e : all) cudaEventDestroy(*e);
+        return st;
+    };
+#define SA_HS(call)                                  \
+    do {                                             \
+        if ((call) != cudaSuccess) return fail(SA_ERR_CUDA); \
+    } while (0)
+    // nothing here starts before the work already queued on the caller's stream
+    SA_HS(cudaEventRecord(ev_start, cs));
+    SA_HS(cudaStreamWaitEvent(h2d, ev_start, 0));
+    SA_HS(cudaStreamWaitEvent(d2h, ev_start, 0));
+    if (mask_d) SA_HS(cudaMemcpyAsync(mask_d, io->mask, (size_t)d.B * d.L, cudaMemcpyHostToDevice, h2d));
+    if (vd_d)
+        SA_HS(cudaMemcpyAsync(vd_d, io->v_dust, (size_t)d.H * kD * sizeof(float),
+                              cudaMemcpyHostToDevice, h2d));
+    SA_HS(cudaEventRecord(ev_const, h2d));
+    SA_HS(cudaStreamWaitEvent(cs, ev_const, 0));
+    if (db) {
+        SA_HS(cudaMemsetAsync(acc_dvd, 0, (size_t)d.H * kD * sizeof(float), cs));
+        SA_HS(cudaMemsetAsync(acc_dsc, 0, sizeof(float), cs));
+    }
+    const void* hin[4] = {io->q, io->k, io->v, io->dO};
+    void* hout[4] = {io->o, io->dq, io->dk, io->dv};
+    for (size_t gi = 0; gi < gs.size(); ++gi) {
+        const Group& g = gs[gi];
+        const int sl = (int)(gi & 1);
+        char* slot = w + sl * l.slot;
+        const size_t first = (size_t)g.b0 * d.H + g.h0;  // first (batch, head) problem
+        const size_t np = (size_t)g.nb * g.nh;
+        // inputs: after the compute of the group that used this slot before
+        if (gi >= 2) SA_HS(cudaStreamWaitEvent(h2d, ev_comp[sl], 0));
+        for (int t = 0; t < 4; ++t)
+            SA_HS(cudaMemcpyAsync(slot + l.mat_off[t], (const char*)hin[t] + first * row, np * row,
+                                  cudaMemcpyHostToDevice, h2d));
+        SA_HS(cudaEventRecord(ev_in[sl], h2d));
+        // compute: after the inputs, and after the previous results left this slot
+        SA_HS(cudaStreamWaitEvent(cs, ev_in[sl], 0));
+        if (gi >= 2) SA_HS(cudaStreamWaitEvent(cs, ev_out[sl], 0));
+        const sa_params q = group_params(p, g);
+        const uint8_t* mk = mask_d ? mask_d + (size_t)g.b0 * d.L : nullptr;
+        const float* vd = vd_d ? vd_d + (size_t)g.h0 * kD : nullptr;
+        float* st = (float*)(slot + l.st_off);
+        float* dvd = (float*)(slot + l.dvd_off);
+        float* dsc = (float*)(slot + l.dsc_off);
+        s = fwd_call(&q, nullptr, slot + l.mat_off[0], slot + l.mat_off[1], slot + l.mat_off[2], mk,
+                     vd, slot + l.mat_off[4], st, slot + l.fws_off, l.fws, cs);
+        if (s != SA_OK) return fail(s);
+        s = bwd_call(&q, nullptr, slot + l.mat_off[0], slot + l.mat_off[1], slot + l.mat_off[2], mk,
+                     vd, slot + l.mat_off[4], slot + l.mat_off[3], st, slot + l.mat_off[5],
+                     slot + l.mat_off[6], slot + l.mat_off[7], db ? dvd : nullptr,
+                     db ? dsc : nullptr, slot + l.bws_off, l.bws, cs);
+        if (s != SA_OK) return fail(s);
+        if (db) {
+            sa::k_add<<<(d.H * kD + 255) / 256, 256, 0, cs>>>(acc_dvd, dvd, d.H * kD);
+            sa::k_add<<<1, 32, 0, cs>>>(acc_dsc, dsc, 1);
+            SA_HS(cudaGetLastError());
+        }
+        SA_HS(cudaEventRecord(ev_comp[sl], cs));
+        // results: after the compute
+        SA_HS(cudaStreamWaitEvent(d2h, ev_comp[sl], 0));
+        for (int t = 0; t < 4; ++t)
+            SA_HS(cudaMemcpyAsync((char*)hout[t] + first * row, slot + l.mat_off[4 + t], np * row,
+                                  cudaMemcpyDeviceToHost, d2h));
+        if (io->state)
+            SA_HS(cudaMemcpyAsync((char*)io->state + first * strow, st, np * strow,
+                                  cudaMemcpyDeviceToHost, d2h));
+        SA_HS(cudaEventRecord(ev_out[sl], d2h));
+    }
+    if (db && io->dv_dust)
+        SA_HS(cudaMemcpyAsync(io->dv_dust, acc_dvd, (size_t)d.H * kD * sizeof(float),
+                              cudaMemcpyDeviceToHost, cs));
+    if (db && io->d_dust_score)
+        SA_HS(cudaMemcpyAsync(io->d_dust_score, acc_dsc, sizeof(float), cudaMemcpyDeviceToHost, cs));
+    // the caller's stream covers every copy
+    SA_HS(cudaEventRecord(ev_end, d2h));
+    SA_HS(cudaStreamWaitEvent(cs, ev_end, 0));
+#undef SA_HS
+    fail(SA_OK);  // events are released once their work completes
+    return SA_OK;
 }
 
 }  // extern "C"

@@ -332,6 +332,8 @@ def main():
     ap.add_argument("--schedule", default="one_reference", choices=["one_reference", "direct"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--e2e-groups", type=int, default=5,
+                    help="problem groups the host-buffer call pipelines its copies over")
     ap.add_argument("--bias-certificate", action="store_true",
                     help="instead of timing steps, print the bias certificate eta_R of the "
                          "workload's solve (N = T + R iterations) on one GPU")
@@ -460,21 +462,26 @@ def main():
     # e2e: pinned host inputs in, results out, inside the timed region
     e2e = None
     if not args.no_e2e:
+        # the library's host-buffer call: it copies groups of problems in and results
+        # out on its own copy streams while other groups compute
         hq, hk, hv, hdO = (t.to("cpu").pin_memory() for t in (q, k, v, dO))
+        hmask = None if mask is None else mask.to("cpu").contiguous().pin_memory()
+        hvd = None if d["v_dust"] is None else d["v_dust"].to("cpu").contiguous().pin_memory()
         ho, hdq, hdk, hdv = (torch.empty(q.shape, dtype=q.dtype).pin_memory() for _ in range(4))
-        h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hdO))
+        h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hdO, hmask, hvd)
+                  if t is not None)
         d2h = sum(t.numel() * t.element_size() for t in (ho, hdq, hdk, hdv))
-        dq2, dk2, dv2 = (torch.empty_like(q) for _ in range(3))
-        qq, kk, vv, dd = (torch.empty_like(q) for _ in range(4))
+        ph = sa.make_params(w.B, w.H, w.L, w.d, W=w.W, eps=w.eps, T=w.T, R=w.R, dtype=q.dtype,
+                            dustbin=w.dustbin, schedule=args.schedule)
+        ws_h = torch.empty(sa.sinkhorn_attn_step_host_workspace_size(ph, args.e2e_groups),
+                           dtype=torch.uint8, device=dev)
+        kwh = dict(W=w.W, eps=w.eps, R=w.R, mask=hmask, dustbin=w.dustbin,
+                   dustbin_score=w.dustbin_score, v_dust=hvd)
 
         def e2e_step():
-            for dst, src in ((qq, hq), (kk, hk), (vv, hv), (dd, hdO)):
-                dst.copy_(src, non_blocking=True)
-            o_, st_ = sa.sinkhorn_attn_fwd(qq, kk, vv, T=w.T, o=o, state=state, ws=ws_f, **kw)
-            sa.sinkhorn_attn_bwd(qq, kk, vv, o_, dd, st_, schedule=args.schedule, dq=dq2,
-                                 dk=dk2, dv=dv2, ws=ws_b, **kw)
-            for dst, src in ((ho, o_), (hdq, dq2), (hdk, dk2), (hdv, dv2)):
-                dst.copy_(src, non_blocking=True)
+            sa.sinkhorn_attn_step_host(hq, hk, hv, hdO, T=w.T, schedule=args.schedule,
+                                       groups=args.e2e_groups, o=ho, dq=hdq, dk=hdk, dv=hdv,
+                                       ws=ws_h, **kwh)
 
         e2e_step()
         torch.cuda.synchronize()
@@ -492,7 +499,8 @@ def main():
         etot = allreduce_max(sum(ems), ws)
         e2e = {"value": ws * units / (etot / args.steps * 1e-3), "unit": UNIT,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-               "ms_per_step": etot / args.steps}
+               "ms_per_step": etot / args.steps, "api": "sinkhorn_attn_step_host",
+               "groups": args.e2e_groups}
 
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:

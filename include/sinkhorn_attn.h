@@ -207,6 +207,43 @@ sa_status sinkhorn_attn_bwd_sharded(const sa_params* p, const sa_shard* shard, c
                                     void* dk, void* dv, void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * One forward + backward step with inputs and results in host memory (no
+ * counterpart in the pages).  Every (batch, head) problem is independent, so
+ * the problems are split into `groups` contiguous groups (whole batches, or
+ * runs of heads within one batch when there are fewer batches than groups;
+ * whole batches with a dustbin) and pipelined: group g+1's inputs are copied
+ * to the device and group g-1's results back while group g runs
+ * sinkhorn_attn_fwd and sinkhorn_attn_bwd, on two copy streams of the library
+ * ordered against `stream` with events.  Host buffers should be page-locked
+ * (cudaHostAlloc / cudaHostRegister) for the copies to overlap; pageable
+ * memory works, serialised by the driver.  The call returns once everything is
+ * enqueued; the results are in host memory when `stream` reaches that point
+ * (synchronise it before reading them).
+ */
+typedef struct {
+    const void *q, *k, *v, *dO;  /* host [B][H][L][d] dtype */
+    const uint8_t* mask;         /* host [B][L] uint8, or NULL (all valid) */
+    const float* v_dust;         /* host [H][d] float32, or NULL (zero); dustbin only */
+    void *o, *dq, *dk, *dv;      /* host [B][H][L][d] dtype, written */
+    float* state;                /* host [B][H][2R+2][L+dustbin] float32, written, or NULL */
+    float* dv_dust;              /* host [H][d] float32, written, or NULL; dustbin only */
+    float* d_dust_score;         /* host, one float32, written, or NULL; dustbin only */
+    int groups;                  /* >= 1; 3-8 overlap copies with compute */
+} sa_host_step;
+
+/* Device workspace bytes for sinkhorn_attn_step_host with `groups` groups:
+ * two groups' device copies of inputs and results plus their fwd/bwd
+ * workspaces. */
+sa_status sinkhorn_attn_step_host_workspace_size(const sa_params* p, int groups, size_t* bytes);
+
+/* SA_ERR_INVALID_ARG for a device pointer where host memory is expected, a NULL
+ * input or output, or groups < 1; SA_ERR_UNSUPPORTED with check_finite;
+ * SA_ERR_WORKSPACE below the size above; otherwise the statuses of the
+ * forward and backward. */
+sa_status sinkhorn_attn_step_host(const sa_params* p, const sa_host_step* io, void* ws,
+                                  size_t ws_bytes, void* stream);
+
+/*
  * Test hook: the plan P^(a,b) (0 <= a, b <= R) from a finished forward state.
  *   band : [B][H][L][2W+1] float32, entry t of row i is column i-W+t (0 off Omega).
  *   dcol : [B][H][L] float32 entries (i, dustbin), or NULL.

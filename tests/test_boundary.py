@@ -163,3 +163,27 @@ def test_sharded_calls_validate_the_shard_on_the_host():
     pd = P(B=1, H=1, L=50, W=4, dustbin=True)
     assert lib.sinkhorn_attn_fwd_sharded(ctypes.byref(pd), ctypes.byref(sa.sa_shard(4, 4, noop, None)),
                                          *([None] * 7), 1 << 30, None) == -2      # dustbin
+
+
+def test_host_step_plans_and_validates_on_the_host():
+    lib = sa._L()
+    p = P(B=1, H=8, L=100)
+    # two slots of the largest group: more groups, smaller workspace
+    w1, w4, w8 = (sa.sinkhorn_attn_step_host_workspace_size(p, g) for g in (1, 4, 8))
+    assert w1 > w4 > w8 > 0
+    with pytest.raises(sa.SinkhornAttnError):
+        sa.sinkhorn_attn_step_host_workspace_size(p, 0)
+    io = sa.sa_host_step()
+    io.groups = 0
+    assert lib.sinkhorn_attn_step_host(ctypes.byref(p), ctypes.byref(io), None, 1 << 40, None) == -1
+    assert lib.sinkhorn_attn_step_host(ctypes.byref(p), None, None, 1 << 40, None) == -1
+    io.groups = 2
+    assert lib.sinkhorn_attn_step_host(ctypes.byref(p), ctypes.byref(io), None, 16, None) == -3
+    pc = P(B=1, H=8, L=100, check_finite=True)
+    assert lib.sinkhorn_attn_step_host(ctypes.byref(pc), ctypes.byref(io), None, 1 << 40, None) == -2
+    # host buffers present, but the workspace is not device memory
+    buf = torch.zeros(8 * 100 * 64)
+    for f in ("q", "k", "v", "dO", "o", "dq", "dk", "dv"):
+        setattr(io, f, buf.data_ptr())
+    assert lib.sinkhorn_attn_step_host(ctypes.byref(p), ctypes.byref(io), buf.data_ptr(), 1 << 40,
+                                       None) == -1
