@@ -428,9 +428,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fused_iter(const FusedArgs a,
         const uint32_t lanebase = (uint32_t)(qd * 32) << 16;
         const float c2 = a.c2;
         ChunkIds ids;
-        // partial of column 128c + lr of tile it_prev (tile t0 + it_prev), from
-        // its two accumulators in TMEM (complete) and the quadrant scales
-        auto put_partial = [&](int it_prev, int c) {
+        // partial of column 128c + lr of tile it_prev (problem pbh, row block prb),
+        // from its two accumulators in TMEM (complete) and the quadrant scales
+        auto put_partial = [&](int it_prev, int pbh, int prb, int c) {
             uint32_t d0[8], d1[8];
             tmem_ld8(tD + lanebase + 32 * c, d0);
             tmem_ld8(tD + lanebase + 32 * c + 16, d1);
@@ -441,14 +441,21 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fused_iter(const FusedArgs a,
             for (int q = 0; q < 4; ++q)
                 s = fmaf(wm[q], (__uint_as_float(d0[2 * q]) + __uint_as_float(d0[2 * q + 1])) +
                                     (__uint_as_float(d1[2 * q]) + __uint_as_float(d1[2 * q + 1])), s);
-            const int tp = t0 + it_prev, pbh = tp / nblk, prb = tp % nblk;
             const int cc = 128 * c + lr, col = prb * 128 - W + cc;
             if (cc < a.ncol && col >= 0 && col < L)
                 a.part_out[((size_t)pbh * L + col) * NSLOT + (prb & (NSLOT - 1))] = s;
         };
         bool ok = true;
+        // (problem, row block) of tile t0 + it, advanced without divisions, and
+        // of the tile before it
+        int bh = t0 / nblk, rb = t0 % nblk, pbh = 0, prb = 0;
         for (int it = 0; ok && it < ntl; ++it) {
-            const int t = t0 + it, bh = t / nblk, rb = t % nblk, r0 = rb * 128;
+            if (it > 0) {
+                pbh = bh;
+                prb = rb;
+                if (++rb == nblk) { rb = 0; ++bh; }
+            }
+            const int r0 = rb * 128;
             const int r = r0 + lr, rw0 = r0 + qd * 32;
             ids.advance(it > 0 && rb > 0, nch);
             if (!ctl.wait(B_CVFULL + (it & 1), (it >> 1) & 1)) { ok = false; break; }
@@ -498,7 +505,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fused_iter(const FusedArgs a,
                 // the previous tile's column sums of chunk c (complete: waited above)
                 if (it >= 1 && hf == 0) {
                     tc::tc_fence_after();
-                    put_partial(it - 1, c);
+                    put_partial(it - 1, pbh, prb, c);
                 }
             }
             if (!ok) break;
@@ -551,7 +558,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fused_iter(const FusedArgs a,
         // the last tile's partials
         if (ok && ntl >= 1 && !*abort_flag && ctl.wait(B_CS + nch - 1, (ntl - 1) & 1)) {
             tc::tc_fence_after();
-            for (int c = pt; c < nch; c += NQ) put_partial(ntl - 1, c);
+            for (int c = pt; c < nch; c += NQ) put_partial(ntl - 1, bh, rb, c);
             tc::tc_fence_before();
         }
     }

@@ -164,20 +164,30 @@ __global__ void __launch_bounds__(nthreads(MODE), ctas_per_sm(MODE)) tc_band_swe
     const int t0 = (int)(((long long)blockIdx.x * ntiles) / gridDim.x);
     const int t1 = (int)(((long long)(blockIdx.x + 1) * ntiles) / gridDim.x);
     const int ntl = t1 - t0;
-    // geometry of tile it of the range
+    // geometry of a tile; the tiles of the range are walked with a (batch, head,
+    // row block) cursor, so that no role divides by a runtime value per tile
     struct Tile {
         int bh, r0, cbeg, cend, nch;
         const uint8_t* mk;
     };
-    auto tile = [&](int it) {
+    struct Cursor {
+        int rb, h, b;
+        __device__ void next(int nb, int H) {
+            if (++rb == nb) {
+                rb = 0;
+                if (++h == H) { h = 0; ++b; }
+            }
+        }
+    };
+    const Cursor cur0{t0 % nblk, (t0 / nblk) % a.H, (t0 / nblk) / a.H};
+    auto tile = [&](const Cursor& c) {
         Tile g;
-        const int t = t0 + it;
-        g.bh = t / nblk;
-        g.r0 = (t % nblk) * 128;
+        g.bh = c.b * a.H + c.h;
+        g.r0 = c.rb * 128;
         g.cbeg = max(0, g.r0 - W);
         g.cend = min(L, g.r0 + 127 + W + 1);
         g.nch = (g.cend - g.cbeg + 127) / 128;
-        g.mk = a.mask ? a.mask + (size_t)(g.bh / a.H) * L : nullptr;
+        g.mk = a.mask ? a.mask + (size_t)c.b * L : nullptr;
         return g;
     };
 
@@ -220,8 +230,9 @@ __global__ void __launch_bounds__(nthreads(MODE), ctas_per_sm(MODE)) tc_band_swe
         }
         int gc = 0, issued = 0, a_issued = 0;
         bool ok = true;
-        for (int it = 0; ok && it < ntl; ++it) {
-            const Tile tl = tile(it);
+        Cursor cur = cur0;
+        for (int it = 0; ok && it < ntl; ++it, cur.next(nblk, a.H)) {
+            const Tile tl = tile(cur);
             const int ab = it % NAB;
             if (lane == 0) {
                 if (it >= NAB && !ctl.wait(B_AEMPTY + ab, ((it / NAB) - 1) & 1)) ok = false;
@@ -341,8 +352,9 @@ __global__ void __launch_bounds__(nthreads(MODE), ctas_per_sm(MODE)) tc_band_swe
             bool ok = true;
             int gc = 0;
             int pg = -1, pit = 0, pc = 0, pn = 0;  // the chunk whose P X is still to issue
-            for (int it = 0; ok && it < ntl; ++it) {
-                const Tile tl = tile(it);
+            Cursor cur = cur0;
+            for (int it = 0; ok && it < ntl; ++it, cur.next(nblk, a.H)) {
+                const Tile tl = tile(cur);
                 const int ab = it % NAB;
                 if (!ctl.wait(B_AFULL + ab, (it / NAB) & 1)) { ok = false; break; }
                 const uint64_t dA = tc::sdesc_add(dA0, off_a(MODE, ab));
@@ -415,9 +427,10 @@ __global__ void __launch_bounds__(nthreads(MODE), ctas_per_sm(MODE)) tc_band_swe
                 }
             }
         };
-        if (ntl >= 1) load_rows(tile(0));
-        for (int it = 0; ok && it < ntl; ++it) {
-            const Tile tl = tile(it);
+        if (ntl >= 1) load_rows(tile(cur0));
+        Cursor cur = cur0;
+        for (int it = 0; ok && it < ntl; ++it, cur.next(nblk, a.H)) {
+            const Tile tl = tile(cur);
             const int bh = tl.bh, r0 = tl.r0, cbeg = tl.cbeg, nch = tl.nch;
             const int r = r0 + lr;              // global row
             const int rw0 = r0 + qd * 32;       // first row of this warp
@@ -629,7 +642,11 @@ __global__ void __launch_bounds__(nthreads(MODE), ctas_per_sm(MODE)) tc_band_swe
             // what the finish still needs of this tile; then the next tile's rows
             const float rd2f = rd2;
             const bool rokf = rok;
-            if (it + 1 < ntl) load_rows(tile(it + 1));
+            if (it + 1 < ntl) {
+                Cursor nx = cur;
+                nx.next(nblk, a.H);
+                load_rows(tile(nx));
+            }
 
             // ---------------------------------------------------------- finish
             if ((MODE == LSE && !ONLINE) || MODE == WSUM) {
