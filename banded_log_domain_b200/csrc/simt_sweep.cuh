@@ -75,6 +75,11 @@ struct SweepArgs {
     int acc_in;             // 1: add acc's contents to this launch's result
     int acc_out;            // 1: write the sum to acc instead of out_mat
     int g_off;              // DS1: leave G out of M (every block but the first)
+    // DS1 on tensor cores with at most five terms: the modifier's K16 operands,
+    // bf16 [BH][L][16], row side (hi, hi, lo) and column side (hi, lo, hi) of each
+    // term (or null: the modifier is formed in the epilogue)
+    const void* aug_row;
+    const void* aug_col;
     int online;             // LSE on tensor cores: 1 = no previous dual, use a running max
 };
 

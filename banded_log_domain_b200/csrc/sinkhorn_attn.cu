@@ -140,7 +140,7 @@ FwdLayout fwd_layout(const Dims& d, const sa_params* p) {
 
 // Backward workspace layout (float32 vectors of BH * ld elements each).
 struct BwdLayout {
-    size_t a, ubar, vbar, eu, ev, w, rv, cv, dvd, dsc, acc, total;
+    size_t a, ubar, vbar, eu, ev, w, rv, cv, dvd, dsc, aug, acc, total;
     size_t vec;  // bytes of one [BH][ld] vector, 256-aligned
 };
 BwdLayout bwd_layout(const Dims& d) {
@@ -157,6 +157,7 @@ BwdLayout bwd_layout(const Dims& d) {
     l.cv = o;   o += l.vec * 2 * d.R;
     l.dvd = o;  o += align_up((size_t)d.BH * kD * sizeof(float));
     l.dsc = o;  o += align_up((size_t)d.BH * sizeof(double));  // dustbin score, per problem
+    l.aug = o;  o += 4 * align_up((size_t)d.BH * d.L * 16 * 2);  // bf16 K16 modifier operands
     l.acc = o;  // fp32 sum of the dS sweeps' term blocks, when 2R > MAXT
     if (2 * d.R > simt::MAXT) o += align_up((size_t)d.BH * d.L * kD * sizeof(float));
     l.total = o;
@@ -303,6 +304,41 @@ __global__ void k_sum_parts(const double* part, int n, float* out) {
     if (threadIdx.x == 0) out[0] = (float)red[0];
 }
 
+// The dS sweep's modifier as K16 operands of the dO V^T contraction:
+// out[bh][t][16] bf16, slots 3k, 3k+1, 3k+2 of term k < n holding the bf16
+// halves (hi, hi, lo) of v_k[bh][t] for the row side and (hi, lo, hi) for the
+// column side (v_k with a null pointer: 1), the other slots 0.
+struct AugTerms {
+    Vec v[4];
+    int n;
+    int row;
+};
+__global__ void k_aug(AugTerms tm, int L, int BH, __nv_bfloat16* out) {
+    const long long g = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (g >= (long long)BH * L) return;
+    const int bh = (int)(g / L), t = (int)(g % L);
+    uint16_t sl[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) sl[i] = 0;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        if (k >= tm.n) break;
+        const float v = tm.v[k].p ? tm.v[k].at(bh, t) : 1.f;
+        const __nv_bfloat16 hi = __float2bfloat16_rn(v);
+        const __nv_bfloat16 lo = __float2bfloat16_rn(v - __bfloat162float(hi));
+        const uint16_t h = __bfloat16_as_ushort(hi), l = __bfloat16_as_ushort(lo);
+        sl[3 * k] = h;
+        sl[3 * k + 1] = tm.row ? h : l;
+        sl[3 * k + 2] = tm.row ? l : h;
+    }
+    uint32_t w[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) w[i] = (uint32_t)sl[2 * i] | ((uint32_t)sl[2 * i + 1] << 16);
+    uint4* o = reinterpret_cast<uint4*>(out + (size_t)g * 16);
+    o[0] = make_uint4(w[0], w[1], w[2], w[3]);
+    o[1] = make_uint4(w[4], w[5], w[6], w[7]);
+}
+
 // out[0] += sum_i (x_i - y_i)^2, out[1] += sum_i y_i^2 in double: grid-stride
 // loop, warp shuffles, one atomic pair per warp.
 template <typename T>
@@ -446,6 +482,20 @@ bool make_map(CUtensorMap* m, const void* ptr, int L, int BH) {
            CUDA_SUCCESS;
 }
 
+// [BH][L][16] bf16 (the dS modifier's K16 operands), 128-token boxes, 32-byte swizzle
+bool make_map_aug(CUtensorMap* m, const void* ptr, int L, int BH) {
+    auto fn = encode_tiled();
+    if (!fn || !ptr) return false;
+    cuuint64_t dims[3] = {16, (cuuint64_t)L, (cuuint64_t)BH};
+    cuuint64_t strides[2] = {16 * 2, (cuuint64_t)L * 16 * 2};
+    cuuint32_t box[3] = {16, 128, 1};
+    cuuint32_t es[3] = {1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box,
+              es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_32B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+           CUDA_SUCCESS;
+}
+
 template <int MODE, bool ONLINE, int NT>
 cudaError_t launch_tc(const simt::SweepArgs& a, int BH, cudaStream_t st, Tracer& tr,
                       int* status) {
@@ -454,6 +504,8 @@ cudaError_t launch_tc(const simt::SweepArgs& a, int BH, cudaStream_t st, Tracer&
     bool ok = make_map(&maps.A, a.A, a.L, BH) && make_map(&maps.B, a.Bo, a.L, BH);
     if (tcs::is_ds(MODE)) ok = ok && make_map(&maps.A2, a.A2, a.L, BH) && make_map(&maps.B2, a.B2, a.L, BH);
     if (MODE == simt::PV) ok = ok && make_map(&maps.X, a.X, a.L, BH);
+    if (tcs::aug(MODE, NT))
+        ok = ok && make_map_aug(&maps.AR, a.aug_row, a.L, BH) && make_map_aug(&maps.AC, a.aug_col, a.L, BH);
     if (!ok) return cudaErrorInvalidValue;
     // persistent: one CTA per SM (two for LSE and WSUM), each a contiguous tile range
     static int nsm = 0;
@@ -465,7 +517,7 @@ cudaError_t launch_tc(const simt::SweepArgs& a, int BH, cudaStream_t st, Tracer&
     }
     const long long ntiles = (long long)((a.L + 127) / 128) * BH;
     const dim3 grid((unsigned)std::min<long long>(ntiles, (long long)nsm * tcs::ctas_per_sm(MODE)));
-    const int smem = tcs::smem_bytes(MODE);
+    const int smem = tcs::smem_bytes(MODE, NT);
     cudaError_t e = cudaFuncSetAttribute(tcs::tc_band_sweep<MODE, ONLINE, NT>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
@@ -846,10 +898,33 @@ sa_status bwd_impl(const Ctx& x, const T* q, const T* k, const T* v, const uint8
     // dQ (query sweep) and dK (key sweep).  A sweep takes at most MAXT terms;
     // longer tails (R > MAXT / 2) run one sweep per block of MAXT terms (the
     // first block carrying G), summed in fp32 in the workspace and rounded once.
+    // The first block takes the remainder of 2R over MAXT, so that it carries G
+    // and the full blocks follow it.
     const int nblk_t = std::max(1, (nt + simt::MAXT - 1) / simt::MAXT);
+    const int first = (nt % simt::MAXT) ? nt % simt::MAXT : std::min(nt, simt::MAXT);
+    // On the tensor cores a first block of at most four terms adds its modifier
+    // to G inside the contraction: its K16 operands, per side (rows of the query
+    // sweep and columns of the key sweep come from rq; the others from rk).
+    __nv_bfloat16* augs[4] = {nullptr, nullptr, nullptr, nullptr};  // row q, col k, row k, col q
+    if (std::is_same<T, __nv_bfloat16>::value && !x.p->dustbin && !direct && first > 0 &&
+        first <= 4) {
+        const size_t one = align_up((size_t)d.BH * d.L * 16 * 2);
+        const long long n = (long long)d.BH * d.L;
+        for (int i = 0; i < 4; ++i) {
+            augs[i] = (__nv_bfloat16*)(ws + l.aug + i * one);
+            AugTerms tm;
+            for (int k = 0; k < 4; ++k) tm.v[k] = Vec{nullptr, 0};
+            const bool from_q = (i == 0 || i == 3);
+            for (int k = 0; k < first; ++k) tm.v[k] = from_q ? rq[k] : rk[k];
+            tm.n = first;
+            tm.row = (i == 0 || i == 2);
+            SA_AUX(x.tr, k_aug<<<(unsigned)((n + 255) / 256), 256, 0, x.st>>>(tm, d.L, d.BH, augs[i]));
+        }
+    }
     for (int side = 0; side < 2; ++side) {
         for (int tb = 0; tb < nblk_t; ++tb) {
-            const int k0 = tb * simt::MAXT, kn = std::min(simt::MAXT, nt - k0);
+            const int k0 = tb == 0 ? 0 : first + (tb - 1) * simt::MAXT;
+            const int kn = tb == 0 ? first : simt::MAXT;
             simt::SweepArgs a = base_args(x);
             a.mask = mask;
             a.dust_cta = 0;
@@ -859,6 +934,10 @@ sa_status bwd_impl(const Ctx& x, const T* q, const T* k, const T* v, const uint8
                 a.acc_in = tb > 0;
                 a.acc_out = tb + 1 < nblk_t;
                 a.g_off = tb > 0;
+            }
+            if (tb == 0) {
+                a.aug_row = augs[side == 0 ? 0 : 2];
+                a.aug_col = augs[side == 0 ? 1 : 3];
             }
             if (side == 0) {
                 a.A = q; a.Bo = k; a.A2 = dO; a.B2 = v; a.X = k;

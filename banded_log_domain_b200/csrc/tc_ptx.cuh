@@ -160,6 +160,18 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo_byt
     d |= (uint64_t)2 << 61;
     return d;
 }
+// Shared-memory matrix descriptor of a K-major operand whose rows are 32 bytes
+// (16 bf16) in the 32-byte swizzle that TMA writes with SWIZZLE_32B: 8-row
+// atoms of 256 bytes, one after another.
+__device__ __forceinline__ uint64_t sdesc_sw32(uint32_t saddr) {
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+    d |= (uint64_t)1 << 16;                 // leading byte offset (unused: K fits one atom)
+    d |= (uint64_t)(256 >> 4) << 32;        // 8-row atom stride
+    d |= (uint64_t)1 << 46;
+    d |= (uint64_t)6 << 61;                 // 32-byte swizzle
+    return d;
+}
 // The descriptor of the same matrix `bytes` further on (bytes a multiple of
 // 16; shared-memory addresses stay below 256 KB, so the 14-bit start field
 // does not carry).  Building descriptors once and advancing them this way keeps

@@ -45,15 +45,24 @@ constexpr int TILE = 16384;  // one 128 x 64 bf16 tile
 constexpr long long kWaitBudget = 4000000000LL;  // clock cycles (about 2 s)
 
 struct Maps {
-    CUtensorMap A, B, A2, B2, X;
+    CUtensorMap A, B, A2, B2, X, AR, AC;  // AR, AC: the modifier's K16 operands (DS1)
 };
 
 __host__ __device__ constexpr bool is_ds(int m) { return m == DS1 || m == DSD; }
 __host__ __device__ constexpr bool has_x(int m) { return m == PV || is_ds(m); }
 __host__ __device__ constexpr int nst(int m) { return is_ds(m) ? 3 : (m == PV ? 3 : 4); }
 __host__ __device__ constexpr int nsb(int m) { return is_ds(m) ? 1 : 2; }
-__host__ __device__ constexpr int ncv(int m) {
-    return m == WSUM ? 2 : (m == DS1 ? 1 + MAXT : (m == DSD ? 2 * MAXT : 1));
+// DS1 with at most five modifier terms adds the modifier to G on the tensor
+// core: one more K16 step of the dO V^T contraction whose operands, prepared
+// once per sweep in global memory and brought in by TMA with the other
+// operands, hold per row (rv_hi, rv_hi, rv_lo) and per column (cv_hi, cv_lo,
+// cv_hi) of every term (bf16 halves, rv = rv_hi + rv_lo), so that
+//   sum_k rv_k cv_k ~ sum_k rv_hi cv_hi + rv_hi cv_lo + rv_lo cv_hi
+// to about 2^-16 of each product, far below the bf16 rounding of dS.
+__host__ __device__ constexpr bool aug(int m, int nt) { return m == DS1 && nt > 0 && 3 * nt <= 16; }
+// column vectors staged per operand stage
+__host__ __device__ constexpr int ncv(int m, int nt) {
+    return m == WSUM ? 2 : (m == DS1 ? (aug(m, nt) ? 1 : 1 + nt) : (m == DSD ? 2 * MAXT : 1));
 }
 __host__ __device__ constexpr int stage_bytes(int m) {
     return TILE * (1 + (is_ds(m) ? 1 : 0) + (m == PV ? 1 : 0));
@@ -72,9 +81,17 @@ __host__ __device__ constexpr int off_a2(int m) { return TILE; }
 __host__ __device__ constexpr int off_stage(int m) { return 2 * TILE; }
 __host__ __device__ constexpr int off_p(int m) { return off_stage(m) + nst(m) * stage_bytes(m); }
 __host__ __device__ constexpr int off_cv(int m) { return off_p(m) + (has_x(m) ? 2 * 2 * TILE : 0); }
-__host__ __device__ constexpr int off_red(int m) { return off_cv(m) + nst(m) * ncv(m) * 128 * 4; }
-__host__ __device__ constexpr int off_bar(int m) { return off_red(m) + 2 * 4 * 128 * 4; }
-__host__ __device__ constexpr int smem_bytes(int m) { return off_bar(m) + 64 * 8 + 64 + 1024; }
+// the modifier's K16 operand tiles (aug): the row block's, then one per operand
+// stage, 4 KB each (128 rows x 32 bytes), 1024-aligned
+constexpr int AUG_BYTES = 4096;
+__host__ __device__ constexpr int off_aug(int m, int nt) {
+    return (off_cv(m) + nst(m) * ncv(m, nt) * 128 * 4 + 1023) / 1024 * 1024;
+}
+__host__ __device__ constexpr int off_red(int m, int nt) {
+    return aug(m, nt) ? off_aug(m, nt) + (1 + nst(m)) * AUG_BYTES : off_cv(m) + nst(m) * ncv(m, nt) * 128 * 4;
+}
+__host__ __device__ constexpr int off_bar(int m, int nt) { return off_red(m, nt) + 2 * 4 * 128 * 4; }
+__host__ __device__ constexpr int smem_bytes(int m, int nt) { return off_bar(m, nt) + 64 * 8 + 64 + 1024; }
 
 // barrier slots (pairs indexed by tile parity, chunk parity or buffer)
 enum { B_AFULL = 0, B_AEMPTY = 2, B_FULL = 4, B_EMPTY = 8, B_SFULL = 12, B_SEMPTY = 14,
@@ -104,8 +121,8 @@ struct Ctl {
 };
 
 // the chunk's column vector k (128 floats) in stage s
-__device__ __forceinline__ float* colvec(uint8_t* sm, int mode, int s, int k) {
-    return reinterpret_cast<float*>(sm + off_cv(mode)) + (s * ncv(mode) + k) * 128;
+__device__ __forceinline__ float* colvec(uint8_t* sm, int mode, int nt, int s, int k) {
+    return reinterpret_cast<float*>(sm + off_cv(mode)) + (s * ncv(mode, nt) + k) * 128;
 }
 
 // Exponent arguments (log2 units) of one thread's 32 columns:
@@ -150,10 +167,11 @@ __global__ void __launch_bounds__(nthreads(MODE), ctas_per_sm(MODE)) tc_band_swe
     constexpr bool DS = is_ds(MODE), HASX = has_x(MODE);
     constexpr int NEPI = nepi(MODE), NPART = NEPI / 4, PW = 128 / NPART, NG = PW / 32;
     constexpr int W_LOAD = NEPI, W_MMA = NEPI + 1;
-    uint64_t* bar = reinterpret_cast<uint64_t*>(sm + off_bar(MODE));
-    uint32_t* tbase = reinterpret_cast<uint32_t*>(sm + off_bar(MODE) + 64 * 8);
+    uint64_t* bar = reinterpret_cast<uint64_t*>(sm + off_bar(MODE, NT));
+    uint32_t* tbase = reinterpret_cast<uint32_t*>(sm + off_bar(MODE, NT) + 64 * 8);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tbase + 1);
-    float* red = reinterpret_cast<float*>(sm + off_red(MODE));
+    float* red = reinterpret_cast<float*>(sm + off_red(MODE, NT));
+    constexpr bool AUG = aug(MODE, NT);
     Ctl ctl{bar, abort_flag, status};
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -237,9 +255,10 @@ __global__ void __launch_bounds__(nthreads(MODE), ctas_per_sm(MODE)) tc_band_swe
             if (lane == 0) {
                 if (it >= NAB && !ctl.wait(B_AEMPTY + ab, ((it / NAB) - 1) & 1)) ok = false;
                 if (ok) {
-                    tc::mbar_expect_tx(bar + B_AFULL + ab, TILE * (DS ? 2 : 1));
+                    tc::mbar_expect_tx(bar + B_AFULL + ab, TILE * (DS ? 2 : 1) + (AUG ? AUG_BYTES : 0));
                     tc::tma_load_3d(sm + off_a(MODE, ab), &maps.A, bar + B_AFULL + ab, 0, tl.r0, tl.bh);
                     if (DS) tc::tma_load_3d(sm + off_a2(MODE), &maps.A2, bar + B_AFULL + ab, 0, tl.r0, tl.bh);
+                    if (AUG) tc::tma_load_3d(sm + off_aug(MODE, NT), &maps.AR, bar + B_AFULL + ab, 0, tl.r0, tl.bh);
                     a_issued = it + 1;
                 }
             }
@@ -252,9 +271,12 @@ __global__ void __launch_bounds__(nthreads(MODE), ctas_per_sm(MODE)) tc_band_swe
                 const uint8_t* mk = tl.mk;
                 uint8_t* st = sm + off_stage(MODE) + s * stage_bytes(MODE);
                 if (lane == 0) {
-                    tc::mbar_expect_tx(bar + B_FULL + s, stage_bytes(MODE));
+                    tc::mbar_expect_tx(bar + B_FULL + s, stage_bytes(MODE) + (AUG ? AUG_BYTES : 0));
                     tc::tma_load_3d(st, &maps.B, bar + B_FULL + s, 0, c0, bh);
                     if (DS) tc::tma_load_3d(st + TILE, &maps.B2, bar + B_FULL + s, 0, c0, bh);
+                    if (AUG)
+                        tc::tma_load_3d(sm + off_aug(MODE, NT) + AUG_BYTES * (1 + s), &maps.AC,
+                                        bar + B_FULL + s, 0, c0, bh);
                     if (MODE == PV) tc::tma_load_3d(st + TILE, &maps.X, bar + B_FULL + s, 0, c0, bh);
                 }
                 // column vectors: -inf / 0 outside [cbeg, cend) and on masked columns.
@@ -275,7 +297,7 @@ __global__ void __launch_bounds__(nthreads(MODE), ctas_per_sm(MODE)) tc_band_swe
                             if (mk) mok[k] = mk[col] != 0;
                             if (MODE != DSD) val[k][0] = a.cd.at(bh, col);
                             if (MODE == WSUM) val[k][1] = a.w.at(bh, col);
-                            if (MODE == DS1) {
+                            if (MODE == DS1 && !AUG) {
     #pragma unroll
                                 for (int e = 0; e < NT; ++e) val[k][1 + e] = a.cv[e].p ? a.cv[e].at(bh, col) : 1.f;
                             }
@@ -292,18 +314,18 @@ __global__ void __launch_bounds__(nthreads(MODE), ctas_per_sm(MODE)) tc_band_swe
                     for (int k = 0; k < 4; ++k) {
                         const int t = 32 * k + lane;
                         const bool ok = inr[k] && mok[k];
-                        colvec(sm, MODE, s, 0)[t] =
+                        colvec(sm, MODE, NT, s, 0)[t] =
                             (MODE == DSD) ? 0.f : (ok ? val[k][0] * kLog2e : -INFINITY);
-                        if (MODE == WSUM) colvec(sm, MODE, s, 1)[t] = ok ? val[k][1] : 0.f;
-                        if (MODE == DS1) {
+                        if (MODE == WSUM) colvec(sm, MODE, NT, s, 1)[t] = ok ? val[k][1] : 0.f;
+                        if (MODE == DS1 && !AUG) {
     #pragma unroll
-                            for (int e = 0; e < NT; ++e) colvec(sm, MODE, s, 1 + e)[t] = ok ? val[k][1 + e] : 0.f;
+                            for (int e = 0; e < NT; ++e) colvec(sm, MODE, NT, s, 1 + e)[t] = ok ? val[k][1 + e] : 0.f;
                         }
                         if (MODE == DSD) {
     #pragma unroll
                             for (int e = 0; e < NT; ++e) {
-                                colvec(sm, MODE, s, e)[t] = ok ? val[k][e] * kLog2e : -INFINITY;
-                                colvec(sm, MODE, s, MAXT + e)[t] = ok ? val[k][NT + e] : 0.f;
+                                colvec(sm, MODE, NT, s, e)[t] = ok ? val[k][e] * kLog2e : -INFINITY;
+                                colvec(sm, MODE, NT, s, MAXT + e)[t] = ok ? val[k][NT + e] : 0.f;
                             }
                         }
                     }
@@ -330,6 +352,7 @@ __global__ void __launch_bounds__(nthreads(MODE), ctas_per_sm(MODE)) tc_band_swe
             const uint64_t dStK = tc::sdesc_sw128(tc::smem_u32(sm + off_stage(MODE)), 16, 1024);
             const uint64_t dStMN = tc::sdesc_sw128(tc::smem_u32(sm + off_stage(MODE)), TILE, 1024);
             const uint64_t dP = tc::sdesc_sw128(tc::smem_u32(sm + off_p(MODE)), 16, 1024);
+            const uint64_t dAug = tc::sdesc_sw32(tc::smem_u32(sm + off_aug(MODE, NT)));
             // O += P X of chunk c (global chunk g) of tile it (nch chunks)
             auto issue_pv = [&](int g, int it, int c, int nch) -> bool {
                 const int pb = g & 1, s = g % NST, ob = it & 1;
@@ -373,6 +396,8 @@ __global__ void __launch_bounds__(nthreads(MODE), ctas_per_sm(MODE)) tc_band_swe
                         for (int k = 0; k < 4; ++k)
                             tc::mma_bf16(tG, tc::sdesc_add(dA2, 32 * k), tc::sdesc_add(dB, TILE + 32 * k),
                                          id_s, k > 0);
+                        if (AUG)  // + the modifier, one more K16 step
+                            tc::mma_bf16(tG, dAug, tc::sdesc_add(dAug, AUG_BYTES * (1 + s)), id_s, 1u);
                     }
                     tc::tc_commit(bar + B_SFULL + b);
                     if (!HASX) tc::tc_commit(bar + B_EMPTY + s);
@@ -419,7 +444,7 @@ __global__ void __launch_bounds__(nthreads(MODE), ctas_per_sm(MODE)) tc_band_swe
                 rmod[k] = 0.f;
                 rmod2[k] = 0.f;
                 if (r < L) {
-                    if (MODE == DS1) rmod[k] = a.rv[k].p ? a.rv[k].at(tl.bh, r) : 1.f;
+                    if (MODE == DS1 && !AUG) rmod[k] = a.rv[k].p ? a.rv[k].at(tl.bh, r) : 1.f;
                     if (MODE == DSD) {
                         rmod[k] = a.er[k].at(tl.bh, r) * kLog2e;
                         rmod2[k] = a.cr[k].p ? a.cr[k].at(tl.bh, r) : 0.f;
@@ -462,7 +487,7 @@ __global__ void __launch_bounds__(nthreads(MODE), ctas_per_sm(MODE)) tc_band_swe
                 if (HASX && gc >= 2 && !ctl.wait(B_PEMPTY + pb, ((gc >> 1) - 1) & 1)) { ok = false; break; }
                 tc::tc_fence_after();
                 const int c0 = cbeg + 128 * c;
-                const float* cvs = colvec(sm, MODE, s, 0) + PW * pt;
+                const float* cvs = colvec(sm, MODE, NT, s, 0) + PW * pt;
                 // Modes with a matrix output (one CTA per SM, registers to spare) read all
                 // of this warp's scores of the chunk (and the dO V^T tile) with one wait
                 // and free the TMEM buffer at once; the others read a group at a time.
@@ -537,7 +562,7 @@ __global__ void __launch_bounds__(nthreads(MODE), ctas_per_sm(MODE)) tc_band_swe
                                                            tc::pk2(ex2(x[2 * q]), ex2(x[2 * q + 1])));
                             } else if (MODE == WSUM) {
                                 const float4* w4 = reinterpret_cast<const float4*>(
-                                    colvec(sm, MODE, s, 1) + PW * pt + 32 * g);
+                                    colvec(sm, MODE, NT, s, 1) + PW * pt + 32 * g);
     #pragma unroll
                                 for (int q = 0; q < 8; ++q) {
                                     const float4 wv = w4[q];
@@ -556,6 +581,12 @@ __global__ void __launch_bounds__(nthreads(MODE), ctas_per_sm(MODE)) tc_band_swe
                     } else if (all_out) {
     #pragma unroll
                         for (int j = 0; j < 32; ++j) pv[j] = 0.f;
+                    } else if (MODE == DS1 && AUG) {
+                        // dS = P * M, M = G + sum_k rv_k[row] cv_k[col] from the contraction
+                        float x[32];
+                        group_args(sv, ce, rd2, c2, !all_in, r, cg, W, x);
+    #pragma unroll
+                        for (int j = 0; j < 32; ++j) pv[j] = ex2(x[j]) * gv[j];
                     } else if (MODE == DS1) {
                         // dS = P * M,  M = G + sum_k rv_k[row] cv_k[col]
                         float x[32];
@@ -567,7 +598,7 @@ __global__ void __launch_bounds__(nthreads(MODE), ctas_per_sm(MODE)) tc_band_swe
     #pragma unroll
                             for (int k = 0; k < NT; ++k) {
                                 const float4 cv = reinterpret_cast<const float4*>(
-                                    colvec(sm, MODE, s, 1 + k) + PW * pt + 32 * g)[q];
+                                    colvec(sm, MODE, NT, s, 1 + k) + PW * pt + 32 * g)[q];
                                 const uint64_t rk = tc::pk2(rmod[k], rmod[k]);
                                 m01 = tc::fma2(rk, tc::pk2(cv.x, cv.y), m01);
                                 m23 = tc::fma2(rk, tc::pk2(cv.z, cv.w), m23);
@@ -589,9 +620,9 @@ __global__ void __launch_bounds__(nthreads(MODE), ctas_per_sm(MODE)) tc_band_swe
     #pragma unroll
                             for (int k = 0; k < NT; ++k) {
                                 const float4 ev = reinterpret_cast<const float4*>(
-                                    colvec(sm, MODE, s, k) + PW * pt + 32 * g)[q];
+                                    colvec(sm, MODE, NT, s, k) + PW * pt + 32 * g)[q];
                                 const float4 cv = reinterpret_cast<const float4*>(
-                                    colvec(sm, MODE, s, MAXT + k) + PW * pt + 32 * g)[q];
+                                    colvec(sm, MODE, NT, s, MAXT + k) + PW * pt + 32 * g)[q];
                                 const uint64_t rk = tc::pk2(rmod[k], rmod[k]);
                                 float x0, x1, x2, x3;
                                 tc::upk2(tc::fma2(tc::pk2(sv[4 * q], sv[4 * q + 1]), c2p,
