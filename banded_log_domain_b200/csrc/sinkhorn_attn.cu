@@ -304,39 +304,47 @@ __global__ void k_sum_parts(const double* part, int n, float* out) {
     if (threadIdx.x == 0) out[0] = (float)red[0];
 }
 
-// The dS sweep's modifier as K16 operands of the dO V^T contraction:
-// out[bh][t][16] bf16, slots 3k, 3k+1, 3k+2 of term k < n holding the bf16
-// halves (hi, hi, lo) of v_k[bh][t] for the row side and (hi, lo, hi) for the
-// column side (v_k with a null pointer: 1), the other slots 0.
+// The dS sweep's modifier as K16 operands of the dO V^T contraction, for both
+// sweeps at once: out[i][bh][t][16] bf16, i = row side of q, column side of k,
+// row side of k, column side of q.  Slots 3k, 3k+1, 3k+2 of term k < n hold the
+// bf16 halves (hi, hi, lo) of the term's vector for a row side and (hi, lo, hi)
+// for a column side (a null vector: 1); the other slots are 0.
 struct AugTerms {
-    Vec v[4];
+    Vec q[4], k[4];  // the terms' query-side and key-side vectors
     int n;
-    int row;
+    __nv_bfloat16* out[4];
 };
-__global__ void k_aug(AugTerms tm, int L, int BH, __nv_bfloat16* out) {
-    const long long g = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-    if (g >= (long long)BH * L) return;
-    const int bh = (int)(g / L), t = (int)(g % L);
+__device__ __forceinline__ void put_aug_row(const Vec (&v)[4], int n, bool row, int bh, int t,
+                                            __nv_bfloat16* dst) {
     uint16_t sl[16];
 #pragma unroll
     for (int i = 0; i < 16; ++i) sl[i] = 0;
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
-        if (k >= tm.n) break;
-        const float v = tm.v[k].p ? tm.v[k].at(bh, t) : 1.f;
-        const __nv_bfloat16 hi = __float2bfloat16_rn(v);
-        const __nv_bfloat16 lo = __float2bfloat16_rn(v - __bfloat162float(hi));
+        if (k >= n) break;
+        const float x = v[k].p ? v[k].at(bh, t) : 1.f;
+        const __nv_bfloat16 hi = __float2bfloat16_rn(x);
+        const __nv_bfloat16 lo = __float2bfloat16_rn(x - __bfloat162float(hi));
         const uint16_t h = __bfloat16_as_ushort(hi), l = __bfloat16_as_ushort(lo);
         sl[3 * k] = h;
-        sl[3 * k + 1] = tm.row ? h : l;
-        sl[3 * k + 2] = tm.row ? l : h;
+        sl[3 * k + 1] = row ? h : l;
+        sl[3 * k + 2] = row ? l : h;
     }
     uint32_t w[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) w[i] = (uint32_t)sl[2 * i] | ((uint32_t)sl[2 * i + 1] << 16);
-    uint4* o = reinterpret_cast<uint4*>(out + (size_t)g * 16);
+    uint4* o = reinterpret_cast<uint4*>(dst);
     o[0] = make_uint4(w[0], w[1], w[2], w[3]);
     o[1] = make_uint4(w[4], w[5], w[6], w[7]);
+}
+__global__ void k_aug(AugTerms tm, int L, int BH) {
+    const long long g = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (g >= (long long)BH * L) return;
+    const int bh = (int)(g / L), t = (int)(g % L);
+    put_aug_row(tm.q, tm.n, true, bh, t, tm.out[0] + (size_t)g * 16);
+    put_aug_row(tm.k, tm.n, false, bh, t, tm.out[1] + (size_t)g * 16);
+    put_aug_row(tm.k, tm.n, true, bh, t, tm.out[2] + (size_t)g * 16);
+    put_aug_row(tm.q, tm.n, false, bh, t, tm.out[3] + (size_t)g * 16);
 }
 
 // out[0] += sum_i (x_i - y_i)^2, out[1] += sum_i y_i^2 in double: grid-stride
@@ -910,16 +918,14 @@ sa_status bwd_impl(const Ctx& x, const T* q, const T* k, const T* v, const uint8
         first <= 4) {
         const size_t one = align_up((size_t)d.BH * d.L * 16 * 2);
         const long long n = (long long)d.BH * d.L;
-        for (int i = 0; i < 4; ++i) {
-            augs[i] = (__nv_bfloat16*)(ws + l.aug + i * one);
-            AugTerms tm;
-            for (int k = 0; k < 4; ++k) tm.v[k] = Vec{nullptr, 0};
-            const bool from_q = (i == 0 || i == 3);
-            for (int k = 0; k < first; ++k) tm.v[k] = from_q ? rq[k] : rk[k];
-            tm.n = first;
-            tm.row = (i == 0 || i == 2);
-            SA_AUX(x.tr, k_aug<<<(unsigned)((n + 255) / 256), 256, 0, x.st>>>(tm, d.L, d.BH, augs[i]));
+        AugTerms tm;
+        for (int k = 0; k < 4; ++k) {
+            tm.q[k] = k < first ? rq[k] : Vec{nullptr, 0};
+            tm.k[k] = k < first ? rk[k] : Vec{nullptr, 0};
         }
+        tm.n = first;
+        for (int i = 0; i < 4; ++i) tm.out[i] = augs[i] = (__nv_bfloat16*)(ws + l.aug + i * one);
+        SA_AUX(x.tr, k_aug<<<(unsigned)((n + 255) / 256), 256, 0, x.st>>>(tm, d.L, d.BH));
     }
     for (int side = 0; side < 2; ++side) {
         for (int tb = 0; tb < nblk_t; ++tb) {
