@@ -218,7 +218,10 @@ sa_status sinkhorn_attn_bwd_sharded(const sa_params* p, const sa_shard* shard, c
  * (cudaHostAlloc / cudaHostRegister) for the copies to overlap; pageable
  * memory works, serialised by the driver.  The call returns once everything is
  * enqueued; the results are in host memory when `stream` reaches that point
- * (synchronise it before reading them).
+ * (synchronise it before reading them).  The two copy streams are created
+ * (non-blocking) on a device's first call and kept for the life of the
+ * process; calls on one device share them, so overlapping calls serialise
+ * their copies.
  */
 typedef struct {
     const void *q, *k, *v, *dO;  /* host [B][H][L][d] dtype */
