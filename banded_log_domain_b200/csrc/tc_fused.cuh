@@ -161,11 +161,11 @@ __device__ __forceinline__ float v_from_partials(const FusedArgs& a, int bh, int
 
 // E = exp2(c2 * s + cv + rd2) for one thread's 32 columns, packed to fp16
 // pairs in `ep`; `CHECK` masks the entries off the band (only the groups that
-// straddle the band's edge).  The fp32 values are added to four row-sum
-// accumulators (columns 4q + k into acc[k]).
+// straddle the band's edge).  The fp32 values are added to two packed pairs of
+// row-sum accumulators (columns 4q, 4q + 1 into acc[0]; 4q + 2, 4q + 3 into acc[1]).
 template <bool CHECK>
 __device__ __forceinline__ void group_exp(const uint32_t (&u)[32], const float* cvp, float c2, float rd2,
-                                          int d_first, int W, uint32_t (&ep)[16], float (&acc)[4]) {
+                                          int d_first, int W, uint32_t (&ep)[16], uint64_t (&acc)[2]) {
     const float4* c4 = reinterpret_cast<const float4*>(cvp);
     const uint64_t c2p = tc::pk2(c2, c2), rdp = tc::pk2(rd2, rd2);
 #pragma unroll
@@ -184,10 +184,8 @@ __device__ __forceinline__ void group_exp(const uint32_t (&u)[32], const float* 
             if ((unsigned)(d0 - 3 + W) > (unsigned)(2 * W)) x3 = -INFINITY;
         }
         const float e0 = ex2(x0), e1 = ex2(x1), e2 = ex2(x2), e3 = ex2(x3);
-        acc[0] += e0;
-        acc[1] += e1;
-        acc[2] += e2;
-        acc[3] += e3;
+        acc[0] = tc::add2(acc[0], tc::pk2(e0, e1));
+        acc[1] = tc::add2(acc[1], tc::pk2(e2, e3));
         ep[2 * q] = pack_f16(e0, e1);
         ep[2 * q + 1] = pack_f16(e2, e3);
     }
@@ -462,7 +460,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fused_iter(const FusedArgs a,
             // invalid rows carry -inf: all their E are 0
             const float rd2 = rowring[(it & 1) * 128 + lr];
             const bool rok = rd2 != -INFINITY;
-            float acc4[4] = {0.f, 0.f, 0.f, 0.f};  // partial row sums
+            uint64_t acc4[2] = {0, 0};  // partial row sums, packed pairs
             for (int c = 0; c < nch; ++c) {
                 const int g = it * nch + c, b = g & 1;
                 if (b != grp) continue;  // the other group's chunk
@@ -516,7 +514,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fused_iter(const FusedArgs a,
             // on to the next tile; part 0 forms u, 1/r and the quadrant's scale.
             tc::fence_async_smem();  // this warp's E stores, for the column MMAs
             float* rq = red + (it & 1) * 512 + qd * 128;
-            const float rpart = (acc4[0] + acc4[1]) + (acc4[2] + acc4[3]);
+            float a0, a1, a2, a3;
+            tc::upk2(acc4[0], a0, a1);
+            tc::upk2(acc4[1], a2, a3);
+            const float rpart = (a0 + a1) + (a2 + a3);
             if (pt != 0) {
                 // part 0 has read this buffer's previous contents (and arrived on
                 // WFULL for the previous tile) once it released tile it - 1
