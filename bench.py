@@ -16,12 +16,16 @@ maximum over ranks.
 Extra keys: ``roofline`` for the dominant kernel (per-launch CUDA events
 recorded by the library around each launch, see sa_params.trace_*),
 ``cpu_baseline`` (the CPU oracle on a bounded sample, rank 0 at N=1), ``e2e``
-(the same step with pinned-host inputs copied in and the results copied out
-inside the timed region), ``gpu_launches`` and ``clocks`` (nvidia-smi sampled
-during the timed region).
+(the same step through the library's host-buffer call
+``sinkhorn_attn_step_host``: pinned-host inputs copied in and the results copied
+out inside the timed region, pipelined by the library over ``--e2e-groups``
+groups of problems), ``gpu_launches`` and ``clocks`` (nvidia-smi sampled every
+50 ms during the timed region).
 
 ``--impl reference`` times the CPU oracle (the only reference implementation
 of this method) on a bounded sample of the same workload.
+``--bias-certificate`` prints the bias certificate of the workload's solve
+instead of timing steps.
 """
 from __future__ import annotations
 
