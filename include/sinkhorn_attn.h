@@ -112,9 +112,10 @@ sa_status sinkhorn_attn_state_size(const sa_params* p, size_t* n_floats);
 /* Workspace bytes needed by sinkhorn_attn_fwd and sinkhorn_attn_bwd (either
  * pointer may be NULL).  Both are O(B*H*L) and include a 256-byte status
  * header at offset 0.  The backward's grows with R (a few float32 vectors of
- * B*H*(L+dustbin) per tail step); for R > 4 it also holds a float32
- * [B][H][L][d] sum of the dQ / dK sweeps over blocks of at most 8 modifier
- * terms. */
+ * B*H*(L+dustbin) per tail step); it holds four bf16 [B][H][L][16] arrays
+ * (the modifier's operands of the bf16 dS contraction, 128 bytes per token),
+ * and for R > 4 a float32 [B][H][L][d] sum of the dQ / dK sweeps over blocks of
+ * at most 8 modifier terms. */
 sa_status sinkhorn_attn_workspace_size(const sa_params* p, size_t* fwd_bytes, size_t* bwd_bytes);
 
 /*
