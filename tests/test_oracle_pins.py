@@ -238,6 +238,9 @@ CASES = [
     (21, 4, 3, 0.8, 2, 4, None, False),       # R = 4
     (18, 4, 3, 0.7, 3, 2, None, True),        # dustbin
     (26, 8, 4, 0.6, 4, 2, "holes", True),     # dustbin + holes
+    (22, 4, 3, 0.8, 2, 6, "holes", False),    # R = 6: more terms than one dS sweep takes
+    (20, 4, 4, 0.9, 1, 9, None, True),        # R = 9 with the dustbin
+    (16, 4, 2, 1.0, 0, 9, "holes", False),    # T = 0, R = 9: full backpropagation
 ]
 
 
