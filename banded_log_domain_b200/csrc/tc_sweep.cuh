@@ -453,6 +453,60 @@ __global__ void __launch_bounds__(nthreads(MODE), ctas_per_sm(MODE)) tc_band_swe
             }
         };
         if (ntl >= 1) load_rows(tile(cur0));
+        // dS modes: a tile's dQ / dK rows are read out of TMEM after the next
+        // tile's first chunk (or after the last tile), by when the tile's last
+        // dS X MMA has long completed; O is double-buffered, and the MMA needs
+        // buffer it & 1 again only for tile it + 2
+        bool pend = false;
+        int p_it = 0, p_bh = 0, p_r = 0;
+        bool p_rok = false;
+        auto ds_finish = [&](int fit, int fbh, int fr, bool frok) -> bool {
+            constexpr int OW = 64 / NPART;
+            const int ob = fit & 1;
+            if (!ctl.wait(B_OFULL + ob, (fit >> 1) & 1)) return false;
+            float o[OW];
+            {
+                tc::tc_fence_after();
+                uint32_t u0[OW];
+                if constexpr (OW == 32) tc::tmem_ld32(tO + 64 * ob + lanebase + OW * pt, u0);
+                else tc::tmem_ld16(tO + 64 * ob + lanebase + OW * pt, u0);
+                tc::tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < OW; ++j) o[j] = __uint_as_float(u0[j]);
+                tc::tc_fence_before();
+                __syncwarp();
+                if (lane == 0) tc::mbar_arrive(bar + B_OEMPTY + ob);
+            }
+#pragma unroll
+            for (int j = 0; j < OW; ++j) o[j] = frok ? o[j] * a.out_scale : 0.f;
+            float* accr = (a.acc && fr < L) ? a.acc + ((size_t)fbh * L + fr) * 64 + OW * pt : nullptr;
+            if (accr && a.acc_in) {
+#pragma unroll
+                for (int q = 0; q < OW / 4; ++q) {
+                    const float4 p = reinterpret_cast<const float4*>(accr)[q];
+                    o[4 * q] += p.x; o[4 * q + 1] += p.y; o[4 * q + 2] += p.z; o[4 * q + 3] += p.w;
+                }
+            }
+            if (accr && a.acc_out) {
+#pragma unroll
+                for (int q = 0; q < OW / 4; ++q)
+                    reinterpret_cast<float4*>(accr)[q] =
+                        make_float4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
+            } else if (fr < L) {
+                __nv_bfloat16* outp =
+                    reinterpret_cast<__nv_bfloat16*>(a.out_mat) + ((size_t)fbh * L + fr) * 64 + OW * pt;
+#pragma unroll
+                for (int q = 0; q < OW / 8; ++q) {
+                    uint4 w;
+                    w.x = tc::pack_bf16(o[8 * q + 0], o[8 * q + 1]);
+                    w.y = tc::pack_bf16(o[8 * q + 2], o[8 * q + 3]);
+                    w.z = tc::pack_bf16(o[8 * q + 4], o[8 * q + 5]);
+                    w.w = tc::pack_bf16(o[8 * q + 6], o[8 * q + 7]);
+                    reinterpret_cast<uint4*>(outp)[q] = w;
+                }
+            }
+            return true;
+        };
         Cursor cur = cur0;
         for (int it = 0; ok && it < ntl; ++it, cur.next(nblk, a.H)) {
             const Tile tl = tile(cur);
@@ -667,6 +721,10 @@ __global__ void __launch_bounds__(nthreads(MODE), ctas_per_sm(MODE)) tc_band_swe
                 }
                 __syncwarp();
                 if (lane == 0) tc::mbar_arrive(bar + B_EMPTY + s);
+                if (DS && c == 0 && pend) {  // the previous tile's rows
+                    if (!ds_finish(p_it, p_bh, p_r, p_rok)) { ok = false; break; }
+                    pend = false;
+                }
             }
 
             if (!ok) break;
@@ -717,6 +775,12 @@ __global__ void __launch_bounds__(nthreads(MODE), ctas_per_sm(MODE)) tc_band_swe
                     }
                     a.out_vec.at(bh, r) = rokf ? out : 0.f;
                 }
+            } else if (DS) {
+                pend = true;
+                p_it = it;
+                p_bh = bh;
+                p_r = r;
+                p_rok = rokf;
             } else {
                 // O accumulator of this tile: this warp reads columns OW*pt..OW*pt+OW-1
                 // of its lanes, then frees the buffer for tile it + 2
@@ -796,6 +860,7 @@ __global__ void __launch_bounds__(nthreads(MODE), ctas_per_sm(MODE)) tc_band_swe
                 }
             }
         }
+        if (DS && ok && pend) ds_finish(p_it, p_bh, p_r, p_rok);  // the last tile's rows
     }
 
     tc::tc_fence_before();

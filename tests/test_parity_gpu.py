@@ -48,6 +48,11 @@ SMALL = [
     (520, 64, 0.6, 0, 5, "bf16", "holes", False),
     (300, 100, 1.0, 2, 9, "bf16", (180, 300), False),
     (384, 64, 1.0, 0, 20, "bf16", None, False),
+    # more tiles than the 148 persistent CTAs (2 x 2 problems x 64 row blocks):
+    # CTAs walk several tiles, and the dS sweeps read a tile's rows out of TMEM
+    # after the next tile's first chunk
+    (8192, 64, 0.9, 3, 2, "bf16", (6000, 8192), False),
+    (8192, 100, 1.0, 2, 1, "bf16", "holes", False),
 ]
 
 
