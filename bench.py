@@ -247,7 +247,7 @@ def oracle_cores():
         return os.cpu_count() or 1
 
 
-def cpu_baseline(w, schedule, target_s=12.0):
+def cpu_baseline(w, schedule, target_s=20.0):
     heads, L_s = size_sample(w, schedule, target_s)
     rate, dt = oracle_sample_rate(w, L_s, schedule, heads)
     return {"value": rate, "unit": UNIT, "cores": oracle_cores(), "kind": "oracle",
