@@ -418,3 +418,49 @@ def test_work_is_linear_in_support(oracle_mod, L, W, T, db):
     _, bvis = oracle_mod.backward(q, k, v, st, dO, W=W, eps=1.0, R=R, dustbin=db,
                                   schedule="direct", count=True)
     assert bvis[0, 0] == 8 * aug
+
+
+# --------------------------------------------------------------------------
+# random small configurations (property-based): every parameter at once
+# --------------------------------------------------------------------------
+
+from hypothesis import HealthCheck, given, settings, strategies as st_
+
+
+@settings(max_examples=60, deadline=None, derandomize=True,
+          suppress_health_check=[HealthCheck.too_slow])
+@given(L=st_.integers(1, 20), d=st_.sampled_from([1, 2, 3, 4, 8]), W=st_.integers(0, 22),
+       eps=st_.floats(0.4, 1.5), T=st_.integers(0, 4), R=st_.integers(1, 5),
+       dustbin=st_.booleans(), seed=st_.integers(0, 2 ** 31 - 1))
+def test_random_configurations_match_dense_autograd(oracle_mod, L, d, W, eps, T, R, dustbin, seed):
+    """Any band (W = 0 up to dense), length (down to one token), head size,
+    depth, random mask (down to a single valid token, or none) and dustbin: the
+    forward, the duals and both backward schedules equal exact autodiff of the
+    dense surrogate, and masked tokens carry exact zeros."""
+    rng = np.random.default_rng(seed)
+    q, k, v, dO = (rng.normal(size=(1, 1, L, d)) for _ in range(4))
+    mask = (rng.random((1, L)) < rng.uniform(0.3, 1.0)).astype(np.uint8)
+    vd = rng.normal(size=(1, d)) if dustbin else None
+    kw = dict(W=W, eps=eps, R=R, dustbin=dustbin, dustbin_score=float(rng.uniform(-3, 1)))
+    o, st = oracle_mod.forward(q, k, v, T=T, mask=mask, v_dust=vd, **kw)
+    grads = {s: oracle_mod.backward(q, k, v, st, dO, mask=mask, v_dust=vd, schedule=s, **kw)
+             for s in ("direct", "one_reference")}
+    m = mask[0].astype(bool)
+    if not m.any():  # nothing valid: every output and dual is zero
+        assert not o.any() and not st[..., :L].any()
+        for dq, dk, dv, _ in grads.values():
+            assert not dq.any() and not dk.any() and not dv.any()
+        return
+    ro, rst, rdq, rdk, rdv, rdvd = ds.surrogate_and_grads(
+        q[0, 0], k[0, 0], v[0, 0], dO[0, 0], mask=mask[0], T=T,
+        v_dust=None if vd is None else vd[0], **kw)
+    np.testing.assert_allclose(o[0, 0], ro, atol=1e-11)
+    np.testing.assert_allclose(st[0, 0], rst, atol=1e-10)
+    for s, (dq, dk, dv, dvd) in grads.items():
+        scale = max(np.abs(rdq).max(), np.abs(rdk).max(), 1.0)
+        np.testing.assert_allclose(dq[0, 0], rdq, atol=1e-9 * scale, err_msg=s)
+        np.testing.assert_allclose(dk[0, 0], rdk, atol=1e-9 * scale, err_msg=s)
+        np.testing.assert_allclose(dv[0, 0], rdv, atol=1e-10, err_msg=s)
+        assert not dq[0, 0, ~m].any() and not dk[0, 0, ~m].any() and not dv[0, 0, ~m].any()
+        if dustbin:
+            np.testing.assert_allclose(dvd[0], rdvd, atol=1e-10, err_msg=s)
