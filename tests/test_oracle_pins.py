@@ -77,6 +77,25 @@ def test_golden_2x2_hand_derived(oracle_mod):
     assert abs(band[0, 0, 0, 1] - _ev(g["limit_p00"])) < 1e-14
 
 
+def test_golden_dustbin_one_token_hand_derived(oracle_mod):
+    """One real token and the dustbin: the augmented 2 x 2 problem solved in exact
+    rationals, including the value cotangents of the token and of the dustbin."""
+    g = json.load(open(os.path.join(GOLDEN, "dustbin_1token.json")))
+    arr = lambda key: np.array([[[[_ev(x) for x in r] for r in g[key]]]])
+    q, k, v, dO = arr("q"), arr("k"), arr("v"), arr("dO")
+    vd = np.array([[_ev(x) for x in g["v_dust"]]])
+    kw = dict(W=g["W"], eps=_ev(g["eps"]), R=g["R"], dustbin=True, dustbin_score=g["dustbin_score"])
+    o, st = oracle_mod.forward(q, k, v, T=g["T"], v_dust=vd, **kw)
+    for r, nm in enumerate(["u0", "v0", "u1", "v1", "u2", "v2"]):
+        np.testing.assert_allclose(st[0, 0, r], [_ev(x) for x in g[nm]], rtol=0, atol=1e-14,
+                                   err_msg=nm)
+    np.testing.assert_allclose(o[0, 0], [[_ev(x) for x in r] for r in g["O"]], atol=1e-14)
+    for s in ("direct", "one_reference"):
+        _, _, dv, dvd = oracle_mod.backward(q, k, v, st, dO, v_dust=vd, schedule=s, **kw)
+        np.testing.assert_allclose(dv[0, 0], [[_ev(x) for x in r] for r in g["dV"]], atol=1e-14)
+        np.testing.assert_allclose(dvd[0], [_ev(x) for x in g["dv_dust"]], atol=1e-14)
+
+
 def test_T0_rows_are_softmax(oracle_mod):
     """T = 0: the base is zero, so P^(1,0) is the row softmax of the masked band
     scores (a library routine), u0 = v0 = 0."""
