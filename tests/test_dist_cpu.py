@@ -10,6 +10,7 @@ import socket
 import time
 
 import pytest
+from hypothesis import given, settings, strategies as st
 
 import bench
 
@@ -165,3 +166,24 @@ def test_shard_bounds():
     assert sa.shard_bounds(10, 2, 2, 3) == (7, 10, 5, 10)
     with pytest.raises(ValueError):
         sa.shard_bounds(10, 4, 0, 3)  # 3 own tokens < W
+
+
+@settings(max_examples=200, deadline=None, derandomize=True)
+@given(L=st.integers(1, 5000), W=st.integers(0, 64), world=st.integers(1, 8))
+def test_shard_bounds_partition_the_sequence(L, W, world):
+    """Own ranges tile [0, L) in rank order with sizes differing by at most one;
+    each local range is the own range widened by W on each side (clipped to the
+    sequence), so a boundary's two halos both hold W tokens."""
+    import banded_log_domain_b200 as sa
+
+    if world > 1 and L // world < max(W, 1):
+        with pytest.raises(ValueError):
+            sa.shard_bounds(L, W, 0, world)
+        return
+    b = [sa.shard_bounds(L, W, r, world) for r in range(world)]
+    assert b[0][0] == 0 and b[-1][1] == L
+    assert all(x[1] == y[0] for x, y in zip(b, b[1:]))
+    sizes = [hi - lo for lo, hi, _, _ in b]
+    assert max(sizes) - min(sizes) <= 1 and min(sizes) >= (max(W, 1) if world > 1 else 0)
+    for own_lo, own_hi, lo, hi in b:
+        assert (lo, hi) == (max(0, own_lo - W), min(L, own_hi + W))
