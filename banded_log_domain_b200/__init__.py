@@ -11,7 +11,6 @@ missing or unloadable library raises on first use.
 from __future__ import annotations
 
 import ctypes
-import math
 import os
 
 import torch
@@ -45,7 +44,7 @@ class sa_params(ctypes.Structure):
     ]
 
 
-KERNEL_KINDS = {1: "lse_sweep", 2: "pv", 3: "wsum", 4: "ds", 5: "aux", 6: "fused_sweep"}
+KERNEL_KINDS = {1: "lse_sweep", 2: "pv", 3: "wsum", 4: "ds", 5: "aux"}
 
 class sa_host_step(ctypes.Structure):
     _fields_ = [("q", ctypes.c_void_p), ("k", ctypes.c_void_p), ("v", ctypes.c_void_p),
@@ -118,6 +117,10 @@ def _L():
     lib.sinkhorn_attn_debug_plan.argtypes = [P, ctypes.c_int, ctypes.c_int, vp, vp, vp, vp, vp,
                                              vp, vp, vp]
     lib.sinkhorn_attn_poll.argtypes = [vp, vp]
+    lib.sinkhorn_attn_poll_static.argtypes = [vp]
+    lib.sinkhorn_attn_bias_certificate.argtypes = [
+        ctypes.c_int, ctypes.POINTER(ctypes.c_int), ctypes.c_int, ctypes.POINTER(ctypes.c_double),
+        ctypes.c_double, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int)]
     lib.sinkhorn_attn_debug_timeout.argtypes = [vp, ctypes.c_longlong, vp]
     lib.sinkhorn_attn_sq_dist.argtypes = [vp, vp, ctypes.c_longlong, ctypes.c_int, vp, vp]
     lib.sinkhorn_attn_step_host_workspace_size.argtypes = [P, ctypes.c_int, ctypes.POINTER(sz)]
@@ -130,6 +133,7 @@ def _L():
     lib.sinkhorn_attn_strerror.restype = ctypes.c_char_p
     for f in ("sinkhorn_attn_state_size", "sinkhorn_attn_workspace_size", "sinkhorn_attn_fwd",
               "sinkhorn_attn_bwd", "sinkhorn_attn_debug_plan", "sinkhorn_attn_poll",
+              "sinkhorn_attn_poll_static", "sinkhorn_attn_bias_certificate",
               "sinkhorn_attn_debug_timeout", "sinkhorn_attn_sq_dist", "sinkhorn_attn_fwd_sharded",
               "sinkhorn_attn_bwd_sharded", "sinkhorn_attn_step_host_workspace_size",
               "sinkhorn_attn_step_host"):
@@ -145,7 +149,8 @@ def load():
 
 EXPORTS = ("sinkhorn_attn_state_size", "sinkhorn_attn_workspace_size", "sinkhorn_attn_fwd",
            "sinkhorn_attn_bwd", "sinkhorn_attn_bwd_static_ws", "sinkhorn_attn_debug_plan",
-           "sinkhorn_attn_poll", "sinkhorn_attn_strerror", "sinkhorn_attn_debug_timeout",
+           "sinkhorn_attn_poll", "sinkhorn_attn_poll_static", "sinkhorn_attn_strerror",
+           "sinkhorn_attn_debug_timeout", "sinkhorn_attn_bias_certificate",
            "sinkhorn_attn_sq_dist", "sinkhorn_attn_fwd_sharded", "sinkhorn_attn_bwd_sharded",
            "sinkhorn_attn_step_host_workspace_size", "sinkhorn_attn_step_host")
 
@@ -173,6 +178,13 @@ def _ptr(t):
 
 def _stream(device):
     return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _on(device, fn, *args):
+    """Calls the C entry point ``fn`` with ``device`` current (the library
+    validates every pointer against the current device and launches there)."""
+    with torch.cuda.device(device):
+        return fn(*args)
 
 
 def sinkhorn_attn_state_size(p: sa_params) -> int:
@@ -217,7 +229,7 @@ def sinkhorn_attn_fwd(q, k, v, *, W, eps, T, R=2, mask=None, dustbin=False, dust
         state = torch.empty(sinkhorn_attn_state_size(p), dtype=torch.float32, device=dev)
     if ws is None:
         ws = torch.zeros(sinkhorn_attn_workspace_size(p)[0], dtype=torch.uint8, device=dev)
-    rc = _L().sinkhorn_attn_fwd(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(mask),
+    rc = _on(dev, _L().sinkhorn_attn_fwd, ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(mask),
                                 _ptr(v_dust), _ptr(o), _ptr(state), _ptr(ws), ws.numel(),
                                 _stream(dev))
     _check(rc, "sinkhorn_attn_fwd")
@@ -245,7 +257,7 @@ def sinkhorn_attn_bwd(q, k, v, o, dO, state, *, W, eps, R=2, mask=None, dustbin=
         dv_dust = torch.empty(q.shape[1], q.shape[3], dtype=torch.float32, device=dev)
     if ws is None:
         ws = torch.zeros(sinkhorn_attn_workspace_size(p)[1], dtype=torch.uint8, device=dev)
-    rc = _L().sinkhorn_attn_bwd(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(mask),
+    rc = _on(dev, _L().sinkhorn_attn_bwd, ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(mask),
                                 _ptr(v_dust), _ptr(o), _ptr(dO), _ptr(state), _ptr(dq), _ptr(dk),
                                 _ptr(dv), _ptr(dv_dust if dustbin else None),
                                 _ptr(d_dust_score if dustbin else None), _ptr(ws), ws.numel(),
@@ -278,7 +290,7 @@ def sinkhorn_attn_bwd_static_ws(q, k, v, o, dO, state, *, W, eps, R=2, mask=None
     dv = torch.empty_like(q) if dv is None else dv
     if dustbin and dv_dust is None:
         dv_dust = torch.empty(q.shape[1], q.shape[3], dtype=torch.float32, device=dev)
-    rc = _L().sinkhorn_attn_bwd_static_ws(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(mask),
+    rc = _on(dev, _L().sinkhorn_attn_bwd_static_ws, ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(mask),
                                           _ptr(v_dust), _ptr(o), _ptr(dO), _ptr(state), _ptr(dq),
                                           _ptr(dk), _ptr(dv), _ptr(dv_dust if dustbin else None),
                                           _ptr(d_dust_score if dustbin else None), _stream(dev))
@@ -326,7 +338,7 @@ def sinkhorn_attn_step_host(q, k, v, dO, *, W, eps, T, R=2, mask=None, dustbin=F
                       _ptr(v_dust if dustbin else None), _ptr(o), _ptr(dq), _ptr(dk), _ptr(dv),
                       _ptr(state), _ptr(dv_dust if dustbin else None),
                       _ptr(d_dust_score if dustbin else None), int(groups))
-    rc = _L().sinkhorn_attn_step_host(ctypes.byref(p), ctypes.byref(io), _ptr(ws), ws.numel(),
+    rc = _on(dev, _L().sinkhorn_attn_step_host, ctypes.byref(p), ctypes.byref(io), _ptr(ws), ws.numel(),
                                       _stream(dev))
     _check(rc, "sinkhorn_attn_step_host")
     return o, dq, dk, dv
@@ -393,7 +405,7 @@ def sinkhorn_attn_fwd_sharded(q, k, v, *, W, eps, T, R=2, mask=None, halo_lo, ha
     if ws is None:
         ws = torch.zeros(sinkhorn_attn_workspace_size(p)[0], dtype=torch.uint8, device=dev)
     sh, errors, _keep = _shard_for(halo_lo, halo_hi, exchange, L, dev)
-    rc = _L().sinkhorn_attn_fwd_sharded(ctypes.byref(p), ctypes.byref(sh), _ptr(q), _ptr(k),
+    rc = _on(dev, _L().sinkhorn_attn_fwd_sharded, ctypes.byref(p), ctypes.byref(sh), _ptr(q), _ptr(k),
                                         _ptr(v), _ptr(mask), _ptr(o), _ptr(state), _ptr(ws),
                                         ws.numel(), _stream(dev))
     _check_sharded(rc, "sinkhorn_attn_fwd_sharded", errors)
@@ -418,7 +430,7 @@ def sinkhorn_attn_bwd_sharded(q, k, v, o, dO, state, *, W, eps, R=2, mask=None, 
     if ws is None:
         ws = torch.zeros(sinkhorn_attn_workspace_size(p)[1], dtype=torch.uint8, device=dev)
     sh, errors, _keep = _shard_for(halo_lo, halo_hi, exchange, L, dev)
-    rc = _L().sinkhorn_attn_bwd_sharded(ctypes.byref(p), ctypes.byref(sh), _ptr(q), _ptr(k),
+    rc = _on(dev, _L().sinkhorn_attn_bwd_sharded, ctypes.byref(p), ctypes.byref(sh), _ptr(q), _ptr(k),
                                         _ptr(v), _ptr(mask), _ptr(o), _ptr(dO), _ptr(state),
                                         _ptr(dq), _ptr(dk), _ptr(dv), _ptr(ws), ws.numel(),
                                         _stream(dev))
@@ -496,7 +508,7 @@ def sinkhorn_attn_debug_plan(q, k, state, a, b, *, W, eps, R=2, mask=None, dustb
     band = torch.empty(B, H, L, 2 * W + 1, dtype=torch.float32, device=dev)
     dcol = torch.empty(B, H, L, dtype=torch.float32, device=dev) if dustbin else None
     drow = torch.empty(B, H, L + 1, dtype=torch.float32, device=dev) if dustbin else None
-    rc = _L().sinkhorn_attn_debug_plan(ctypes.byref(p), int(a), int(b), _ptr(q), _ptr(k),
+    rc = _on(dev, _L().sinkhorn_attn_debug_plan, ctypes.byref(p), int(a), int(b), _ptr(q), _ptr(k),
                                        _ptr(mask), _ptr(state), _ptr(band), _ptr(dcol),
                                        _ptr(drow), _stream(dev))
     _check(rc, "sinkhorn_attn_debug_plan")
@@ -505,18 +517,33 @@ def sinkhorn_attn_debug_plan(q, k, state, a, b, *, W, eps, R=2, mask=None, dustb
 
 def sinkhorn_attn_poll(ws) -> int:
     """Status word recorded in ``ws`` (after synchronising the current stream)."""
-    return int(_L().sinkhorn_attn_poll(_ptr(ws), _stream(ws.device)))
+    return int(_on(ws.device, _L().sinkhorn_attn_poll, _ptr(ws), _stream(ws.device)))
+
+
+def sinkhorn_attn_poll_static(device=None) -> int:
+    """Status word of the fixed scratch array of :func:`sinkhorn_attn_bwd_static_ws`
+    on ``device`` (default: the current one), read and reset after synchronising
+    that device's current stream."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    return int(_on(dev, _L().sinkhorn_attn_poll_static, _stream(dev)))
 
 
 def sinkhorn_attn_strerror(status: int) -> str:
     return strerror(status)
 
 
-def sinkhorn_attn_debug_timeout(ws, budget_cycles: int = 1_000_000) -> int:
+def sinkhorn_attn_debug_timeout(ws, budget_cycles: int = 1_000_000, device=None) -> int:
     """Runs the library's bounded wait on a barrier nothing completes (test hook
     for the failure path); the timeout lands in the status word of ``ws`` (a
-    CUDA tensor of at least 256 bytes) and is read by :func:`sinkhorn_attn_poll`."""
-    return int(_L().sinkhorn_attn_debug_timeout(_ptr(ws), int(budget_cycles), _stream(ws.device)))
+    CUDA tensor of at least 256 bytes) and is read by :func:`sinkhorn_attn_poll`.
+    With ``ws=None`` it lands in the static scratch's status word on ``device``
+    (read by :func:`sinkhorn_attn_poll_static`)."""
+    if ws is not None:
+        dev = ws.device
+    else:
+        dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    return int(_on(dev, _L().sinkhorn_attn_debug_timeout, _ptr(ws), int(budget_cycles),
+                   _stream(dev)))
 
 
 def sinkhorn_attn_sq_dist(x, y):
@@ -527,8 +554,8 @@ def sinkhorn_attn_sq_dist(x, y):
         raise ValueError("x and y must have one shape and dtype")
     dt = {torch.float32: SA_F32, torch.bfloat16: SA_BF16}[x.dtype]
     out = torch.empty(2, dtype=torch.float64, device=x.device)
-    _check(_L().sinkhorn_attn_sq_dist(_ptr(x), _ptr(y), x.numel(), dt, _ptr(out),
-                                      _stream(x.device)), "sinkhorn_attn_sq_dist")
+    _check(_on(x.device, _L().sinkhorn_attn_sq_dist, _ptr(x), _ptr(y), x.numel(), dt, _ptr(out),
+               _stream(x.device)), "sinkhorn_attn_sq_dist")
     s = out.cpu()
     return float(s[0]), float(s[1])
 
@@ -540,9 +567,10 @@ def bias_certificate(q, k, v, dO, *, N, Rs=(0, 1, 2, 4), tau=1e-5, W, eps, mask=
     ``Rs`` (0 <= R <= N) the gradients g_R of <dO, O> come from
     :func:`sinkhorn_attn_fwd` / :func:`sinkhorn_attn_bwd` with T = N - R stopped
     iterations; g_full, full backpropagation, from T = 0 and R = N.  Then
-    eta_R = ||g_R - g_full|| / ||g_full|| over (dQ, dK, dV), the norms from
-    :func:`sinkhorn_attn_sq_dist`.  Returns ``({R: eta_R}, R*)``, R* the smallest
-    R in ``Rs`` with eta_R <= tau (None if none is).  No dustbin."""
+    eta_R = ||g_R - g_full|| / ||g_full|| over (dQ, dK, dV), the squared norms from
+    :func:`sinkhorn_attn_sq_dist` and eta_R, R* from the C entry point
+    ``sinkhorn_attn_bias_certificate``.  Returns ``({R: eta_R}, R*)``, R* the
+    smallest R in ``Rs`` with eta_R <= tau (None if none is).  No dustbin."""
     if any(not 0 <= R <= N for R in Rs):
         raise ValueError("every R must lie in [0, N]")
 
@@ -553,18 +581,19 @@ def bias_certificate(q, k, v, dO, *, N, Rs=(0, 1, 2, 4), tau=1e-5, W, eps, mask=
         return g
 
     full = grads(0, N)
-    eta = {}
-    for R in sorted(set(Rs)):
+    depths = sorted(set(Rs))
+    sums = []
+    for R in depths:
         g = full if R == N else grads(N - R, R)
-        num = den = 0.0
         for a, b in zip(g, full):
-            d2, n2 = sinkhorn_attn_sq_dist(a, b)
-            num += d2
-            den += n2
-        eta[R] = math.sqrt(num / den) if den > 0 else math.sqrt(num)
-    ok = [R for R in sorted(eta) if eta[R] <= tau]
-    return eta, (ok[0] if ok else None)
-
-
-def score_scale(d: int, eps: float) -> float:
-    return 1.0 / (math.sqrt(d) * eps)
+            sums.extend(sinkhorn_attn_sq_dist(a, b))
+    n = len(depths)
+    c_depths = (ctypes.c_int * n)(*depths)
+    c_sums = (ctypes.c_double * len(sums))(*sums)
+    c_eta = (ctypes.c_double * n)()
+    c_rstar = ctypes.c_int(-1)
+    _check(_L().sinkhorn_attn_bias_certificate(n, c_depths, len(full), c_sums, float(tau), c_eta,
+                                               ctypes.byref(c_rstar)),
+           "sinkhorn_attn_bias_certificate")
+    eta = {R: float(c_eta[i]) for i, R in enumerate(depths)}
+    return eta, (None if c_rstar.value < 0 else int(c_rstar.value))

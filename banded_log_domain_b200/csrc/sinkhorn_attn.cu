@@ -31,7 +31,6 @@
 
 #include "../../include/sinkhorn_attn.h"
 #include "simt_sweep.cuh"
-#include "tc_fused.cuh"
 #include "tc_sweep.cuh"
 
 namespace sa {
@@ -76,67 +75,36 @@ sa_status check_params(const sa_params* p, Dims* dd) {
 
 bool aligned16(const void* x) { return ((uintptr_t)x & 15u) == 0; }
 
-// Rejects pointers the device cannot dereference (plain pageable host memory).
-bool device_ok(const void* x) {
-    if (!x || !aligned16(x)) return false;
+// Memory the current device's kernels may read and write at full speed: device
+// memory of the current device, or managed memory.  Pinned host memory (read
+// over PCIe), pageable host memory, and another device's memory (a tensor on
+// another GPU, or the wrong device current) are rejected before any launch.
+bool on_current_device(const void* x) {
     cudaPointerAttributes at;
     if (cudaPointerGetAttributes(&at, x) != cudaSuccess) {
         cudaGetLastError();
         return false;
     }
-    return at.type == cudaMemoryTypeDevice || at.type == cudaMemoryTypeManaged ||
-           at.type == cudaMemoryTypeHost;
+    if (at.type == cudaMemoryTypeManaged) return true;
+    if (at.type != cudaMemoryTypeDevice) return false;
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        return false;
+    }
+    return at.device == dev;
 }
+bool device_ok(const void* x) { return x && aligned16(x) && on_current_device(x); }
 // A device float that may sit anywhere a float may (4-byte alignment).
-bool device_f32_ok(const void* x) {
-    if (!x || ((uintptr_t)x & 3u)) return false;
-    cudaPointerAttributes at;
-    if (cudaPointerGetAttributes(&at, x) != cudaSuccess) {
-        cudaGetLastError();
-        return false;
-    }
-    return at.type == cudaMemoryTypeDevice || at.type == cudaMemoryTypeManaged ||
-           at.type == cudaMemoryTypeHost;
-}
-bool mask_ok(const void* x) {
-    if (!x) return true;
-    cudaPointerAttributes at;
-    if (cudaPointerGetAttributes(&at, x) != cudaSuccess) {
-        cudaGetLastError();
-        return false;
-    }
-    return at.type != cudaMemoryTypeUnregistered;
-}
+bool device_f32_ok(const void* x) { return x && ((uintptr_t)x & 3u) == 0 && on_current_device(x); }
+// The byte mask (any alignment; NULL means every token is valid).
+bool mask_ok(const void* x) { return !x || on_current_device(x); }
 
-// The fused forward (one pass per iteration) applies to bf16 storage without a
-// dustbin, W <= 256, and at least two iterations (the first is two sweeps).
-bool fused_fwd(const sa_params* p) {
-    return p->dtype == SA_BF16 && !p->dustbin && p->W <= 256 && p->T + p->R >= 2;
-}
-
-// Forward workspace: status header; for the fused forward two ping-pong column
-// dual vectors and two buffers of per-row-block column partials.
+// Forward workspace: the status header only (the duals live in the state).
 struct FwdLayout {
-    size_t va, vb, p0, p1, total;
-    int nblk, ncol, nch;
+    size_t total;
 };
-FwdLayout fwd_layout(const Dims& d, const sa_params* p) {
-    FwdLayout l{};
-    l.total = kHeader;
-    if (!fused_fwd(p)) return l;
-    l.nblk = (d.L + 127) / 128;
-    l.ncol = 2 * p->W + 128;
-    l.nch = (l.ncol + 127) / 128;
-    const size_t vec = align_up((size_t)d.BH * d.ld * sizeof(float));
-    const size_t part = align_up((size_t)d.BH * d.L * tcf::NSLOT * sizeof(float));
-    size_t o = kHeader;
-    l.va = o; o += vec;
-    l.vb = o; o += vec;
-    l.p0 = o; o += part;
-    l.p1 = o; o += part;
-    l.total = o;
-    return l;
-}
+FwdLayout fwd_layout(const Dims&, const sa_params*) { return FwdLayout{kHeader}; }
 
 // Backward workspace layout (float32 vectors of BH * ld elements each).
 struct BwdLayout {
@@ -675,97 +643,6 @@ sa_status fwd_impl(const Ctx& x, const T* q, const T* k, const T* v, const uint8
     return SA_OK;
 }
 
-// Forward with fused iterations (bf16, see fused_fwd).  Where each iterate lives:
-//   u_m: the state's u0 row while m <= T (updated in place), u^(m-T) after;
-//   v_m: ping-pong workspace vectors while m < T, the state's v0 row at m = T,
-//        v^(m-T) after; v_0 = 0 is the (zeroed) state v0 row.
-sa_status fwd_fused(const Ctx& x, const __nv_bfloat16* q, const __nv_bfloat16* k,
-                    const __nv_bfloat16* v, const uint8_t* mask, __nv_bfloat16* o, float* state,
-                    char* ws) {
-    const Dims& d = x.d;
-    const int T = x.p->T, R = d.R, K = T + R;
-    const FwdLayout l = fwd_layout(d, x.p);
-    SA_CUDA(cudaMemsetAsync(state, 0, (size_t)d.BH * (2 * R + 2) * d.ld * sizeof(float), x.st));
-    float* VA = (float*)(ws + l.va);
-    float* VB = (float*)(ws + l.vb);
-    float* PART[2] = {(float*)(ws + l.p0), (float*)(ws + l.p1)};
-    auto u_home = [&](int m) { return Vec{state + (size_t)(m <= T ? 0 : 2 * (m - T)) * d.ld, x.sst}; };
-    auto v_home = [&](int m) {
-        if (m == 0) return Vec{state + (size_t)d.ld, x.sst};
-        if (m < T) return Vec{(m & 1) ? VA : VB, (long long)d.ld};
-        return Vec{state + (size_t)(2 * (m - T) + 1) * d.ld, x.sst};
-    };
-    auto mv = [](Vec a) { return MVec{const_cast<float*>(a.p), a.s}; };
-
-    // iteration 1: row sweep with a running max, then column sweep
-    simt::SweepArgs a = base_args(x);
-    a.mask = mask;
-    a.A = q; a.Bo = k;
-    a.cd = v_home(0);
-    a.rd = v_home(0);
-    a.online = 1;
-    a.out_vec = mv(u_home(1));
-    SA_CUDA((launch_sweep<__nv_bfloat16, simt::LSE>(a, d.BH, x.st, x.tr, x.status)));
-    a.A = k; a.Bo = q;
-    a.cd = u_home(1);
-    a.rd = v_home(0);
-    a.online = 0;
-    a.out_vec = mv(v_home(1));
-    SA_CUDA((launch_sweep<__nv_bfloat16, simt::LSE>(a, d.BH, x.st, x.tr, x.status)));
-
-    // iterations 2..K: one fused pass each
-    CUtensorMap mq, mk;
-    if (!make_map(&mq, q, d.L, d.BH) || !make_map(&mk, k, d.L, d.BH)) return SA_ERR_CUDA;
-    int dev = 0, nsm = 148;
-    if (cudaGetDevice(&dev) == cudaSuccess)
-        cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
-    const int ntiles = d.BH * l.nblk;
-    const dim3 grid(std::min(nsm, ntiles));
-    SA_CUDA(cudaFuncSetAttribute(tcf::tc_fused_iter, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 tcf::SMEM_BYTES));
-    tcf::FusedArgs f;
-    std::memset(&f, 0, sizeof(f));
-    f.L = d.L; f.W = x.p->W; f.H = d.H; f.BH = d.BH;
-    f.nblk = l.nblk; f.ncol = l.ncol; f.nch = l.nch;
-    f.c2 = x.c * kLog2e;
-    f.mask = mask;
-    f.status = x.status;
-    for (int it = 2; it <= K; ++it) {
-        f.u_prev = u_home(it - 1);
-        f.u_out = mv(u_home(it));
-        if (it == 2) {
-            f.v_src = v_home(1);
-            f.v_out = MVec{nullptr, 0};
-            f.part_in = nullptr;
-        } else {
-            f.v_src = v_home(it - 2);
-            f.v_out = mv(v_home(it - 1));
-            f.part_in = PART[(it - 1) & 1];
-        }
-        f.part_out = PART[it & 1];
-        x.tr.begin(SA_KERNEL_FUSED_SWEEP);
-        tcf::tc_fused_iter<<<grid, tcf::NTHREADS, tcf::SMEM_BYTES, x.st>>>(f, mq, mk);
-        x.tr.end();
-        SA_CUDA(cudaGetLastError());
-    }
-    // v_K from the last partials
-    f.v_src = v_home(K - 1);
-    f.part_in = PART[K & 1];
-    const long long n = (long long)d.BH * d.L;
-    SA_AUX(x.tr, tcf::k_finalize_v<<<(unsigned)((n + 255) / 256), 256, 0, x.st>>>(f, mv(v_home(K))));
-
-    // O = P^(R,R) V
-    simt::SweepArgs b = base_args(x);
-    b.mask = mask;
-    b.dust_cta = 0;
-    b.A = q; b.Bo = k; b.X = v;
-    b.rd = x.srow(2 * R);
-    b.cd = x.srow(2 * R + 1);
-    b.out_mat = o;
-    SA_CUDA((launch_sweep<__nv_bfloat16, simt::PV>(b, d.BH, x.st, x.tr, x.status)));
-    return SA_OK;
-}
-
 template <typename T>
 sa_status bwd_impl(const Ctx& x, const T* q, const T* k, const T* v, const uint8_t* mask,
                    const float* v_dust, const T* o, const T* dO, T* dq, T* dk, T* dv,
@@ -1056,9 +933,6 @@ sa_status fwd_call(const sa_params* p, const sa_shard* shard, const void* q, con
     if (p->dtype == SA_F32)
         s = fwd_impl<float>(x, (const float*)q, (const float*)k, (const float*)v, mask, vd,
                             (float*)o, state);
-    else if (fused_fwd(p) && !shard)
-        s = fwd_fused(x, (const __nv_bfloat16*)q, (const __nv_bfloat16*)k,
-                      (const __nv_bfloat16*)v, mask, (__nv_bfloat16*)o, state, (char*)ws);
     else
         s = fwd_impl<__nv_bfloat16>(x, (const __nv_bfloat16*)q, (const __nv_bfloat16*)k,
                                     (const __nv_bfloat16*)v, mask, vd, (__nv_bfloat16*)o, state);
@@ -1439,29 +1313,24 @@ sa_status sinkhorn_attn_step_host(const sa_params* p, const sa_host_step* io, vo
 // Fixed scratch for sinkhorn_attn_bwd_static_ws: one array per device that
 // loads the library, alive until the process exits.  Host code must not use
 // this name as a pointer (it is a host-side stand-in); the device address is
-// looked up once per device below.
+// looked up with cudaGetSymbolAddress, with the device current, on every call.
+// Being a static __device__ array it starts zeroed, so its status word (the
+// first int) reads SA_OK until a backward records a condition in it.
 static __device__ __align__(256) unsigned char g_bwd_scratch[SA_STATIC_SCRATCH_BYTES];
 
 namespace {
-constexpr int kMaxDevices = 64;
-void* g_bwd_scratch_addr[kMaxDevices];   // device address of g_bwd_scratch, per device
-std::mutex g_bwd_scratch_mu;
-
-// Address of the scratch array on the current device (looked up on first use).
+// Address of the scratch array on the current device.  The lookup allocates
+// nothing; it is repeated on every call rather than cached, so that it stays
+// right if the caller tears down and recreates the device's context.  The first
+// call on a device may load the library's module there (CUDA's lazy loading),
+// which is why that first call should come before any stream capture.
 sa_status bwd_scratch_current_device(void** out) {
-    int dev = -1;
-    if (cudaGetDevice(&dev) != cudaSuccess) return SA_ERR_CUDA;
-    if (dev < 0 || dev >= kMaxDevices) return SA_ERR_UNSUPPORTED;
-    std::lock_guard<std::mutex> lock(g_bwd_scratch_mu);
-    if (!g_bwd_scratch_addr[dev]) {
-        void* ptr = nullptr;
-        if (cudaGetSymbolAddress(&ptr, g_bwd_scratch) != cudaSuccess || !ptr) {
-            cudaGetLastError();
-            return SA_ERR_CUDA;
-        }
-        g_bwd_scratch_addr[dev] = ptr;
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_bwd_scratch) != cudaSuccess || !ptr) {
+        cudaGetLastError();
+        return SA_ERR_CUDA;
     }
-    *out = g_bwd_scratch_addr[dev];
+    *out = ptr;
     return SA_OK;
 }
 }  // namespace
@@ -1491,8 +1360,9 @@ sa_status sinkhorn_attn_bwd_static_ws(const sa_params* p, const void* q, const v
     s = bwd_scratch_current_device(&ws);
     if (s != SA_OK) return s;
     cudaStream_t st = (cudaStream_t)stream;
-    // the status header is the only part of the workspace read before it is written
-    if (cudaMemsetAsync(ws, 0, kHeader, st) != cudaSuccess) return SA_ERR_CUDA;
+    // The status word (the only part of the scratch read before it is written)
+    // is not cleared here: a timeout recorded by an earlier call stays there until
+    // sinkhorn_attn_poll_static reads and resets it, as with a workspace.
     Ctx x;
     x.p = p;
     x.d = d;
@@ -1555,8 +1425,19 @@ sa_status sinkhorn_attn_poll(void* ws, void* stream) {
     return (sa_status)h;
 }
 
+sa_status sinkhorn_attn_poll_static(void* stream) {
+    void* ws = nullptr;
+    const sa_status s = bwd_scratch_current_device(&ws);
+    if (s != SA_OK) return s;
+    return sinkhorn_attn_poll(ws, stream);
+}
+
 sa_status sinkhorn_attn_debug_timeout(void* ws, long long budget_cycles, void* stream) {
-    if (!ws || ((uintptr_t)ws & 15)) return SA_ERR_INVALID_ARG;
+    if (!ws) {  // the static scratch's status word on the current device
+        const sa_status s = bwd_scratch_current_device(&ws);
+        if (s != SA_OK) return s;
+    }
+    if (((uintptr_t)ws & 15) || !device_ok(ws)) return SA_ERR_INVALID_ARG;
     const long long b = budget_cycles < 1 ? 1 : (budget_cycles > 100000000LL ? 100000000LL : budget_cycles);
     sa::k_stall<<<1, 32, 0, (cudaStream_t)stream>>>((int*)ws, b);
     return cudaGetLastError() == cudaSuccess ? SA_OK : SA_ERR_CUDA;
@@ -1577,6 +1458,29 @@ sa_status sinkhorn_attn_sq_dist(const void* x, const void* y, long long n, sa_dt
         sa::k_sq_dist<__nv_bfloat16><<<(unsigned)blocks, 256, 0, st>>>(
             (const __nv_bfloat16*)x, (const __nv_bfloat16*)y, n, out);
     return cudaGetLastError() == cudaSuccess ? SA_OK : SA_ERR_CUDA;
+}
+
+sa_status sinkhorn_attn_bias_certificate(int n_depths, const int* depths, int n_tensors,
+                                         const double* sums, double tau, double* eta,
+                                         int* r_star) {
+    if (n_depths < 1 || n_tensors < 1 || !depths || !sums || !eta || !r_star || !(tau >= 0.0))
+        return SA_ERR_INVALID_ARG;
+    for (int i = 0; i < n_depths; ++i)
+        if (depths[i] < 0) return SA_ERR_INVALID_ARG;
+    *r_star = -1;
+    for (int i = 0; i < n_depths; ++i) {
+        double num = 0.0, den = 0.0;  // ||g_R - g_full||^2 and ||g_full||^2 over the tensors
+        for (int t = 0; t < n_tensors; ++t) {
+            const double d2 = sums[((size_t)i * n_tensors + t) * 2];
+            const double n2 = sums[((size_t)i * n_tensors + t) * 2 + 1];
+            if (!(d2 >= 0.0) || !(n2 >= 0.0)) return SA_ERR_INVALID_ARG;
+            num += d2;
+            den += n2;
+        }
+        eta[i] = den > 0.0 ? std::sqrt(num / den) : std::sqrt(num);
+        if (eta[i] <= tau && (*r_star < 0 || depths[i] < *r_star)) *r_star = depths[i];
+    }
+    return SA_OK;
 }
 
 const char* sinkhorn_attn_strerror(sa_status s) {

@@ -71,15 +71,12 @@ def fp32_alu_peak_tflops(sm_max_mhz):
 
 
 # algorithmic band contractions (2 d |Omega| FLOPs each) per launch of each kernel kind
-CONTRACTIONS = {"lse_sweep": 1, "fused_sweep": 1, "pv": 2, "wsum": 1, "ds": 3}
+CONTRACTIONS = {"lse_sweep": 1, "pv": 2, "wsum": 1, "ds": 3}
 
 # DRAM bytes (read + write) per launch from one ncu capture (profiles/), keyed by
 # (workload, kernel kind), with the SHA-256 of the kernel source the capture was
 # taken from: a changed source reports traffic as null until it is captured again.
-MEASURED_TRAFFIC = {
-    ("long32k", "fused_sweep"): (191.4e6, "banded_log_domain_b200/csrc/tc_fused.cuh",
-                                 "67a1c5d4af123c8603fee6eb067c40a72117f1ff85acdec9aa0738b94861b6ce"),
-}
+MEASURED_TRAFFIC = {}
 
 
 def measured_traffic(workload, kind):
@@ -438,7 +435,7 @@ def main():
     achieved = CONTRACTIONS.get(dom_kind, 1) * unit_flops / (avg_ms * 1e-3) / 1e12
     # exponentials: one per support entry per launch of a sweep (diagnostic ceiling)
     mufu_peak = 148 * 16 * peaks["sm_max_mhz"] * 1e6
-    exp_rate = (omega / (avg_ms * 1e-3)) if dom_kind in ("lse_sweep", "fused_sweep", "wsum", "pv") else None
+    exp_rate = (omega / (avg_ms * 1e-3)) if dom_kind in ("lse_sweep", "wsum", "pv") else None
     if simt:
         peak = fp32_alu_peak_tflops(peaks["sm_max_mhz"])
         roof = {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
@@ -446,11 +443,13 @@ def main():
                 "peak_source": "FP32 FFMA: 148 SMs x 128 lanes x 2 FLOP x max SM clock",
                 "launches_per_step": dom_n / args.steps, "avg_launch_ms": avg_ms}
     else:
-        peak = peaks["bf16_tflops_sustained"]
+        # the burst peak: each launch is well under a millisecond, inside a step of a
+        # few milliseconds, not a seconds-long loop under the power cap
+        peak = peaks["bf16_tflops"]
         roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                 "frac": achieved / peak, "traffic": measured_traffic(w.name, dom_kind),
                 "kernel": dom_kind,
-                "peak_source": f"{peaks['source']} bf16 dense (sustained)",
+                "peak_source": f"{peaks['source']} bf16 dense (burst)",
                 "launches_per_step": dom_n / args.steps, "avg_launch_ms": avg_ms,
                 "exp_per_s": exp_rate, "exp_frac_of_mufu": (exp_rate / mufu_peak) if exp_rate else None,
                 "mufu_peak_per_s": mufu_peak}

@@ -26,9 +26,11 @@
  *     memory in any call and keeps no mutable global state, so concurrent
  *     calls on different buffers are safe (sinkhorn_attn_bwd_static_ws is the
  *     one exception: it uses a fixed scratch array inside the library).
- *   - Device pointers must be 16-byte aligned and the tensors contiguous in
+ *   - Device pointers must be 16-byte aligned, point to device memory of the
+ *     current device (or to managed memory), and the tensors be contiguous in
  *     the stated layout; otherwise the call returns SA_ERR_INVALID_ARG before
- *     launching anything.
+ *     launching anything.  Page-locked host memory and another GPU's memory
+ *     are rejected (make the tensors' device current before the call).
  *   - Work is enqueued asynchronously on `stream` (a cudaStream_t; NULL means
  *     the legacy default stream).  Argument and launch errors are returned at
  *     once.  Conditions found on the device (a non-finite dual or output when
@@ -99,8 +101,7 @@ typedef enum {
     SA_KERNEL_PV = 2,          /* O = P V, or dV = P^T dO with vbar = rowdot(V, dV) */
     SA_KERNEL_WSUM = 3,        /* vector cotangent sweep: weighted plan row sums */
     SA_KERNEL_DS = 4,          /* dQ = c dS K or dK = c dS^T Q */
-    SA_KERNEL_AUX = 5,         /* O(L) elementwise helpers */
-    SA_KERNEL_FUSED_SWEEP = 6  /* tensor-core fused iteration (row LSE + column partials) */
+    SA_KERNEL_AUX = 5          /* O(L) elementwise helpers */
 } sa_kernel_kind;
 
 /* Number of float32 elements of the dual state: B*H*(2R+2)*(L+dustbin).
@@ -172,9 +173,8 @@ sa_status sinkhorn_attn_bwd(const sa_params* p, const void* q, const void* k, co
  * the one that ends it; an interior halo must hold at least W tokens (every
  * band neighbour of an own token is then local) and every shard at least W
  * own tokens (a halo then comes from one neighbour).  The sharded calls run the
- * same path with one iteration as a row sweep and a column sweep (the fused
- * single-pass iteration needs both halves of an iteration on one device), and
- * after every sweep that produces a dual or vector cotangent they call
+ * same sweeps as the unsharded ones, and after every sweep that produces a dual
+ * or vector cotangent they call
  *     exchange(vec, row_stride, rows, user, stream)
  * on the host, in stream order (the sweep has been launched on `stream`, not
  * necessarily finished): vec + r * row_stride (r < rows = B*H) is row r's p->L
@@ -274,13 +274,18 @@ sa_status sinkhorn_attn_debug_plan(const sa_params* p, int a, int b, const void*
  * rejected with SA_ERR_WORKSPACE before anything is launched.
  *   - The call allocates nothing: no cudaMalloc/cudaFree or allocating
  *     library routine.
- *   - The first call on a device looks up the array's device address (with
- *     that device current); make that first call before any stream capture.
+ *   - Every call looks up the array's device address on the current device
+ *     (make the tensors' device current); the lookup allocates nothing.  The
+ *     first call on a device may load the library's module on it, so make
+ *     that first call before any stream capture.
  *   - All calls share the one array and it keeps the last call's contents, so
  *     calls whose work overlaps on the GPU (different streams, or different
  *     host threads on one device) race: serialise them.
- *   - check_finite is not supported here (there is no workspace to poll):
- *     SA_ERR_UNSUPPORTED.
+ *   - Conditions found on the device (a bounded wait that gave up:
+ *     SA_ERR_TIMEOUT) go to the status word at the start of the array, where
+ *     they stay, across calls, until sinkhorn_attn_poll_static() reads and
+ *     resets them; poll after the calls whose results you use.
+ *   - check_finite is not supported here: SA_ERR_UNSUPPORTED.
  */
 #define SA_STATIC_SCRATCH_BYTES (32u << 20)
 sa_status sinkhorn_attn_bwd_static_ws(const sa_params* p, const void* q, const void* k,
@@ -293,6 +298,14 @@ sa_status sinkhorn_attn_bwd_static_ws(const sa_params* p, const void* q, const v
  * last forward/backward that used it (SA_OK, SA_ERR_NONFINITE or
  * SA_ERR_TIMEOUT) and resets it to SA_OK. */
 sa_status sinkhorn_attn_poll(void* ws, void* stream);
+
+/* sinkhorn_attn_poll for the fixed scratch array of
+ * sinkhorn_attn_bwd_static_ws on the current device: synchronises `stream`,
+ * returns the status word that the static-scratch backward calls have recorded
+ * since the last poll (SA_OK or SA_ERR_TIMEOUT), and resets it to SA_OK.
+ * No counterpart in the paper (see sinkhorn_attn_bwd_static_ws).  Returns
+ * SA_ERR_CUDA if the array's address cannot be looked up. */
+sa_status sinkhorn_attn_poll_static(void* stream);
 
 /* Static English description of a status code. */
 const char* sinkhorn_attn_strerror(sa_status s);
@@ -313,6 +326,26 @@ const char* sinkhorn_attn_strerror(sa_status s);
 sa_status sinkhorn_attn_sq_dist(const void* x, const void* y, long long n, sa_dtype dtype,
                                double* out, void* stream);
 
+/* The a-posteriori bias certificate from the squared distances (gist.science/de
+ * section 3, section 4.1): for tail depth R the certificate is
+ *     eta_R = ||g_R - g_full|| / ||g_full||
+ * over all gradient tensors together (dQ, dK, dV), g_R the gradients with
+ * T = N - R stopped iterations and g_full full backpropagation (T = 0, R = N);
+ * the depth the pages select at tolerance tau is the smallest R with
+ * eta_R <= tau.  Host-only arithmetic (no device work).
+ *   depths : n_depths tail depths R (>= 0), host.
+ *   sums   : [n_depths][n_tensors][2] doubles, host: entry (i, t) holds
+ *            sinkhorn_attn_sq_dist's (sum (x - y)^2, sum y^2) for tensor t with
+ *            x from depth depths[i] and y from full backpropagation.
+ *   eta    : n_depths doubles, host, written (eta = ||x - y|| when every
+ *            ||y|| is 0).
+ *   r_star : one int, host, written: the smallest depth with eta <= tau, or -1.
+ * Returns SA_ERR_INVALID_ARG for n_depths or n_tensors < 1, a NULL pointer, a
+ * negative depth, tau < 0 or NaN, or a negative or NaN sum; else SA_OK. */
+sa_status sinkhorn_attn_bias_certificate(int n_depths, const int* depths, int n_tensors,
+                                         const double* sums, double tau, double* eta,
+                                         int* r_star);
+
 /* Test hook for the failure path; no counterpart in the pages.  Launches on
  * `stream` one CTA whose thread waits, through the same bounded mbarrier wait
  * every kernel of this library uses, on a barrier that nothing ever arrives on;
@@ -321,8 +354,11 @@ sa_status sinkhorn_attn_sq_dist(const void* x, const void* y, long long n, sa_dt
  * `ws` (a workspace of at least 256 bytes, device memory), exactly as a
  * stalled pipeline stage would.  Nothing faults and the CUDA context stays
  * usable; sinkhorn_attn_poll(ws, stream) then returns SA_ERR_TIMEOUT.
- * Returns SA_ERR_INVALID_ARG for a null or misaligned `ws`, SA_ERR_CUDA on a
- * launch error, else SA_OK. */
+ * With ws == NULL the timeout is recorded in the status word of the fixed
+ * scratch array of sinkhorn_attn_bwd_static_ws on the current device, and
+ * sinkhorn_attn_poll_static(stream) returns it.
+ * Returns SA_ERR_INVALID_ARG for a misaligned `ws` or one that is not device
+ * memory of the current device, SA_ERR_CUDA on a launch error, else SA_OK. */
 sa_status sinkhorn_attn_debug_timeout(void* ws, long long budget_cycles, void* stream);
 
 #ifdef __cplusplus

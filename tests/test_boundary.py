@@ -187,3 +187,49 @@ def test_host_step_plans_and_validates_on_the_host():
         setattr(io, f, buf.data_ptr())
     assert lib.sinkhorn_attn_step_host(ctypes.byref(p), ctypes.byref(io), buf.data_ptr(), 1 << 40,
                                        None) == -1
+
+
+def test_bias_certificate_arithmetic_on_the_host():
+    # eta_R = sqrt(sum_t d2 / sum_t n2) over the tensors; R* = smallest R with eta <= tau
+    lib = sa._L()
+    depths = [4, 0, 2, 1]
+    # per depth, three tensors' (d2, n2); ||g_full||^2 = 1 + 2 + 1 = 4 every time
+    rows = {0: (0.5, 0.3, 0.2), 1: (1e-6, 0.0, 3e-6), 2: (2e-11, 1e-11, 1e-11), 4: (0.0, 0.0, 0.0)}
+    sums = []
+    for R in depths:
+        for d2, n2 in zip(rows[R], (1.0, 2.0, 1.0)):
+            sums += [d2, n2]
+    c_d = (ctypes.c_int * 4)(*depths)
+    c_s = (ctypes.c_double * len(sums))(*sums)
+    eta = (ctypes.c_double * 4)()
+    rs = ctypes.c_int(99)
+    assert lib.sinkhorn_attn_bias_certificate(4, c_d, 3, c_s, 1e-5, eta, ctypes.byref(rs)) == 0
+    want = {0: (1.0 / 4) ** 0.5, 1: (4e-6 / 4) ** 0.5, 2: (4e-11 / 4) ** 0.5, 4: 0.0}
+    for i, R in enumerate(depths):
+        assert abs(eta[i] - want[R]) <= 1e-15 * max(1.0, want[R])
+    assert rs.value == 2  # eta_1 = 1e-3 > tau; eta_2 = 3.2e-6 <= tau; 4 is larger
+    assert lib.sinkhorn_attn_bias_certificate(4, c_d, 3, c_s, 1e-12, eta, ctypes.byref(rs)) == 0
+    assert rs.value == 4
+    assert lib.sinkhorn_attn_bias_certificate(4, c_d, 3, c_s, 0.0, eta, ctypes.byref(rs)) == 0
+    assert rs.value == 4  # eta_4 = 0 <= 0
+    c_s1 = (ctypes.c_double * 6)(0.0, 0.0, 1e-12, 0.0, 0.0, 0.0)  # ||g_full|| = 0
+    c_d1 = (ctypes.c_int * 1)(3)
+    assert lib.sinkhorn_attn_bias_certificate(1, c_d1, 3, c_s1, 1.0, eta, ctypes.byref(rs)) == 0
+    assert eta[0] == 1e-6 and rs.value == 3
+    # invalid arguments
+    bad = (ctypes.c_double * 6)(-1.0, 1.0, 0.0, 1.0, 0.0, 1.0)
+    assert lib.sinkhorn_attn_bias_certificate(1, c_d1, 3, bad, 1.0, eta, ctypes.byref(rs)) == -1
+    assert lib.sinkhorn_attn_bias_certificate(0, c_d, 3, c_s, 1.0, eta, ctypes.byref(rs)) == -1
+    assert lib.sinkhorn_attn_bias_certificate(4, c_d, 0, c_s, 1.0, eta, ctypes.byref(rs)) == -1
+    assert lib.sinkhorn_attn_bias_certificate(4, c_d, 3, c_s, -1.0, eta, ctypes.byref(rs)) == -1
+    assert lib.sinkhorn_attn_bias_certificate(4, c_d, 3, c_s, float("nan"), eta,
+                                              ctypes.byref(rs)) == -1
+    assert lib.sinkhorn_attn_bias_certificate(4, c_d, 3, None, 1.0, eta, ctypes.byref(rs)) == -1
+    neg = (ctypes.c_int * 1)(-2)
+    assert lib.sinkhorn_attn_bias_certificate(1, neg, 3, c_s1, 1.0, eta, ctypes.byref(rs)) == -1
+
+
+def test_binding_does_none_of_the_methods_arithmetic():
+    # the score scale and the certificate's eta / R* live in the C library
+    src = open(os.path.join(ROOT, "banded_log_domain_b200", "__init__.py")).read()
+    assert "score_scale" not in src and "math.sqrt" not in src and "import math" not in src

@@ -34,5 +34,8 @@ def test_timeout_hook_rejects_bad_workspace():
     import banded_log_domain_b200 as sa
 
     lib = sa.load()
-    assert lib.sinkhorn_attn_debug_timeout(None, 1000, None) == -1
+    # misaligned, and plain host memory (not device memory of the current device)
     assert lib.sinkhorn_attn_debug_timeout(ctypes.c_void_p(0x1001), 1000, None) == -1
+    buf = ctypes.create_string_buffer(512)
+    addr = (ctypes.addressof(buf) + 15) & ~15
+    assert lib.sinkhorn_attn_debug_timeout(ctypes.c_void_p(addr), 1000, None) == -1

@@ -58,3 +58,29 @@ def test_host_step_rejects_device_tensors():
     q = torch.zeros(1, 1, 8, 64, device="cuda")
     with pytest.raises(ValueError):
         sa.sinkhorn_attn_step_host(q, q, q, q, W=2, eps=1.0, T=1)
+
+
+@pytest.mark.slow
+def test_host_step_long32k_matches_the_oracle():
+    """The call bench.py's end-to-end number times, at the full long-context
+    size (B=1, H=16, L=32768, W=256, T=20, R=2, bf16) from pinned host buffers,
+    against the CPU oracle on two sampled heads (every (batch, head) problem is
+    independent)."""
+    import numpy as np
+
+    import banded_log_domain_b200 as sa
+    import workloads
+
+    w, x = workloads.make("long32k")
+    h = {k_: (None if v_ is None else v_.contiguous().pin_memory()) for k_, v_ in x.items()}
+    hst = torch.empty(w.B, w.H, 2 * w.R + 2, w.L, dtype=torch.float32).pin_memory()
+    o, dq, dk, dv = sa.sinkhorn_attn_step_host(h["q"], h["k"], h["v"], h["dO"], W=w.W, eps=w.eps,
+                                               T=w.T, R=w.R, groups=5, state=hst)
+    torch.cuda.synchronize()
+    heads = [2, 13]
+    r = parity.oracle_run(x, W=w.W, eps=w.eps, T=w.T, R=w.R, heads=heads)
+    to = lambda t: t.float().double().numpy()
+    g = {"o": to(o), "state": hst.double().numpy(),
+         "one_reference": (to(dq), to(dk), to(dv), None, None)}
+    parity.compare(x, g, r, dtype="bf16", dustbin=False, heads=heads, label="long32k host step")
+    assert np.isfinite(g["state"]).all()
