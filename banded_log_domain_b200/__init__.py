@@ -123,6 +123,7 @@ def _L():
         ctypes.c_double, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int)]
     lib.sinkhorn_attn_debug_timeout.argtypes = [vp, ctypes.c_longlong, vp]
     lib.sinkhorn_attn_sq_dist.argtypes = [vp, vp, ctypes.c_longlong, ctypes.c_int, vp, vp]
+    lib.sinkhorn_attn_debug_exp2.argtypes = [vp, ctypes.c_longlong, vp, vp, vp]
     lib.sinkhorn_attn_step_host_workspace_size.argtypes = [P, ctypes.c_int, ctypes.POINTER(sz)]
     lib.sinkhorn_attn_step_host.argtypes = [P, ctypes.POINTER(sa_host_step), vp, sz, vp]
     SP = ctypes.POINTER(sa_shard)
@@ -134,6 +135,7 @@ def _L():
     for f in ("sinkhorn_attn_state_size", "sinkhorn_attn_workspace_size", "sinkhorn_attn_fwd",
               "sinkhorn_attn_bwd", "sinkhorn_attn_debug_plan", "sinkhorn_attn_poll",
               "sinkhorn_attn_poll_static", "sinkhorn_attn_bias_certificate",
+              "sinkhorn_attn_debug_exp2",
               "sinkhorn_attn_debug_timeout", "sinkhorn_attn_sq_dist", "sinkhorn_attn_fwd_sharded",
               "sinkhorn_attn_bwd_sharded", "sinkhorn_attn_step_host_workspace_size",
               "sinkhorn_attn_step_host"):
@@ -151,6 +153,7 @@ EXPORTS = ("sinkhorn_attn_state_size", "sinkhorn_attn_workspace_size", "sinkhorn
            "sinkhorn_attn_bwd", "sinkhorn_attn_bwd_static_ws", "sinkhorn_attn_debug_plan",
            "sinkhorn_attn_poll", "sinkhorn_attn_poll_static", "sinkhorn_attn_strerror",
            "sinkhorn_attn_debug_timeout", "sinkhorn_attn_bias_certificate",
+           "sinkhorn_attn_debug_exp2",
            "sinkhorn_attn_sq_dist", "sinkhorn_attn_fwd_sharded", "sinkhorn_attn_bwd_sharded",
            "sinkhorn_attn_step_host_workspace_size", "sinkhorn_attn_step_host")
 
@@ -544,6 +547,16 @@ def sinkhorn_attn_debug_timeout(ws, budget_cycles: int = 1_000_000, device=None)
         dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
     return int(_on(dev, _L().sinkhorn_attn_debug_timeout, _ptr(ws), int(budget_cycles),
                    _stream(dev)))
+
+
+def sinkhorn_attn_debug_exp2(x):
+    """``(y_poly, y_mufu)``: 2^x as the row-sum sweeps evaluate it on the FMA pipe
+    and on the MUFU unit, for a contiguous float32 CUDA tensor ``x`` (x <= 0)."""
+    _contig(x)
+    yp, ym = torch.empty_like(x), torch.empty_like(x)
+    _check(_on(x.device, _L().sinkhorn_attn_debug_exp2, _ptr(x), x.numel(), _ptr(yp), _ptr(ym),
+               _stream(x.device)), "sinkhorn_attn_debug_exp2")
+    return yp, ym
 
 
 def sinkhorn_attn_sq_dist(x, y):

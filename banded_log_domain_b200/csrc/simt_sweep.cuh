@@ -81,6 +81,12 @@ struct SweepArgs {
     const void* aug_row;
     const void* aug_col;
     int online;             // LSE on tensor cores: 1 = no previous dual, use a running max
+    // Row-sum sweeps on tensor cores (shifted LSE, WSUM): the duals as working
+    // copies, log2(e) times the dual on valid tokens and -inf on masked ones
+    // ([BH][L], stride s), which the loader copies to shared memory as they are
+    Vec cdw;                // column side
+    Vec rdw;                // row side (LSE: the shift source; WSUM: the row dual)
+    MVec outw;              // LSE: the new dual's working copy (or p null)
 };
 
 // ---------------------------------------------------------------------------

@@ -32,6 +32,7 @@
 #include "../../include/sinkhorn_attn.h"
 #include "simt_sweep.cuh"
 #include "tc_sweep.cuh"
+#include "tc_rowsum.cuh"
 
 namespace sa {
 namespace {
@@ -100,18 +101,29 @@ bool device_f32_ok(const void* x) { return x && ((uintptr_t)x & 3u) == 0 && on_c
 // The byte mask (any alignment; NULL means every token is valid).
 bool mask_ok(const void* x) { return !x || on_current_device(x); }
 
-// Forward workspace: the status header only (the duals live in the state).
+// The row-sum sweeps on the tensor cores (bf16 storage without a dustbin) read
+// the duals as a working copy of the state: [BH][2R+2][L] float32, log2(e)
+// times each dual on valid tokens and -inf on masked ones.
+bool uses_work_state(const sa_params* p) { return p->dtype == SA_BF16 && !p->dustbin; }
+size_t work_state_bytes(const Dims& d) { return align_up((size_t)d.BH * (2 * d.R + 2) * d.L * sizeof(float)); }
+
+// Forward workspace: the status header, then the working copy of the state
+// (tensor-core path only).
 struct FwdLayout {
-    size_t total;
+    size_t work, total;
 };
-FwdLayout fwd_layout(const Dims&, const sa_params*) { return FwdLayout{kHeader}; }
+FwdLayout fwd_layout(const Dims& d, const sa_params* p) {
+    FwdLayout l{kHeader, kHeader};
+    if (uses_work_state(p)) l.total += work_state_bytes(d);
+    return l;
+}
 
 // Backward workspace layout (float32 vectors of BH * ld elements each).
 struct BwdLayout {
-    size_t a, ubar, vbar, eu, ev, w, rv, cv, dvd, dsc, aug, acc, total;
+    size_t a, ubar, vbar, eu, ev, w, rv, cv, dvd, dsc, aug, acc, work, total;
     size_t vec;  // bytes of one [BH][ld] vector, 256-aligned
 };
-BwdLayout bwd_layout(const Dims& d) {
+BwdLayout bwd_layout(const Dims& d, const sa_params* p) {
     BwdLayout l;
     l.vec = align_up((size_t)d.BH * d.ld * sizeof(float));
     size_t o = kHeader;
@@ -128,6 +140,8 @@ BwdLayout bwd_layout(const Dims& d) {
     l.aug = o;  o += 4 * align_up((size_t)d.BH * d.L * 16 * 2);  // bf16 K16 modifier operands
     l.acc = o;  // fp32 sum of the dS sweeps' term blocks, when 2R > MAXT
     if (2 * d.R > simt::MAXT) o += align_up((size_t)d.BH * d.L * kD * sizeof(float));
+    l.work = o;  // the working copy of the state (tensor-core path)
+    if (uses_work_state(p)) o += work_state_bytes(d);
     l.total = o;
     return l;
 }
@@ -188,6 +202,21 @@ __global__ void k_vmul(const float* x, const float* y, float s, float* out, long
     if (x) v *= x[g];
     if (y) v *= y[g];
     out[g] = v;
+}
+
+// Working copy of state rows [r_lo, r_hi) of every problem: w = log2(e) * dual
+// on valid tokens, -inf on masked ones (state [BH][2R+2][ld], work [BH][2R+2][L]).
+__global__ void k_work(const float* state, int nrows, int ld, int L, int H, int BH,
+                       const uint8_t* mask, int r_lo, int r_hi, float* work) {
+    const long long g = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    const int nr = r_hi - r_lo;
+    if (g >= (long long)BH * nr * L) return;
+    const int t = (int)(g % L);
+    const long long rest = g / L;
+    const int row = r_lo + (int)(rest % nr), bh = (int)(rest / nr);
+    const bool ok = mask == nullptr || mask[(size_t)(bh / H) * L + t];
+    const float v = state[((size_t)bh * nrows + row) * ld + t];
+    work[((size_t)bh * nrows + row) * L + t] = ok ? v * kLog2e : -INFINITY;
 }
 
 // dv_dust[h][e] = sum_b part[(b*H + h)][e]
@@ -351,6 +380,22 @@ __global__ void k_stall(int* status, long long budget) {
     __syncthreads();
 }
 
+// The two exponentials of the row-sum sweeps side by side (test hook): y_poly
+// from the FMA-pipe polynomial, y_mufu from ex2.approx, of each x <= 0.
+__global__ void k_exp2_pair(const float* x, long long n, float* y_poly, float* y_mufu) {
+    const long long i = 2 * ((long long)blockIdx.x * blockDim.x + threadIdx.x);
+    if (i >= n) return;
+    const float x0 = x[i], x1 = i + 1 < n ? x[i + 1] : 0.f;
+    float e0, e1;
+    tcr::exp2_poly2(x0, x1, e0, e1);
+    y_poly[i] = e0;
+    y_mufu[i] = ex2(x0);
+    if (i + 1 < n) {
+        y_poly[i + 1] = e1;
+        y_mufu[i + 1] = ex2(x1);
+    }
+}
+
 // Sets the status word when any element is NaN or Inf.
 template <typename T>
 __global__ void k_finite(const T* x, long long n, int* status) {
@@ -503,6 +548,44 @@ cudaError_t launch_tc(const simt::SweepArgs& a, int BH, cudaStream_t st, Tracer&
     return cudaGetLastError();
 }
 
+int sm_count() {
+    static int nsm = 0;
+    if (nsm == 0) {
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || nsm <= 0)
+            nsm = 148;
+    }
+    return nsm;
+}
+
+// Exponentials of every 32 entries of a row-sum sweep's in-band group that run
+// on the FMA pipe (the rest on the MUFU unit).
+#ifndef SA_ROWSUM_KP
+#define SA_ROWSUM_KP 8
+#endif
+
+// The row-sum sweeps (shifted LSE, WSUM) on the tensor cores: persistent, one
+// CTA per SM.
+template <int MODE>
+cudaError_t launch_rowsum(const simt::SweepArgs& a, int BH, cudaStream_t st, Tracer& tr,
+                          int* status) {
+    tcr::Maps maps;
+    std::memset(&maps, 0, sizeof(maps));
+    if (!make_map(&maps.A, a.A, a.L, BH) || !make_map(&maps.B, a.Bo, a.L, BH))
+        return cudaErrorInvalidValue;
+    const long long ntiles = (long long)((a.L + 127) / 128) * BH;
+    const dim3 grid((unsigned)std::min<long long>(ntiles, (long long)sm_count()));
+    auto kern = tcr::tc_rowsum_sweep<MODE, SA_ROWSUM_KP>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         tcr::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    tr.begin(kind_of(MODE));
+    kern<<<grid, tcr::NTHREADS, tcr::SMEM_BYTES, st>>>(a, maps, status, BH);
+    tr.end();
+    return cudaGetLastError();
+}
+
 template <typename T, int MODE>
 cudaError_t launch_sweep(const simt::SweepArgs& a, int BH, cudaStream_t st, Tracer& tr,
                          int* status) {
@@ -511,7 +594,9 @@ cudaError_t launch_sweep(const simt::SweepArgs& a, int BH, cudaStream_t st, Trac
         if (!a.dustbin) {
             if constexpr (MODE == simt::LSE) {
                 if (a.online) return launch_tc<MODE, true, 0>(a, BH, st, tr, status);
-                return launch_tc<MODE, false, 0>(a, BH, st, tr, status);
+                return launch_rowsum<MODE>(a, BH, st, tr, status);
+            } else if constexpr (MODE == simt::WSUM) {
+                return launch_rowsum<MODE>(a, BH, st, tr, status);
             } else if constexpr (MODE == simt::DS1 || MODE == simt::DSD) {
                 if (MODE == simt::DS1 && a.nterms == 0)  // R = 0: dS = P * G
                     return launch_tc<MODE, false, 0>(a, BH, st, tr, status);
@@ -562,6 +647,22 @@ struct Ctx {
     const sa_shard* shard = nullptr;  // sequence-sharded call, else null
     // state row r (0..2R+1) as a Vec
     Vec srow(int r) const { return vec(state + (size_t)r * d.ld, sst); }
+    // its working copy (tensor-core row-sum sweeps), or a null Vec
+    float* work = nullptr;
+    Vec wrow(int r) const {
+        return work ? vec(work + (size_t)r * d.L, (long long)(2 * d.R + 2) * d.L) : Vec{nullptr, 0};
+    }
+    MVec mwrow(int r) const { Vec v = wrow(r); return MVec{const_cast<float*>(v.p), v.s}; }
+    // rebuilds working rows [lo, hi) from the state
+    sa_status refresh_work(const uint8_t* mask, int lo, int hi) const {
+        if (!work) return SA_OK;
+        const long long n = (long long)d.BH * (hi - lo) * d.L;
+        tr.begin(SA_KERNEL_AUX);
+        k_work<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(state, 2 * d.R + 2, d.ld, d.L, d.H,
+                                                             d.BH, mask, lo, hi, work);
+        tr.end();
+        return cudaGetLastError() == cudaSuccess ? SA_OK : SA_ERR_CUDA;
+    }
     // sharded calls: the neighbours' values into the halo entries of a vector
     // just produced (rows of d.L entries, row_stride apart)
     sa_status halo(const float* v, long long row_stride) const {
@@ -606,6 +707,8 @@ sa_status fwd_impl(const Ctx& x, const T* q, const T* k, const T* v, const uint8
     const Dims& d = x.d;
     // v0 = 0 and u0 = 0 (u0 stays 0 when T == 0)
     SA_CUDA(cudaMemsetAsync(state, 0, (size_t)d.BH * (2 * d.R + 2) * d.ld * sizeof(float), x.st));
+    sa_status s = x.refresh_work(mask, 1, 2);  // v0's working copy
+    if (s != SA_OK) return s;
     simt::SweepArgs a = base_args(x);
     a.mask = mask;
     const int iters = x.p->T + d.R;
@@ -617,18 +720,34 @@ sa_status fwd_impl(const Ctx& x, const T* q, const T* k, const T* v, const uint8
         a.A = q; a.Bo = k;
         a.cd = x.srow(2 * rin + 1);
         a.rd = x.srow(2 * rin);
+        a.cdw = x.wrow(2 * rin + 1);
+        a.rdw = x.wrow(2 * rin);
+        a.outw = x.mwrow(2 * rout);
         a.online = (it == 0);
         a.out_vec = mvec(state + (size_t)(2 * rout) * d.ld, x.sst);
         SA_CUDA((launch_sweep<T, simt::LSE>(a, d.BH, x.st, x.tr, x.status)));
         SA_HALO(x, a.out_vec.p, x.sst);
+        // the first update (a running max, no working copy) and sharded calls
+        // (the exchange refills the state's halo entries) renew the working copy
+        if (it == 0 || x.shard) {
+            s = x.refresh_work(mask, 2 * rout, 2 * rout + 1);
+            if (s != SA_OK) return s;
+        }
         // columns: v^(rout) = -LSE_i(S + u^(rout)), shifted by the previous v
         a.A = k; a.Bo = q;
         a.cd = x.srow(2 * rout);
         a.rd = x.srow(2 * rin + 1);
+        a.cdw = x.wrow(2 * rout);
+        a.rdw = x.wrow(2 * rin + 1);
+        a.outw = x.mwrow(2 * rout + 1);
         a.online = 0;
         a.out_vec = mvec(state + (size_t)(2 * rout + 1) * d.ld, x.sst);
         SA_CUDA((launch_sweep<T, simt::LSE>(a, d.BH, x.st, x.tr, x.status)));
         SA_HALO(x, a.out_vec.p, x.sst);
+        if (x.shard) {
+            s = x.refresh_work(mask, 2 * rout + 1, 2 * rout + 2);
+            if (s != SA_OK) return s;
+        }
     }
     // O = P^(R,R) V (+ dustbin column times v_dust)
     simt::SweepArgs b = base_args(x);
@@ -649,7 +768,7 @@ sa_status bwd_impl(const Ctx& x, const T* q, const T* k, const T* v, const uint8
                    float* dv_dust, float* d_score, char* ws) {
     const Dims& d = x.d;
     const int R = d.R;
-    const BwdLayout l = bwd_layout(d);
+    const BwdLayout l = bwd_layout(d, x.p);
     const long long vs = d.ld;  // per-bh stride of a workspace vector
     const size_t vstride = l.vec / sizeof(float);
     auto W_ = [&](size_t off, int idx) { return (float*)(ws + off + (size_t)idx * l.vec); };
@@ -660,6 +779,11 @@ sa_status bwd_impl(const Ctx& x, const T* q, const T* k, const T* v, const uint8
     const unsigned egrid = (unsigned)((nvec + eb - 1) / eb);
     const bool direct = x.p->bwd == SA_BWD_DIRECT;
 
+    // the working copy of the whole state (read by the row-sum sweeps)
+    {
+        const sa_status s = x.refresh_work(mask, 0, 2 * R + 2);
+        if (s != SA_OK) return s;
+    }
     // a = rowdot(dO, O); orbit factors
     {
         const long long thr = nvec * (kD / (16 / (long long)sizeof(T)));
@@ -695,6 +819,7 @@ sa_status bwd_impl(const Ctx& x, const T* q, const T* k, const T* v, const uint8
         a.mask = mask;
         a.A = q; a.Bo = k;
         a.rd = uR; a.cd = vR;
+        a.rdw = x.wrow(2 * R); a.cdw = x.wrow(2 * R + 1);
         a.w = vec(vb(R), vs);
         a.base = vec(A_, vs);
         a.sgn = -1.f;
@@ -711,10 +836,12 @@ sa_status bwd_impl(const Ctx& x, const T* q, const T* k, const T* v, const uint8
         a.out_vec = mvec(vb(r - 1), vs);
         if (direct) {
             a.rd = V(r - 1); a.cd = U(r);
+            a.rdw = x.wrow(2 * (r - 1) + 1); a.cdw = x.wrow(2 * r);
             a.w = vec(ub(r), vs);
         } else {
             SA_AUX(x.tr, k_vmul<<<egrid, eb, 0, x.st>>>(eu(r), ub(r), 1.f, W_(l.w, 0), nvec));
             a.rd = vR; a.cd = uR;
+            a.rdw = x.wrow(2 * R + 1); a.cdw = x.wrow(2 * R);
             a.w = vec(W_(l.w, 0), vs);
             a.mult = vec(ev(r - 1), vs);
         }
@@ -728,10 +855,12 @@ sa_status bwd_impl(const Ctx& x, const T* q, const T* k, const T* v, const uint8
         b.out_vec = mvec(ub(r - 1), vs);
         if (direct) {
             b.rd = U(r - 1); b.cd = V(r - 1);
+            b.rdw = x.wrow(2 * (r - 1)); b.cdw = x.wrow(2 * (r - 1) + 1);
             b.w = vec(vb(r - 1), vs);
         } else {
             SA_AUX(x.tr, k_vmul<<<egrid, eb, 0, x.st>>>(ev(r - 1), vb(r - 1), 1.f, W_(l.w, 0), nvec));
             b.rd = uR; b.cd = vR;
+            b.rdw = x.wrow(2 * R); b.cdw = x.wrow(2 * R + 1);
             b.w = vec(W_(l.w, 0), vs);
             b.mult = vec(eu(r - 1), vs);
         }
@@ -889,7 +1018,7 @@ sa_status sinkhorn_attn_workspace_size(const sa_params* p, size_t* fwd_bytes, si
     sa_status s = check_params(p, &d);
     if (s != SA_OK) return s;
     if (fwd_bytes) *fwd_bytes = fwd_layout(d, p).total;
-    if (bwd_bytes) *bwd_bytes = bwd_layout(d).total;
+    if (bwd_bytes) *bwd_bytes = bwd_layout(d, p).total;
     return SA_OK;
 }
 
@@ -929,6 +1058,7 @@ sa_status fwd_call(const sa_params* p, const sa_shard* shard, const void* q, con
     x.tr.p = p;
     x.tr.st = x.st;
     x.shard = shard;
+    if (uses_work_state(p)) x.work = (float*)((char*)ws + fwd_layout(d, p).work);
     const float* vd = p->dustbin ? v_dust : nullptr;
     if (p->dtype == SA_F32)
         s = fwd_impl<float>(x, (const float*)q, (const float*)k, (const float*)v, mask, vd,
@@ -958,7 +1088,7 @@ sa_status bwd_call(const sa_params* p, const sa_shard* shard, const void* q, con
     Dims d;
     sa_status s = check_params(p, &d);
     if (s != SA_OK) return s;
-    if (ws_bytes < bwd_layout(d).total) return SA_ERR_WORKSPACE;
+    if (ws_bytes < bwd_layout(d, p).total) return SA_ERR_WORKSPACE;
     if (d.BH == 0 || d.L == 0) return SA_OK;
     if (!device_ok(q) || !device_ok(k) || !device_ok(v) || !device_ok(o) || !device_ok(dO) ||
         !device_ok(state) || !device_ok(dq) || !device_ok(dk) || !device_ok(dv) ||
@@ -978,6 +1108,7 @@ sa_status bwd_call(const sa_params* p, const sa_shard* shard, const void* q, con
     x.tr.p = p;
     x.tr.st = x.st;
     x.shard = shard;
+    if (uses_work_state(p)) x.work = (float*)((char*)ws + bwd_layout(d, p).work);
     const float* vd = p->dustbin ? v_dust : nullptr;
     float* dvd = p->dustbin ? dv_dust : nullptr;
     float* dsc = p->dustbin ? d_dust_score : nullptr;
@@ -1127,7 +1258,7 @@ HostLayout host_layout(const sa_params* p, const std::vector<Group>& gs) {
         Dims d;
         check_params(&q, &d);
         l.fws = align_up(fwd_layout(d, &q).total);
-        l.bws = align_up(bwd_layout(d).total);
+        l.bws = align_up(bwd_layout(d, &q).total);
     }
     size_t o = 0;
     for (int i = 0; i < 8; ++i) { l.mat_off[i] = o; o += l.mat; }
@@ -1346,7 +1477,7 @@ sa_status sinkhorn_attn_bwd_static_ws(const sa_params* p, const void* q, const v
     sa_status s = check_params(p, &d);
     if (s != SA_OK) return s;
     if (p->check_finite) return SA_ERR_UNSUPPORTED;
-    const size_t need = bwd_layout(d).total;
+    const size_t need = bwd_layout(d, p).total;
     if (need > (size_t)SA_STATIC_SCRATCH_BYTES) return SA_ERR_WORKSPACE;
     if (d.BH == 0 || d.L == 0) return SA_OK;
     if (!device_ok(q) || !device_ok(k) || !device_ok(v) || !device_ok(o) || !device_ok(dO) ||
@@ -1373,6 +1504,7 @@ sa_status sinkhorn_attn_bwd_static_ws(const sa_params* p, const void* q, const v
     x.status = (int*)ws;
     x.tr.p = p;
     x.tr.st = st;
+    if (uses_work_state(p)) x.work = (float*)((char*)ws + bwd_layout(d, p).work);
     const float* vd = p->dustbin ? v_dust : nullptr;
     float* dvd = p->dustbin ? dv_dust : nullptr;
     float* dsc = p->dustbin ? d_dust_score : nullptr;
@@ -1440,6 +1572,18 @@ sa_status sinkhorn_attn_debug_timeout(void* ws, long long budget_cycles, void* s
     if (((uintptr_t)ws & 15) || !device_ok(ws)) return SA_ERR_INVALID_ARG;
     const long long b = budget_cycles < 1 ? 1 : (budget_cycles > 100000000LL ? 100000000LL : budget_cycles);
     sa::k_stall<<<1, 32, 0, (cudaStream_t)stream>>>((int*)ws, b);
+    return cudaGetLastError() == cudaSuccess ? SA_OK : SA_ERR_CUDA;
+}
+
+sa_status sinkhorn_attn_debug_exp2(const float* x, long long n, float* y_poly, float* y_mufu,
+                                   void* stream) {
+    if (n < 0) return SA_ERR_INVALID_ARG;
+    if (n == 0) return SA_OK;
+    if (!sa::device_f32_ok(x) || !sa::device_f32_ok(y_poly) || !sa::device_f32_ok(y_mufu))
+        return SA_ERR_INVALID_ARG;
+    const long long pairs = (n + 1) / 2;
+    sa::k_exp2_pair<<<(unsigned)((pairs + 255) / 256), 256, 0, (cudaStream_t)stream>>>(x, n, y_poly,
+                                                                                      y_mufu);
     return cudaGetLastError() == cudaSuccess ? SA_OK : SA_ERR_CUDA;
 }
 

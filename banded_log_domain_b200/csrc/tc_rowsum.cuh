@@ -1,0 +1,520 @@
+// Row-sum band sweeps on the tensor cores (bf16 storage): the dual update
+// (LSE) and the vector-cotangent sweep (WSUM) of the method, one launch per
+// sweep over every (batch, head) problem.
+//
+//   LSE : out_i = -log sum_j exp(S_ij + cd_j)                   (rd: the shift source)
+//   WSUM: out_i = base_i + sgn * mult_i * sum_j exp(S_ij + rd_i + cd_j) w_j
+//
+// with S = QK^T / (sqrt(d) eps) on the band |i - j| <= W (both tokens valid).
+// These are the two sweeps whose per-entry work is one exponential and one
+// addition (or FMA) into a row sum, so their speed is the exponential rate.
+//
+// Layout of the work.  A CTA per SM walks a contiguous range of (problem, row
+// block of 128) tiles.  A tile's columns are the chunks r0 - W + 128 c,
+// c < nch = ceil((2W + 128) / 128), on one grid for the whole problem, so that
+// the next row block of the same problem needs only one new chunk: the K-side
+// chunks (TMA tiles with their column duals) sit in a ring of NRING slots and
+// a chunk stays until the last tile that reads it has (reuse; streaming when
+// W is so large that a tile's chunks do not fit the ring).  Scores go to one
+// of four TMEM buffers (chunk g of the range in buffer g % 4), and epilogue
+// warp (quadrant q, part p) processes the 32 rows of quadrant q of every chunk
+// g with g % 4 == p: a whole 128-column chunk per warp, so the MMA runs up to
+// four chunks ahead.  The four parts' partial row sums of a tile meet in
+// shared memory; the last part of a quadrant to finish the tile writes its 32
+// outputs (a counter per quadrant, no waiting).
+//
+// Operand traffic.  Q and K tiles come by TMA; the O(L) vectors by 4-byte
+// cp.async into the same ring slots (completion counted on the slot's
+// mbarrier), so the loader never waits for a global load.  The duals are read
+// as working copies (log2(e) times the dual, -inf on masked tokens), which
+// each LSE sweep writes next to its natural-unit output for the sweep after it:
+// no mask or scaling on the loader's path.  Columns outside [0, L) are
+// zero-filled and excluded by the band-edge test.
+//
+// Exponent shift.  Every term is a plan entry of a plan with unit columns (or
+// rows) and so is at most 1 when shifted by the row's previous dual rd_i.  A
+// warp uses one shift for its 32 rows, the smallest rd_i of the valid rows, so
+// that the per-entry argument is one FMA, c2 * s + (cd_j + shift), with the
+// column part formed once per chunk; all arguments stay <= 0.  When the rows'
+// duals spread over more than 64 (log2 units) the warp falls back to per-row
+// shifts (one more addition per entry).
+//
+// Exponentials: 2^x on the MUFU unit (ex2.approx), and for KP of every 32
+// entries of a group that lies inside the band on the FMA pipe: range
+// reduction x = n + f, |f| <= 1/2, n by round-to-nearest (adding 1.5 * 2^23),
+// 2^f from a degree-5 polynomial fitted by least squares on Chebyshev nodes to
+// the relative error (at most 2.2e-7 with fp32 Horner FMAs, the accuracy of
+// ex2.approx), and 2^n added to the result's exponent field.  Arguments are
+// clamped at -126 (the result is then below 2^-125, nothing next to a row sum
+// that holds a term close to 1).
+#pragma once
+
+#include "common.cuh"
+#include "simt_sweep.cuh"
+#include "tc_ptx.cuh"
+
+namespace sa {
+namespace tcr {
+
+using simt::SweepArgs;
+constexpr int LSE = simt::LSE, WSUM = simt::WSUM;
+
+constexpr int NEPI = 16;                 // epilogue warps: quadrant w % 4, part w / 4
+constexpr int W_LOAD = NEPI, W_MMA = NEPI + 1;
+constexpr int NTHREADS = (NEPI + 2) * 32;
+constexpr int NRING = 8;                 // K-chunk ring slots
+constexpr int NRED = 8;                  // ring of per-tile partial row sums
+constexpr int TILE = 16384;              // 128 tokens x 64 bf16, 128-byte swizzle
+constexpr long long kWaitBudget = 4000000000LL;  // clock cycles (about 2 s)
+constexpr float kFallbackSpread = 64.f;  // log2 units
+
+// nch chunks of one tile fit the ring with two to spare: chunks are reused
+__host__ __device__ constexpr int nchunks(int W) { return (2 * W + 128 + 127) / 128; }
+__host__ __device__ constexpr bool reuse_ok(int W) { return nchunks(W) + 2 <= NRING; }
+
+// shared memory (offsets from a 1024-aligned base)
+constexpr int OFF_A = 0;                              // 2 row-block tiles (tile parity)
+constexpr int OFF_K = OFF_A + 2 * TILE;               // NRING chunk tiles
+constexpr int OFF_CV = OFF_K + NRING * TILE;          // NRING x 128 column duals (log2)
+constexpr int OFF_WV = OFF_CV + NRING * 128 * 4;      // NRING x 128 weights (WSUM)
+constexpr int OFF_SCR = OFF_WV + NRING * 128 * 4;     // per warp: 128 shifted column duals
+constexpr int OFF_RED = OFF_SCR + NEPI * 128 * 4;     // NRED x 4 parts x 128 partial sums
+constexpr int OFF_CNT = OFF_RED + NRED * 4 * 128 * 4; // NRED x 4 arrival counters
+// Per-tile row data, copied by the loader ahead of the epilogue (a ring of NRI
+// tiles): the rows' working duals (shift sources or row duals), and the WSUM
+// base and multiplier.
+constexpr int NRI = 4;
+struct RowInfo {
+    float rw[128];
+    float base[128];
+    float mult[128];
+};
+constexpr int OFF_RI = OFF_CNT + NRED * 4 * 4;
+constexpr int OFF_BAR = (OFF_RI + NRI * (int)sizeof(RowInfo) + 7) / 8 * 8;
+enum { B_AFULL = 0, B_AEMPTY = 2, B_FULL = 4, B_EMPTY = B_FULL + NRING, B_SFULL = B_EMPTY + NRING,
+       B_SEMPTY = B_SFULL + 4, B_RFULL = B_SEMPTY + 4, B_REMPTY = B_RFULL + NRI,
+       B_DRAIN = B_REMPTY + NRI, NBAR = B_DRAIN + 1 };
+constexpr int SMEM_BYTES = OFF_BAR + NBAR * 8 + 16 + 1024;
+static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
+
+struct Maps {
+    CUtensorMap A, B;
+};
+
+struct Ctl {
+    uint64_t* bar;
+    volatile int* abort;
+    int* status;
+    __device__ bool wait(int slot, uint32_t parity) {
+        if (tc::mbar_try_wait(bar + slot, parity)) return true;
+        if (*abort) return false;
+        if (tc::mbar_wait(bar + slot, parity, kWaitBudget)) return true;
+        *abort = 1;
+        if (status) atomicCAS(status, 0, (int)SA_ERR_TIMEOUT);
+        return false;
+    }
+};
+
+// (problem, row block) of the tiles of a range, advanced without divisions
+struct Cursor {
+    int rb, h, b;
+    __device__ void next(int nb, int H) {
+        if (++rb == nb) {
+            rb = 0;
+            if (++h == H) { h = 0; ++b; }
+        }
+    }
+};
+
+// Ring positions of a tile's chunks: tile `it` reads load numbers base ..
+// base + nch - 1 (slot = number mod NRING).  A successor (the next row block of
+// the same problem, with reuse) shares all but its last chunk with the tile
+// before it.
+struct ChunkIds {
+    int base = 0, next = 0;
+    __device__ int advance(bool successor, int nch) {  // the first chunk to load
+        base = successor ? base + 1 : next;
+        next = base + nch;
+        return successor ? nch - 1 : 0;
+    }
+};
+
+// 2^x on the FMA pipe for a pair of arguments (see the file comment); x <= 0.
+__device__ __forceinline__ void exp2_poly2(float x0, float x1, float& e0, float& e1) {
+    const uint64_t xx = tc::pk2(fmaxf(x0, -126.f), fmaxf(x1, -126.f));
+    const uint64_t mag = tc::pk2(12582912.f, 12582912.f);  // 1.5 * 2^23
+    const uint64_t t = tc::add2(xx, mag);                   // 1.5 * 2^23 + round(x)
+    const uint64_t n = tc::add2(t, tc::pk2(-12582912.f, -12582912.f));
+    const uint64_t f = tc::sub2(xx, n);                     // x - round(x), in [-1/2, 1/2]
+    uint64_t p = tc::fma2(tc::pk2(1.327647129073739e-3f, 1.327647129073739e-3f), f,
+                          tc::pk2(9.675540961325169e-3f, 9.675540961325169e-3f));
+    p = tc::fma2(p, f, tc::pk2(5.550713092088699e-2f, 5.550713092088699e-2f));
+    p = tc::fma2(p, f, tc::pk2(2.4022120237350464e-1f, 2.4022120237350464e-1f));
+    p = tc::fma2(p, f, tc::pk2(6.931469440460205e-1f, 6.931469440460205e-1f));
+    p = tc::fma2(p, f, tc::pk2(1.0000001192092896f, 1.0000001192092896f));
+    float p0, p1, t0, t1;
+    tc::upk2(p, p0, p1);
+    tc::upk2(t, t0, t1);
+    // the low bits of t hold round(x); shifted into the exponent field they add
+    // round(x) to the exponent of p (the shifter's own bits shift out)
+    e0 = __uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23));
+    e1 = __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23));
+}
+
+// One warp's 32 rows x 32 columns: arguments x_j = c2 s_j + cs_j (+ delta), the
+// exponentials (KP of them on the FMA pipe when the group is inside the band),
+// and their sum into acc (LSE) or their w-weighted sum (WSUM).
+template <int MODE, int KP, bool EDGE, bool FB>
+__device__ __forceinline__ void group(const uint32_t (&u)[32], const float* cs, const float* wv,
+                                      float c2, float delta, int d_first, int W, int cg, int L,
+                                      uint64_t (&acc)[4]) {
+    const uint64_t c2p = tc::pk2(c2, c2), dp = tc::pk2(delta, delta);
+    const float4* c4 = reinterpret_cast<const float4*>(cs);
+    const float4* w4 = reinterpret_cast<const float4*>(wv);
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+        const float4 cv = c4[q];
+        uint64_t a01 = tc::fma2(tc::pk2(__uint_as_float(u[4 * q]), __uint_as_float(u[4 * q + 1])), c2p,
+                                tc::pk2(cv.x, cv.y));
+        uint64_t a23 = tc::fma2(tc::pk2(__uint_as_float(u[4 * q + 2]), __uint_as_float(u[4 * q + 3])), c2p,
+                                tc::pk2(cv.z, cv.w));
+        if (FB) {
+            a01 = tc::add2(a01, dp);
+            a23 = tc::add2(a23, dp);
+        }
+        float x[4];
+        tc::upk2(a01, x[0], x[1]);
+        tc::upk2(a23, x[2], x[3]);
+        if (EDGE) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int d = d_first - (4 * q + e);  // row - column
+                const int col = cg + 4 * q + e;
+                if ((unsigned)(d + W) > (unsigned)(2 * W) || (unsigned)col >= (unsigned)L) x[e] = -INFINITY;
+            }
+        }
+        float e[4];
+        if (!EDGE && 4 * q + 4 > 32 - KP) {
+            exp2_poly2(x[0], x[1], e[0], e[1]);
+            exp2_poly2(x[2], x[3], e[2], e[3]);
+        } else {
+#pragma unroll
+            for (int k = 0; k < 4; ++k) e[k] = ex2(x[k]);
+        }
+        if (MODE == WSUM) {
+            const float4 w = w4[q];
+            acc[(2 * q) & 3] = tc::fma2(tc::pk2(e[0], e[1]), tc::pk2(w.x, w.y), acc[(2 * q) & 3]);
+            acc[(2 * q + 1) & 3] = tc::fma2(tc::pk2(e[2], e[3]), tc::pk2(w.z, w.w), acc[(2 * q + 1) & 3]);
+        } else {
+            acc[(2 * q) & 3] = tc::add2(acc[(2 * q) & 3], tc::pk2(e[0], e[1]));
+            acc[(2 * q + 1) & 3] = tc::add2(acc[(2 * q + 1) & 3], tc::pk2(e[2], e[3]));
+        }
+    }
+}
+
+template <int MODE, int KP>
+__global__ void __launch_bounds__(NTHREADS, 1) tc_rowsum_sweep(const SweepArgs a,
+                                                              const __grid_constant__ Maps maps,
+                                                              int* status, int BH) {
+    static_assert(KP % 4 == 0 && KP >= 0 && KP <= 32, "poly exponentials per group");
+    extern __shared__ uint8_t smraw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>(((uintptr_t)smraw + 1023) & ~(uintptr_t)1023);
+    uint64_t* bar = reinterpret_cast<uint64_t*>(sm + OFF_BAR);
+    uint32_t* tbase = reinterpret_cast<uint32_t*>(sm + OFF_BAR + NBAR * 8);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tbase + 1);
+    float* cvring = reinterpret_cast<float*>(sm + OFF_CV);
+    float* wring = reinterpret_cast<float*>(sm + OFF_WV);
+    float* red = reinterpret_cast<float*>(sm + OFF_RED);
+    int* cnt = reinterpret_cast<int*>(sm + OFF_CNT);
+    RowInfo* rinfo = reinterpret_cast<RowInfo*>(sm + OFF_RI);
+    Ctl ctl{bar, abort_flag, status};
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int L = a.L, W = a.W, H = a.H;
+    const int nblk = (L + 127) / 128, nch = nchunks(W);
+    const bool reuse = reuse_ok(W);
+    const int ntiles = BH * nblk;
+    const int t0 = (int)(((long long)blockIdx.x * ntiles) / gridDim.x);
+    const int t1 = (int)(((long long)(blockIdx.x + 1) * ntiles) / gridDim.x);
+    const int ntl = t1 - t0;
+    const Cursor cur0{t0 % nblk, (t0 / nblk) % H, (t0 / nblk) / H};
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < 2; ++i) {
+            tc::mbar_init(bar + B_AFULL + i, 1);
+            tc::mbar_init(bar + B_AEMPTY + i, 1);
+        }
+        for (int s = 0; s < NRING; ++s) {
+            tc::mbar_init(bar + B_FULL + s, 33);      // the TMA bytes + 32 column-vector lanes
+            tc::mbar_init(bar + B_EMPTY + s, 1 + 4);  // the last MMA + the 4 quadrant warps
+        }
+        for (int b = 0; b < 4; ++b) {
+            tc::mbar_init(bar + B_SFULL + b, 1);
+            tc::mbar_init(bar + B_SEMPTY + b, 4);
+        }
+        for (int i = 0; i < NRI; ++i) {
+            tc::mbar_init(bar + B_RFULL + i, 32);     // the loader lanes' copies
+            tc::mbar_init(bar + B_REMPTY + i, NEPI);  // every epilogue warp has read it
+        }
+        tc::mbar_init(bar + B_DRAIN, 1);
+        *abort_flag = 0;
+        tc::fence_mbar_init();
+    }
+    for (int i = threadIdx.x; i < NRED * 4; i += NTHREADS) cnt[i] = 0;
+    if (warp == 0) {
+        tc::tmem_alloc(tbase, 512);
+        tc::tmem_relinquish();
+    }
+    tc::tc_fence_before();
+    __syncthreads();
+    tc::tc_fence_after();
+    const uint32_t tS = *tbase;  // score buffer b at columns 128 b
+
+    if (warp == W_LOAD) {
+        // ------------------------------------------------------------ loader
+        if (lane == 0) {
+            tc::prefetch_tmap(&maps.A);
+            tc::prefetch_tmap(&maps.B);
+        }
+        ChunkIds ids;
+        int issued = 0, a_issued = 0, pbh = -1, prb = -1;
+        bool ok = true;
+        Cursor cur = cur0;
+        for (int it = 0; ok && it < ntl; ++it, cur.next(nblk, H)) {
+            const int bh = cur.b * H + cur.h, r0 = cur.rb * 128;
+            const bool succ = reuse && bh == pbh && cur.rb == prb + 1;
+            pbh = bh;
+            prb = cur.rb;
+            const int first = ids.advance(succ, nch);
+            if (lane == 0) {
+                if (it >= 2 && !ctl.wait(B_AEMPTY + (it & 1), ((it >> 1) - 1) & 1)) ok = false;
+                if (ok) {
+                    tc::mbar_expect_tx(bar + B_AFULL + (it & 1), TILE);
+                    tc::tma_load_3d(sm + OFF_A + (it & 1) * TILE, &maps.A, bar + B_AFULL + (it & 1), 0,
+                                    r0, bh);
+                    a_issued = it + 1;
+                }
+            }
+            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+            // the tile's row data (lane l copies rows 32k + l)
+            if (ok && it >= NRI && !ctl.wait(B_REMPTY + it % NRI, ((it / NRI) - 1) & 1)) ok = false;
+            if (ok) {
+                RowInfo& ri = rinfo[it % NRI];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const int r = r0 + 32 * k + lane;
+                    const bool in = r < L;
+                    const long long o = (long long)bh * a.rdw.s + (in ? r : 0);
+                    tc::cp_async4(&ri.rw[32 * k + lane], a.rdw.p + o, in);
+                    if (MODE == WSUM) {
+                        const long long ob = (long long)bh * a.base.s + (in ? r : 0);
+                        const long long om = (long long)bh * a.mult.s + (in ? r : 0);
+                        tc::cp_async4(&ri.base[32 * k + lane], a.base.p ? a.base.p + ob : a.rdw.p + o,
+                                      in && a.base.p);
+                        tc::cp_async4(&ri.mult[32 * k + lane], a.mult.p ? a.mult.p + om : a.rdw.p + o,
+                                      in && a.mult.p);
+                    }
+                }
+                tc::cp_async_arrive(bar + B_RFULL + it % NRI);
+            }
+            for (int c = first; ok && c < nch; ++c) {
+                const int id = ids.base + c, s = id % NRING;
+                if (id >= NRING && !ctl.wait(B_EMPTY + s, ((id / NRING) - 1) & 1)) { ok = false; break; }
+                const int col0 = r0 - W + 128 * c;
+                if (lane == 0) {
+                    tc::mbar_expect_tx(bar + B_FULL + s, TILE);
+                    tc::tma_load_3d(sm + OFF_K + s * TILE, &maps.B, bar + B_FULL + s, 0, col0, bh);
+                }
+                issued = id + 1;
+                // working column duals and WSUM weights; zero off [0, L)
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const int col = col0 + 32 * k + lane;
+                    const bool in = col >= 0 && col < L;
+                    tc::cp_async4(&cvring[s * 128 + 32 * k + lane],
+                                  a.cdw.p + (long long)bh * a.cdw.s + (in ? col : 0), in);
+                    if (MODE == WSUM)
+                        tc::cp_async4(&wring[s * 128 + 32 * k + lane],
+                                      a.w.p + (long long)bh * a.w.s + (in ? col : 0), in);
+                }
+                tc::cp_async_arrive(bar + B_FULL + s);
+            }
+        }
+        asm volatile("cp.async.wait_all;" ::: "memory");  // nothing in flight at exit
+        if (lane == 0 && *abort_flag) {  // let issued loads land before teardown
+            for (int x = max(0, a_issued - 2); x < a_issued; ++x)
+                tc::mbar_wait(bar + B_AFULL + (x & 1), (x >> 1) & 1, kWaitBudget);
+            for (int x = max(0, issued - NRING); x < issued; ++x)
+                tc::mbar_wait(bar + B_FULL + x % NRING, (x / NRING) & 1, kWaitBudget);
+        }
+        __syncwarp();
+    } else if (warp == W_MMA) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            const uint32_t id_s = tc::idesc_bf16(128, 128, false, false);
+            const uint64_t dA0 = tc::sdesc_sw128(tc::smem_u32(sm + OFF_A), 16, 1024);
+            const uint64_t dK0 = tc::sdesc_sw128(tc::smem_u32(sm + OFF_K), 16, 1024);
+            ChunkIds ids;
+            int g = 0, pbh = -1, prb = -1;
+            bool ok = true;
+            Cursor cur = cur0;
+            for (int it = 0; ok && it < ntl; ++it) {
+                const int bh = cur.b * H + cur.h;
+                const bool succ = reuse && bh == pbh && cur.rb == prb + 1;
+                pbh = bh;
+                prb = cur.rb;
+                ids.advance(succ, nch);
+                Cursor nx = cur;
+                nx.next(nblk, H);
+                const bool next_succ = reuse && it + 1 < ntl && nx.b * H + nx.h == bh && nx.rb == cur.rb + 1;
+                if (!ctl.wait(B_AFULL + (it & 1), (it >> 1) & 1)) { ok = false; break; }
+                const uint64_t dA = tc::sdesc_add(dA0, (it & 1) * TILE);
+                for (int c = 0; c < nch; ++c, ++g) {
+                    const int id = ids.base + c, s = id % NRING, b = g & 3;
+                    if (!ctl.wait(B_FULL + s, (id / NRING) & 1)) { ok = false; break; }
+                    if (g >= 4 && !ctl.wait(B_SEMPTY + b, ((g >> 2) - 1) & 1)) { ok = false; break; }
+                    tc::tc_fence_after();
+                    const uint64_t dB = tc::sdesc_add(dK0, s * TILE);
+#pragma unroll
+                    for (int k = 0; k < 4; ++k)
+                        tc::mma_bf16(tS + 128 * b, tc::sdesc_add(dA, 32 * k), tc::sdesc_add(dB, 32 * k),
+                                     id_s, k > 0);
+                    tc::tc_commit(bar + B_SFULL + b);
+                    if (!next_succ || c == 0) tc::tc_commit(bar + B_EMPTY + s);  // its last reader
+                }
+                if (!ok) break;
+                tc::tc_commit(bar + B_AEMPTY + (it & 1));
+                cur = nx;
+            }
+            tc::tc_commit(bar + B_DRAIN);
+            tc::mbar_wait(bar + B_DRAIN, 0, kWaitBudget);
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------------ epilogue
+        const int qd = warp & 3, pt = warp >> 2;
+        const uint32_t lanebase = (uint32_t)(qd * 32) << 16;
+        float* scr = reinterpret_cast<float*>(sm + OFF_SCR) + warp * 128;
+        const float c2 = a.c2;
+        ChunkIds ids;
+        int g = 0, pbh = -1, prb = -1;
+        bool ok = true;
+        Cursor cur = cur0;
+        for (int it = 0; ok && it < ntl; ++it) {
+            const int bh = cur.b * H + cur.h, r0 = cur.rb * 128;
+            const bool succ = reuse && bh == pbh && cur.rb == prb + 1;
+            pbh = bh;
+            prb = cur.rb;
+            ids.advance(succ, nch);
+            Cursor nx = cur;
+            nx.next(nblk, H);
+            const bool next_succ = reuse && it + 1 < ntl && nx.b * H + nx.h == bh && nx.rb == cur.rb + 1;
+            // this thread's row and the warp's shift (the smallest working dual of
+            // the quadrant's valid rows; per-row shifts past a spread of 64)
+            const int rw0 = r0 + qd * 32, r = rw0 + lane;
+            if (!ctl.wait(B_RFULL + it % NRI, (it / NRI) & 1)) { ok = false; break; }
+            const RowInfo& ri = rinfo[it % NRI];
+            const float rwv = ri.rw[qd * 32 + lane];
+            const bool valid = r < L && rwv != -INFINITY;
+            const float sr = valid ? rwv : 0.f;
+            const float bb = MODE == WSUM ? ri.base[qd * 32 + lane] : 0.f;
+            const float mu = (MODE == WSUM && a.mult.p) ? ri.mult[qd * 32 + lane] : 1.f;  // none: 1
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(bar + B_REMPTY + it % NRI);
+            float mn = valid ? sr : INFINITY, mx = valid ? sr : -INFINITY;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+            }
+            const float sq = mn == INFINITY ? 0.f : mn;
+            const bool fb = mn != INFINITY && mx - mn > kFallbackSpread;
+            const float seff = (fb && valid) ? sr : sq;  // this row's shift
+            const float delta = seff - sq;
+            uint64_t acc[4] = {0, 0, 0, 0};
+            for (int c = 0; c < nch; ++c, ++g) {
+                if ((g & 3) != pt) continue;
+                const int id = ids.base + c, s = id % NRING;
+                if (!ctl.wait(B_SFULL + pt, (g >> 2) & 1)) { ok = false; break; }
+                if (!ctl.wait(B_FULL + s, (id / NRING) & 1)) { ok = false; break; }
+                tc::tc_fence_after();
+                const int col0 = r0 - W + 128 * c;
+                // this warp's copy of the chunk's column duals with its shift added
+#pragma unroll
+                for (int k = 0; k < 4; ++k) scr[32 * k + lane] = cvring[s * 128 + 32 * k + lane] + sq;
+                __syncwarp();
+                const float* wv = wring + s * 128;
+#pragma unroll 1
+                for (int gr = 0; gr < 4; ++gr) {
+                    const int cg = col0 + 32 * gr;
+                    const bool all_out = (cg + 31 < rw0 - W) || (cg > rw0 + 31 + W) || cg + 31 < 0 || cg >= L;
+                    if (all_out) continue;
+                    const bool all_in = (cg >= rw0 + 31 - W) && (cg + 31 <= rw0 + W) && cg >= 0 && cg + 31 < L;
+                    uint32_t u[32];
+                    tc::tmem_ld32(tS + 128 * pt + lanebase + 32 * gr, u);
+                    tc::tmem_wait_ld();
+                    const float* cs = scr + 32 * gr;
+                    const float* ws = wv + 32 * gr;
+                    if (fb) {
+                        if (all_in) group<MODE, KP, false, true>(u, cs, ws, c2, delta, r - cg, W, cg, L, acc);
+                        else group<MODE, KP, true, true>(u, cs, ws, c2, delta, r - cg, W, cg, L, acc);
+                    } else {
+                        if (all_in) group<MODE, KP, false, false>(u, cs, ws, c2, 0.f, r - cg, W, cg, L, acc);
+                        else group<MODE, KP, true, false>(u, cs, ws, c2, 0.f, r - cg, W, cg, L, acc);
+                    }
+                }
+                // every TMEM read and shared-memory read of the chunk is done
+                tc::tc_fence_before();
+                __syncwarp();
+                if (lane == 0) {
+                    tc::mbar_arrive(bar + B_SEMPTY + pt);
+                    if (!next_succ || c == 0) tc::mbar_arrive(bar + B_EMPTY + s);
+                }
+            }
+            if (!ok) break;
+            // ---------------------------------------------------------- end of tile
+            float a0, a1, a2, a3, a4, a5, a6, a7;
+            tc::upk2(acc[0], a0, a1);
+            tc::upk2(acc[1], a2, a3);
+            tc::upk2(acc[2], a4, a5);
+            tc::upk2(acc[3], a6, a7);
+            const int slot = it % NRED;
+            float* rs = red + slot * 512;
+            rs[pt * 128 + qd * 32 + lane] = ((a0 + a1) + (a2 + a3)) + ((a4 + a5) + (a6 + a7));
+            __syncwarp();
+            __threadfence_block();
+            int old = 0;
+            if (lane == 0) old = atomicAdd(cnt + slot * 4 + qd, 1);
+            old = __shfl_sync(0xffffffffu, old, 0);
+            if ((old & 3) == 3) {  // the last of the quadrant's four parts: write its rows
+                __threadfence_block();
+                const float tot = (rs[qd * 32 + lane] + rs[128 + qd * 32 + lane]) +
+                                  (rs[256 + qd * 32 + lane] + rs[384 + qd * 32 + lane]);
+                if (r < L) {
+                    float out = 0.f, outw = -INFINITY;
+                    if (valid) {
+                        if (MODE == LSE) {
+                            outw = seff - lg2(tot);
+                            out = outw * kLn2;
+                        } else {
+                            out = bb + a.sgn * mu * (tot * ex2(sr - seff));
+                        }
+                    }
+                    a.out_vec.at(bh, r) = out;
+                    if (MODE == LSE && a.outw.p) a.outw.at(bh, r) = outw;
+                }
+            }
+            cur = nx;
+        }
+    }
+
+    tc::tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc::tc_fence_after();
+        tc::tmem_dealloc(tS, 512);
+    }
+}
+
+}  // namespace tcr
+}  // namespace sa

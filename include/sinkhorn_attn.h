@@ -346,6 +346,17 @@ sa_status sinkhorn_attn_bias_certificate(int n_depths, const int* depths, int n_
                                          const double* sums, double tau, double* eta,
                                          int* r_star);
 
+/* Test hook for the exponentials of the row-sum sweeps (the dual updates and
+ * the vector-cotangent sweeps); no counterpart in the pages.  For each of the
+ * n float32 arguments x (x <= 0; device, 4-byte aligned) it writes 2^x as those
+ * sweeps evaluate it on the FMA pipe (y_poly: round-to-nearest range
+ * reduction and a degree-5 polynomial, arguments clamped at -126) and on the
+ * MUFU unit (y_mufu: ex2.approx).  Returns SA_ERR_INVALID_ARG for n < 0 or a
+ * pointer that is not device memory of the current device, SA_ERR_CUDA on a
+ * launch error, else SA_OK. */
+sa_status sinkhorn_attn_debug_exp2(const float* x, long long n, float* y_poly, float* y_mufu,
+                                   void* stream);
+
 /* Test hook for the failure path; no counterpart in the pages.  Launches on
  * `stream` one CTA whose thread waits, through the same bounded mbarrier wait
  * every kernel of this library uses, on a barrier that nothing ever arrives on;
