@@ -562,7 +562,7 @@ int sm_count() {
 // Exponentials of every 32 entries of a row-sum sweep's in-band group that run
 // on the FMA pipe (the rest on the MUFU unit).
 #ifndef SA_ROWSUM_KP
-#define SA_ROWSUM_KP 8
+#define SA_ROWSUM_KP 0
 #endif
 
 // The row-sum sweeps (shifted LSE, WSUM) on the tensor cores: persistent, one

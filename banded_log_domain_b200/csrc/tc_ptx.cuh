@@ -158,6 +158,18 @@ __device__ __forceinline__ void fence_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// One lane of the (converged) warp, the same one for the same mask: the
+// issuing thread of a tcgen05 operation.  The code around it stays
+// warp-uniform, which keeps descriptors and addresses in uniform registers;
+// an MMA loop run by lane 0 alone issues each MMA 1.5-2x slower (measured).
+__device__ __forceinline__ bool elect_one() {
+    uint32_t pred = 0;
+    asm volatile("{\n\t.reg .pred P;\n\telect.sync _|P, %1;\n\tselp.u32 %0, 1, 0, P;\n\t}"
+                 : "=r"(pred)
+                 : "r"(0xffffffffu));
+    return pred != 0;
+}
+
 // ---------------------------------------------------------------- descriptors
 // Shared-memory matrix descriptor, 128-byte swizzle (tile base 1024-byte
 // aligned): start address, leading and stride byte offsets (16-byte units),

@@ -161,54 +161,53 @@ __device__ __forceinline__ void exp2_poly2(float x0, float x1, float& e0, float&
     e1 = __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23));
 }
 
-// One warp's 32 rows x 32 columns: arguments x_j = c2 s_j + cs_j (+ delta), the
-// exponentials (KP of them on the FMA pipe when the group is inside the band),
-// and their sum into acc (LSE) or their w-weighted sum (WSUM).
+// One warp's 32 rows x 32 columns, staged: all arguments, then all
+// exponentials, then the sums.  EDGE keeps only local columns lo..hi.
 template <int MODE, int KP, bool EDGE, bool FB>
 __device__ __forceinline__ void group(const uint32_t (&u)[32], const float* cs, const float* wv,
-                                      float c2, float delta, int d_first, int W, int cg, int L,
-                                      uint64_t (&acc)[4]) {
+                                      float c2, float delta, int lo, int hi, uint64_t (&acc)[4]) {
     const uint64_t c2p = tc::pk2(c2, c2), dp = tc::pk2(delta, delta);
     const float4* c4 = reinterpret_cast<const float4*>(cs);
-    const float4* w4 = reinterpret_cast<const float4*>(wv);
+    uint64_t xp[16];
 #pragma unroll
     for (int q = 0; q < 8; ++q) {
         const float4 cv = c4[q];
-        uint64_t a01 = tc::fma2(tc::pk2(__uint_as_float(u[4 * q]), __uint_as_float(u[4 * q + 1])), c2p,
-                                tc::pk2(cv.x, cv.y));
-        uint64_t a23 = tc::fma2(tc::pk2(__uint_as_float(u[4 * q + 2]), __uint_as_float(u[4 * q + 3])), c2p,
-                                tc::pk2(cv.z, cv.w));
+        xp[2 * q] = tc::fma2(tc::pk2(__uint_as_float(u[4 * q]), __uint_as_float(u[4 * q + 1])), c2p,
+                             tc::pk2(cv.x, cv.y));
+        xp[2 * q + 1] = tc::fma2(tc::pk2(__uint_as_float(u[4 * q + 2]), __uint_as_float(u[4 * q + 3])), c2p,
+                                 tc::pk2(cv.z, cv.w));
         if (FB) {
-            a01 = tc::add2(a01, dp);
-            a23 = tc::add2(a23, dp);
+            xp[2 * q] = tc::add2(xp[2 * q], dp);
+            xp[2 * q + 1] = tc::add2(xp[2 * q + 1], dp);
         }
-        float x[4];
-        tc::upk2(a01, x[0], x[1]);
-        tc::upk2(a23, x[2], x[3]);
+    }
+    float e[32];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+        float x0, x1;
+        tc::upk2(xp[j], x0, x1);
         if (EDGE) {
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int d = d_first - (4 * q + e);  // row - column
-                const int col = cg + 4 * q + e;
-                if ((unsigned)(d + W) > (unsigned)(2 * W) || (unsigned)col >= (unsigned)L) x[e] = -INFINITY;
-            }
+            if ((unsigned)(2 * j - lo) > (unsigned)(hi - lo)) x0 = -INFINITY;
+            if ((unsigned)(2 * j + 1 - lo) > (unsigned)(hi - lo)) x1 = -INFINITY;
         }
-        float e[4];
-        if (!EDGE && 4 * q + 4 > 32 - KP) {
-            exp2_poly2(x[0], x[1], e[0], e[1]);
-            exp2_poly2(x[2], x[3], e[2], e[3]);
+        if (!EDGE && 2 * j + 2 > 32 - KP) {
+            exp2_poly2(x0, x1, e[2 * j], e[2 * j + 1]);
         } else {
-#pragma unroll
-            for (int k = 0; k < 4; ++k) e[k] = ex2(x[k]);
+            e[2 * j] = ex2(x0);
+            e[2 * j + 1] = ex2(x1);
         }
-        if (MODE == WSUM) {
+    }
+    if (MODE == WSUM) {
+        const float4* w4 = reinterpret_cast<const float4*>(wv);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
             const float4 w = w4[q];
-            acc[(2 * q) & 3] = tc::fma2(tc::pk2(e[0], e[1]), tc::pk2(w.x, w.y), acc[(2 * q) & 3]);
-            acc[(2 * q + 1) & 3] = tc::fma2(tc::pk2(e[2], e[3]), tc::pk2(w.z, w.w), acc[(2 * q + 1) & 3]);
-        } else {
-            acc[(2 * q) & 3] = tc::add2(acc[(2 * q) & 3], tc::pk2(e[0], e[1]));
-            acc[(2 * q + 1) & 3] = tc::add2(acc[(2 * q + 1) & 3], tc::pk2(e[2], e[3]));
+            acc[(2 * q) & 3] = tc::fma2(tc::pk2(e[4 * q], e[4 * q + 1]), tc::pk2(w.x, w.y), acc[(2 * q) & 3]);
+            acc[(2 * q + 1) & 3] = tc::fma2(tc::pk2(e[4 * q + 2], e[4 * q + 3]), tc::pk2(w.z, w.w), acc[(2 * q + 1) & 3]);
         }
+    } else {
+#pragma unroll
+        for (int j = 0; j < 16; ++j) acc[j & 3] = tc::add2(acc[j & 3], tc::pk2(e[2 * j], e[2 * j + 1]));
     }
 }
 
@@ -350,31 +349,33 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_rowsum_sweep(const SweepArgs a
         __syncwarp();
     } else if (warp == W_MMA) {
         // ------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
-            const uint32_t id_s = tc::idesc_bf16(128, 128, false, false);
-            const uint64_t dA0 = tc::sdesc_sw128(tc::smem_u32(sm + OFF_A), 16, 1024);
-            const uint64_t dK0 = tc::sdesc_sw128(tc::smem_u32(sm + OFF_K), 16, 1024);
-            ChunkIds ids;
-            int g = 0, pbh = -1, prb = -1;
-            bool ok = true;
-            Cursor cur = cur0;
-            for (int it = 0; ok && it < ntl; ++it) {
-                const int bh = cur.b * H + cur.h;
-                const bool succ = reuse && bh == pbh && cur.rb == prb + 1;
-                pbh = bh;
-                prb = cur.rb;
-                ids.advance(succ, nch);
-                Cursor nx = cur;
-                nx.next(nblk, H);
-                const bool next_succ = reuse && it + 1 < ntl && nx.b * H + nx.h == bh && nx.rb == cur.rb + 1;
-                if (!ctl.wait(B_AFULL + (it & 1), (it >> 1) & 1)) { ok = false; break; }
-                const uint64_t dA = tc::sdesc_add(dA0, (it & 1) * TILE);
-                for (int c = 0; c < nch; ++c, ++g) {
-                    const int id = ids.base + c, s = id % NRING, b = g & 3;
-                    if (!ctl.wait(B_FULL + s, (id / NRING) & 1)) { ok = false; break; }
-                    if (g >= 4 && !ctl.wait(B_SEMPTY + b, ((g >> 2) - 1) & 1)) { ok = false; break; }
-                    tc::tc_fence_after();
-                    const uint64_t dB = tc::sdesc_add(dK0, s * TILE);
+        // The whole warp runs the loop (uniform control flow and values); one
+        // elected lane issues the MMAs and commits.
+        const uint32_t id_s = tc::idesc_bf16(128, 128, false, false);
+        const uint64_t dA0 = tc::sdesc_sw128(tc::smem_u32(sm + OFF_A), 16, 1024);
+        const uint64_t dK0 = tc::sdesc_sw128(tc::smem_u32(sm + OFF_K), 16, 1024);
+        ChunkIds ids;
+        int g = 0, pbh = -1, prb = -1;
+        bool ok = true;
+        Cursor cur = cur0;
+        for (int it = 0; ok && it < ntl; ++it) {
+            const int bh = cur.b * H + cur.h;
+            const bool succ = reuse && bh == pbh && cur.rb == prb + 1;
+            pbh = bh;
+            prb = cur.rb;
+            ids.advance(succ, nch);
+            Cursor nx = cur;
+            nx.next(nblk, H);
+            const bool next_succ = reuse && it + 1 < ntl && nx.b * H + nx.h == bh && nx.rb == cur.rb + 1;
+            if (!ctl.wait(B_AFULL + (it & 1), (it >> 1) & 1)) { ok = false; break; }
+            const uint64_t dA = tc::sdesc_add(dA0, (it & 1) * TILE);
+            for (int c = 0; c < nch; ++c, ++g) {
+                const int id = ids.base + c, s = id % NRING, b = g & 3;
+                if (!ctl.wait(B_FULL + s, (id / NRING) & 1)) { ok = false; break; }
+                if (g >= 4 && !ctl.wait(B_SEMPTY + b, ((g >> 2) - 1) & 1)) { ok = false; break; }
+                tc::tc_fence_after();
+                const uint64_t dB = tc::sdesc_add(dK0, s * TILE);
+                if (tc::elect_one()) {
 #pragma unroll
                     for (int k = 0; k < 4; ++k)
                         tc::mma_bf16(tS + 128 * b, tc::sdesc_add(dA, 32 * k), tc::sdesc_add(dB, 32 * k),
@@ -382,14 +383,16 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_rowsum_sweep(const SweepArgs a
                     tc::tc_commit(bar + B_SFULL + b);
                     if (!next_succ || c == 0) tc::tc_commit(bar + B_EMPTY + s);  // its last reader
                 }
-                if (!ok) break;
-                tc::tc_commit(bar + B_AEMPTY + (it & 1));
-                cur = nx;
+                __syncwarp();
             }
-            tc::tc_commit(bar + B_DRAIN);
-            tc::mbar_wait(bar + B_DRAIN, 0, kWaitBudget);
+            if (!ok) break;
+            if (tc::elect_one()) tc::tc_commit(bar + B_AEMPTY + (it & 1));
+            __syncwarp();
+            cur = nx;
         }
+        if (tc::elect_one()) tc::tc_commit(bar + B_DRAIN);
         __syncwarp();
+        tc::mbar_wait(bar + B_DRAIN, 0, kWaitBudget);
     } else {
         // ------------------------------------------------------------ epilogue
         const int qd = warp & 3, pt = warp >> 2;
@@ -455,12 +458,14 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_rowsum_sweep(const SweepArgs a
                     tc::tmem_wait_ld();
                     const float* cs = scr + 32 * gr;
                     const float* ws = wv + 32 * gr;
+                    // this row's band and [0, L), as local columns of the group
+                    const int lo = max(r - W, 0) - cg, hi = min(r + W, L - 1) - cg;
                     if (fb) {
-                        if (all_in) group<MODE, KP, false, true>(u, cs, ws, c2, delta, r - cg, W, cg, L, acc);
-                        else group<MODE, KP, true, true>(u, cs, ws, c2, delta, r - cg, W, cg, L, acc);
+                        if (all_in) group<MODE, KP, false, true>(u, cs, ws, c2, delta, lo, hi, acc);
+                        else group<MODE, KP, true, true>(u, cs, ws, c2, delta, lo, hi, acc);
                     } else {
-                        if (all_in) group<MODE, KP, false, false>(u, cs, ws, c2, 0.f, r - cg, W, cg, L, acc);
-                        else group<MODE, KP, true, false>(u, cs, ws, c2, 0.f, r - cg, W, cg, L, acc);
+                        if (all_in) group<MODE, KP, false, false>(u, cs, ws, c2, 0.f, lo, hi, acc);
+                        else group<MODE, KP, true, false>(u, cs, ws, c2, 0.f, lo, hi, acc);
                     }
                 }
                 // every TMEM read and shared-memory read of the chunk is done

@@ -343,7 +343,9 @@ __global__ void __launch_bounds__(nthreads(MODE), ctas_per_sm(MODE)) tc_band_swe
         __syncwarp();
     } else if (warp == W_MMA) {
         // ------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
+        // The whole warp runs the loop (uniform control flow and values); one
+        // elected lane issues the MMAs and commits.
+        {
             const uint32_t id_s = tc::idesc_bf16(128, 128, false, false);
             const uint32_t id_o = tc::idesc_bf16(128, 64, false, true);
             // descriptors built once; offsets are added in 16-byte units
@@ -362,14 +364,17 @@ __global__ void __launch_bounds__(nthreads(MODE), ctas_per_sm(MODE)) tc_band_swe
                 tc::tc_fence_after();
                 const uint64_t dX = tc::sdesc_add(dStMN, s * stage_bytes(MODE) + (MODE == PV ? TILE : 0));
                 const uint64_t dPb = tc::sdesc_add(dP, pb * 2 * TILE);
+                if (tc::elect_one()) {
 #pragma unroll
-                for (int k = 0; k < 8; ++k) {
-                    tc::mma_bf16(tO + 64 * ob, tc::sdesc_add(dPb, (k >> 2) * TILE + (k & 3) * 32),
-                                 tc::sdesc_add(dX, k * 2048), id_o, (c > 0 || k > 0) ? 1u : 0u);
+                    for (int k = 0; k < 8; ++k) {
+                        tc::mma_bf16(tO + 64 * ob, tc::sdesc_add(dPb, (k >> 2) * TILE + (k & 3) * 32),
+                                     tc::sdesc_add(dX, k * 2048), id_o, (c > 0 || k > 0) ? 1u : 0u);
+                    }
+                    tc::tc_commit(bar + B_PEMPTY + pb);
+                    tc::tc_commit(bar + B_EMPTY + s);
+                    if (c == nch - 1) tc::tc_commit(bar + B_OFULL + ob);
                 }
-                tc::tc_commit(bar + B_PEMPTY + pb);
-                tc::tc_commit(bar + B_EMPTY + s);
-                if (c == nch - 1) tc::tc_commit(bar + B_OFULL + ob);
+                __syncwarp();
                 return true;
             };
             bool ok = true;
@@ -387,31 +392,36 @@ __global__ void __launch_bounds__(nthreads(MODE), ctas_per_sm(MODE)) tc_band_swe
                     if (gc >= NSB && !ctl.wait(B_SEMPTY + b, ((gc / NSB) - 1) & 1)) { ok = false; break; }
                     tc::tc_fence_after();
                     const uint64_t dB = tc::sdesc_add(dStK, s * stage_bytes(MODE));
-#pragma unroll
-                    for (int k = 0; k < 4; ++k)
-                        tc::mma_bf16(tS + 128 * b, tc::sdesc_add(dA, 32 * k), tc::sdesc_add(dB, 32 * k),
-                                     id_s, k > 0);
-                    if (DS) {
+                    if (tc::elect_one()) {
 #pragma unroll
                         for (int k = 0; k < 4; ++k)
-                            tc::mma_bf16(tG, tc::sdesc_add(dA2, 32 * k), tc::sdesc_add(dB, TILE + 32 * k),
+                            tc::mma_bf16(tS + 128 * b, tc::sdesc_add(dA, 32 * k), tc::sdesc_add(dB, 32 * k),
                                          id_s, k > 0);
-                        if (AUG)  // + the modifier, one more K16 step
-                            tc::mma_bf16(tG, dAug, tc::sdesc_add(dAug, AUG_BYTES * (1 + s)), id_s, 1u);
+                        if (DS) {
+#pragma unroll
+                            for (int k = 0; k < 4; ++k)
+                                tc::mma_bf16(tG, tc::sdesc_add(dA2, 32 * k), tc::sdesc_add(dB, TILE + 32 * k),
+                                             id_s, k > 0);
+                            if (AUG)  // + the modifier, one more K16 step
+                                tc::mma_bf16(tG, dAug, tc::sdesc_add(dAug, AUG_BYTES * (1 + s)), id_s, 1u);
+                        }
+                        tc::tc_commit(bar + B_SFULL + b);
+                        if (!HASX) tc::tc_commit(bar + B_EMPTY + s);
                     }
-                    tc::tc_commit(bar + B_SFULL + b);
-                    if (!HASX) tc::tc_commit(bar + B_EMPTY + s);
+                    __syncwarp();
                     if (HASX) {
                         if (pg >= 0 && !issue_pv(pg, pit, pc, pn)) { ok = false; break; }
                         pg = gc; pit = it; pc = c; pn = tl.nch;
                     }
                 }
                 if (!ok) break;
-                tc::tc_commit(bar + B_AEMPTY + ab);  // every score MMA of the tile has read A
+                if (tc::elect_one()) tc::tc_commit(bar + B_AEMPTY + ab);  // every score MMA of the tile has read A
+                __syncwarp();
             }
             if (HASX && ok && pg >= 0) ok = issue_pv(pg, pit, pc, pn);
             // drain: every MMA issued above has completed once this arrives
-            tc::tc_commit(bar + B_DRAIN);
+            if (tc::elect_one()) tc::tc_commit(bar + B_DRAIN);
+            __syncwarp();
             tc::mbar_wait(bar + B_DRAIN, 0, kWaitBudget);
         }
         __syncwarp();
