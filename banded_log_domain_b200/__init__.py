@@ -17,13 +17,17 @@ import torch
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libsinkhorn_attn.so")
+# the same library built with device-side bounds checks (-DSA_DEBUG)
+DEBUG_LIB_PATH = os.path.join(_PKG, "libsinkhorn_attn_debug.so")
+if os.environ.get("SINKHORN_ATTN_DEBUG_LIB") == "1":
+    LIB_PATH = DEBUG_LIB_PATH
 
 SA_OK = 0
 SA_F32, SA_BF16 = 0, 1
 SA_BWD_ONE_REFERENCE, SA_BWD_DIRECT = 0, 1
 _STATUS = {0: "SA_OK", -1: "SA_ERR_INVALID_ARG", -2: "SA_ERR_UNSUPPORTED",
            -3: "SA_ERR_WORKSPACE", -4: "SA_ERR_CUDA", -5: "SA_ERR_NONFINITE",
-           -6: "SA_ERR_TIMEOUT", -7: "SA_ERR_EXCHANGE"}
+           -6: "SA_ERR_TIMEOUT", -7: "SA_ERR_EXCHANGE", -8: "SA_ERR_BOUNDS"}
 SCHEDULES = {"one_reference": SA_BWD_ONE_REFERENCE, "direct": SA_BWD_DIRECT}
 
 

@@ -32,21 +32,26 @@ def deps():
             glob.glob(os.path.join(ROOT, "include", "*.h")))
 
 
-def stale() -> bool:
-    if not os.path.exists(LIB):
+DEBUG_LIB = os.path.join(PKG, "libsinkhorn_attn_debug.so")
+
+
+def stale_lib(lib: str) -> bool:
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return any(os.path.getmtime(f) > t for f in deps())
 
 
 def build(force: bool = False, verbose: bool = False) -> str:
-    if force or stale():
-        tmp = LIB + f".tmp{os.getpid()}"
-        cmd = [NVCC, *FLAGS, "-o", tmp, *sources()]
-        if verbose:
-            print(" ".join(cmd), flush=True)
-        subprocess.check_call(cmd)
-        os.replace(tmp, LIB)
+    """Builds the library and its bounds-checked debug twin (-DSA_DEBUG)."""
+    for lib, extra in ((LIB, []), (DEBUG_LIB, ["-DSA_DEBUG"])):
+        if force or stale_lib(lib):
+            tmp = lib + f".tmp{os.getpid()}"
+            cmd = [NVCC, *FLAGS, *extra, "-o", tmp, *sources()]
+            if verbose:
+                print(" ".join(cmd), flush=True)
+            subprocess.check_call(cmd)
+            os.replace(tmp, lib)
     return LIB
 
 

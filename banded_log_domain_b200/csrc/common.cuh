@@ -7,6 +7,20 @@
 
 namespace sa {
 
+// Debug builds (-DSA_DEBUG): device-side bounds checks.  A failed check
+// records SA_ERR_BOUNDS in the status word (the first one wins) and the
+// access it guards is skipped: the kernel never traps.  In the normal build the
+// checks compile to nothing.
+#ifdef SA_DEBUG
+__device__ __forceinline__ bool debug_bounds(bool ok, int* status) {
+    if (!ok && status) atomicCAS(status, 0, -8 /* SA_ERR_BOUNDS */);
+    return ok;
+}
+#define SA_BOUNDS(cond, status) ::sa::debug_bounds((cond), (status))
+#else
+#define SA_BOUNDS(cond, status) true
+#endif
+
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 

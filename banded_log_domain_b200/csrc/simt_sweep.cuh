@@ -84,6 +84,7 @@ struct SweepArgs {
     // Row-sum sweeps on tensor cores (shifted LSE, WSUM): the duals as working
     // copies, log2(e) times the dual on valid tokens and -inf on masked ones
     // ([BH][L], stride s), which the loader copies to shared memory as they are
+    int* status;            // the workspace's status word (debug bounds checks)
     Vec cdw;                // column side
     Vec rdw;                // row side (LSE: the shift source; WSUM: the row dual)
     MVec outw;              // LSE: the new dual's working copy (or p null)
@@ -425,7 +426,7 @@ __global__ void __launch_bounds__(NT) band_sweep(const SweepArgs a) {
                 const float s2 = __shfl_xor_sync(0xffffffffu, s[i], o);
                 lse_merge(m[i], s[i], m2, s2);
             }
-            if (tx == 0 && rr[i] < L)
+            if (tx == 0 && rr[i] < L && SA_BOUNDS(rr[i] >= 0 && bh < (int)gridDim.y, a.status))
                 a.out_vec.at(bh, rr[i]) = rv_ok[i] ? -(m[i] + lg2(s[i])) * kLn2 : 0.f;
         }
     } else if (MODE == WSUM) {
@@ -434,7 +435,7 @@ __global__ void __launch_bounds__(NT) band_sweep(const SweepArgs a) {
             if (a.dustbin && tx == 0 && rv_ok[i]) s[i] += ex2(a.sd2 + rd2[i] + ce_d) * a.w.at(bh, L);
 #pragma unroll
             for (int o = 8; o > 0; o >>= 1) s[i] += __shfl_xor_sync(0xffffffffu, s[i], o);
-            if (tx == 0 && rr[i] < L) {
+            if (tx == 0 && rr[i] < L && SA_BOUNDS(rr[i] >= 0 && bh < (int)gridDim.y, a.status)) {
                 float v = 0.f;
                 if (rv_ok[i]) {
                     const float b = a.base.p ? a.base.at(bh, rr[i]) : 0.f;
@@ -465,7 +466,7 @@ __global__ void __launch_bounds__(NT) band_sweep(const SweepArgs a) {
             float o4[4];
 #pragma unroll
             for (int j = 0; j < 4; ++j) o4[j] = rv_ok[i] ? oacc[i][j] * scale : 0.f;
-            if (r < L) {
+            if (r < L && SA_BOUNDS(r >= 0 && bh < (int)gridDim.y && tx * 4 + 4 <= D, a.status)) {
                 float* accr = (DS && a.acc) ? a.acc + off + (size_t)r * D + tx * 4 : nullptr;
                 if (DS && accr && a.acc_in) {
                     const float4 p = *reinterpret_cast<const float4*>(accr);

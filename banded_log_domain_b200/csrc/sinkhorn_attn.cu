@@ -692,6 +692,7 @@ simt::SweepArgs base_args(const Ctx& x) {
     a.sd2 = x.p->dustbin ? x.p->dustbin_score * kLog2e : 0.f;
     a.sgn = 1.f;
     a.out_scale = x.c;
+    a.status = x.status;
     return a;
 }
 
@@ -1637,6 +1638,7 @@ const char* sinkhorn_attn_strerror(sa_status s) {
         case SA_ERR_NONFINITE: return "non-finite value in duals or outputs";
         case SA_ERR_TIMEOUT: return "bounded device wait gave up";
         case SA_ERR_EXCHANGE: return "halo exchange callback failed (sequence-sharded call)";
+        case SA_ERR_BOUNDS: return "device-side bounds check failed (debug build)";
     }
     return "unknown status";
 }

@@ -14,12 +14,16 @@
 // c < nch = ceil((2W + 128) / 128), on one grid for the whole problem, so that
 // the next row block of the same problem needs only one new chunk: the K-side
 // chunks (TMA tiles with their column duals) sit in a ring of NRING slots and
-// a chunk stays until the last tile that reads it has (reuse; streaming when
-// W is so large that a tile's chunks do not fit the ring).  Scores go to one
-// of four TMEM buffers (chunk g of the range in buffer g % 4), and epilogue
-// warp (quadrant q, part p) processes the 32 rows of quadrant q of every chunk
-// g with g % 4 == p: a whole 128-column chunk per warp, so the MMA runs up to
-// four chunks ahead.  The four parts' partial row sums of a tile meet in
+// a chunk stays until every tile that reads it has (reuse; streaming when W is
+// so large that a tile's chunks do not fit the ring).  A slot's EMPTY barrier
+// expects 4 arrivals (one per quadrant warp) from each of up to nch uses and
+// one MMA commit at the last use; the loader, which knows how many tiles of its
+// range will read a chunk, arrives for the uses that will not happen.  Scores go to one
+// of four TMEM buffers, one per epilogue part: epilogue warp (quadrant q,
+// part p) processes the 32 rows of quadrant q of the chunks assigned to part
+// p, from buffer p: a whole 128-column chunk per warp, so the MMA runs up to
+// four chunks ahead; the assignment rotates the band-edge chunks over the
+// parts.  The four parts' partial row sums of a tile meet in
 // shared memory; the last part of a quadrant to finish the tile writes its 32
 // outputs (a counter per quadrant, no waiting).
 //
@@ -232,6 +236,12 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_rowsum_sweep(const SweepArgs a
     const int L = a.L, W = a.W, H = a.H;
     const int nblk = (L + 127) / 128, nch = nchunks(W);
     const bool reuse = reuse_ok(W);
+    // Chunk g of tile it goes to part (g + rot * it) % 4.  With nch not a
+    // multiple of 4, g % 4 alone already moves a tile's chunks over the parts
+    // from tile to tile; with nch a multiple of 4 it would give chunk c of every
+    // tile to part c (the band-edge chunks, with fewer groups inside the band,
+    // always to parts 0 and 3), so the tile index is added.
+    const int rot = (nch & 3) == 0 ? 1 : 0;
     const int ntiles = BH * nblk;
     const int t0 = (int)(((long long)blockIdx.x * ntiles) / gridDim.x);
     const int t1 = (int)(((long long)(blockIdx.x + 1) * ntiles) / gridDim.x);
@@ -245,7 +255,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_rowsum_sweep(const SweepArgs a
         }
         for (int s = 0; s < NRING; ++s) {
             tc::mbar_init(bar + B_FULL + s, 33);      // the TMA bytes + 32 column-vector lanes
-            tc::mbar_init(bar + B_EMPTY + s, 1 + 4);  // the last MMA + the 4 quadrant warps
+            tc::mbar_init(bar + B_EMPTY + s, 1 + 4 * nch);  // the last MMA + 4 warps x nch uses
         }
         for (int b = 0; b < 4; ++b) {
             tc::mbar_init(bar + B_SFULL + b, 1);
@@ -287,7 +297,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_rowsum_sweep(const SweepArgs a
             const int first = ids.advance(succ, nch);
             if (lane == 0) {
                 if (it >= 2 && !ctl.wait(B_AEMPTY + (it & 1), ((it >> 1) - 1) & 1)) ok = false;
-                if (ok) {
+                if (ok && SA_BOUNDS(bh < BH && r0 >= 0 && r0 < L, status)) {
                     tc::mbar_expect_tx(bar + B_AFULL + (it & 1), TILE);
                     tc::tma_load_3d(sm + OFF_A + (it & 1) * TILE, &maps.A, bar + B_AFULL + (it & 1), 0,
                                     r0, bh);
@@ -320,9 +330,25 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_rowsum_sweep(const SweepArgs a
                 const int id = ids.base + c, s = id % NRING;
                 if (id >= NRING && !ctl.wait(B_EMPTY + s, ((id / NRING) - 1) & 1)) { ok = false; break; }
                 const int col0 = r0 - W + 128 * c;
-                if (lane == 0) {
+                if (lane == 0 && SA_BOUNDS(s < NRING && col0 >= -W - 128 && col0 < L + W + 128, status)) {
                     tc::mbar_expect_tx(bar + B_FULL + s, TILE);
                     tc::tma_load_3d(sm + OFF_K + s * TILE, &maps.B, bar + B_FULL + s, 0, col0, bh);
+                    // The slot is released once every tile that reads the chunk has
+                    // (each use arrives 4 times, the last use's MMA once): the uses
+                    // are this tile and the successors that follow it, at most c of
+                    // them; the uses that will not happen are arrived for here.
+                    int uses = 1;
+                    if (reuse) {
+                        Cursor ln = cur;
+                        int pb = bh, pr = cur.rb;
+                        for (int k = 1; k <= c && it + k < ntl; ++k) {
+                            ln.next(nblk, H);
+                            if (ln.b * H + ln.h != pb || ln.rb != pr + 1) break;
+                            pr = ln.rb;
+                            ++uses;
+                        }
+                    }
+                    if (uses < nch) tc::mbar_arrive_cnt(bar + B_EMPTY + s, 4 * (nch - uses));
                 }
                 issued = id + 1;
                 // working column duals and WSUM weights; zero off [0, L)
@@ -356,6 +382,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_rowsum_sweep(const SweepArgs a
         const uint64_t dK0 = tc::sdesc_sw128(tc::smem_u32(sm + OFF_K), 16, 1024);
         ChunkIds ids;
         int g = 0, pbh = -1, prb = -1;
+        int nb[4] = {0, 0, 0, 0};  // uses of each TMEM buffer so far
         bool ok = true;
         Cursor cur = cur0;
         for (int it = 0; ok && it < ntl; ++it) {
@@ -370,9 +397,12 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_rowsum_sweep(const SweepArgs a
             if (!ctl.wait(B_AFULL + (it & 1), (it >> 1) & 1)) { ok = false; break; }
             const uint64_t dA = tc::sdesc_add(dA0, (it & 1) * TILE);
             for (int c = 0; c < nch; ++c, ++g) {
-                const int id = ids.base + c, s = id % NRING, b = g & 3;
+                // buffer = the part that processes the chunk (see the epilogue)
+                const int id = ids.base + c, s = id % NRING, b = (g + rot * it) & 3;
+                const int u = b == 0 ? nb[0] : b == 1 ? nb[1] : b == 2 ? nb[2] : nb[3];
                 if (!ctl.wait(B_FULL + s, (id / NRING) & 1)) { ok = false; break; }
-                if (g >= 4 && !ctl.wait(B_SEMPTY + b, ((g >> 2) - 1) & 1)) { ok = false; break; }
+                if (u >= 1 && !ctl.wait(B_SEMPTY + b, (u - 1) & 1)) { ok = false; break; }
+                if (b == 0) ++nb[0]; else if (b == 1) ++nb[1]; else if (b == 2) ++nb[2]; else ++nb[3];
                 tc::tc_fence_after();
                 const uint64_t dB = tc::sdesc_add(dK0, s * TILE);
                 if (tc::elect_one()) {
@@ -401,6 +431,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_rowsum_sweep(const SweepArgs a
         const float c2 = a.c2;
         ChunkIds ids;
         int g = 0, pbh = -1, prb = -1;
+        int nu = 0;  // chunks this part has processed (uses of its TMEM buffer)
         bool ok = true;
         Cursor cur = cur0;
         for (int it = 0; ok && it < ntl; ++it) {
@@ -436,9 +467,13 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_rowsum_sweep(const SweepArgs a
             const float delta = seff - sq;
             uint64_t acc[4] = {0, 0, 0, 0};
             for (int c = 0; c < nch; ++c, ++g) {
-                if ((g & 3) != pt) continue;
-                const int id = ids.base + c, s = id % NRING;
-                if (!ctl.wait(B_SFULL + pt, (g >> 2) & 1)) { ok = false; break; }
+                // chunk g of tile it goes to part (g + rot * it) % 4, in that
+                // part's own TMEM buffer, whose phases its one part consumes in
+                // order
+                if (((g + rot * it) & 3) != pt) continue;
+                const int id = ids.base + c, s = id % NRING, b = pt;
+                if (!ctl.wait(B_SFULL + b, nu & 1)) { ok = false; break; }
+                ++nu;
                 if (!ctl.wait(B_FULL + s, (id / NRING) & 1)) { ok = false; break; }
                 tc::tc_fence_after();
                 const int col0 = r0 - W + 128 * c;
@@ -454,7 +489,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_rowsum_sweep(const SweepArgs a
                     if (all_out) continue;
                     const bool all_in = (cg >= rw0 + 31 - W) && (cg + 31 <= rw0 + W) && cg >= 0 && cg + 31 < L;
                     uint32_t u[32];
-                    tc::tmem_ld32(tS + 128 * pt + lanebase + 32 * gr, u);
+                    if (SA_BOUNDS(128 * b + 32 * gr + 32 <= 512, status))
+                        tc::tmem_ld32(tS + 128 * b + lanebase + 32 * gr, u);
                     tc::tmem_wait_ld();
                     const float* cs = scr + 32 * gr;
                     const float* ws = wv + 32 * gr;
@@ -472,8 +508,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_rowsum_sweep(const SweepArgs a
                 tc::tc_fence_before();
                 __syncwarp();
                 if (lane == 0) {
-                    tc::mbar_arrive(bar + B_SEMPTY + pt);
-                    if (!next_succ || c == 0) tc::mbar_arrive(bar + B_EMPTY + s);
+                    tc::mbar_arrive(bar + B_SEMPTY + b);
+                    tc::mbar_arrive(bar + B_EMPTY + s);  // this use has read the slot
                 }
             }
             if (!ok) break;
@@ -485,7 +521,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_rowsum_sweep(const SweepArgs a
             tc::upk2(acc[3], a6, a7);
             const int slot = it % NRED;
             float* rs = red + slot * 512;
-            rs[pt * 128 + qd * 32 + lane] = ((a0 + a1) + (a2 + a3)) + ((a4 + a5) + (a6 + a7));
+            if (SA_BOUNDS(slot < NRED && pt < 4, status)) rs[pt * 128 + qd * 32 + lane] = ((a0 + a1) + (a2 + a3)) + ((a4 + a5) + (a6 + a7));
             __syncwarp();
             __threadfence_block();
             int old = 0;
@@ -505,8 +541,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_rowsum_sweep(const SweepArgs a
                             out = bb + a.sgn * mu * (tot * ex2(sr - seff));
                         }
                     }
-                    a.out_vec.at(bh, r) = out;
-                    if (MODE == LSE && a.outw.p) a.outw.at(bh, r) = outw;
+                    if (SA_BOUNDS(bh < BH && r >= 0, status)) {
+                        a.out_vec.at(bh, r) = out;
+                        if (MODE == LSE && a.outw.p) a.outw.at(bh, r) = outw;
+                    }
                 }
             }
             cur = nx;

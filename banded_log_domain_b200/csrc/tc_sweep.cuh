@@ -502,7 +502,7 @@ __global__ void __launch_bounds__(nthreads(MODE), ctas_per_sm(MODE)) tc_band_swe
                 for (int q = 0; q < OW / 4; ++q)
                     reinterpret_cast<float4*>(accr)[q] =
                         make_float4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
-            } else if (fr < L) {
+            } else if (fr < L && SA_BOUNDS(fbh < BH && fr >= 0, status)) {
                 __nv_bfloat16* outp =
                     reinterpret_cast<__nv_bfloat16*>(a.out_mat) + ((size_t)fbh * L + fr) * 64 + OW * pt;
 #pragma unroll
@@ -577,7 +577,8 @@ __global__ void __launch_bounds__(nthreads(MODE), ctas_per_sm(MODE)) tc_band_swe
                         for (int j = 0; j < 32; ++j)
                             sv[j] = __uint_as_float(g ? su[(UPFRONT && NG > 1) ? 1 : 0][j] : su[0][j]);
                     } else {
-                        tc::tmem_ld32(tS + 128 * b + lanebase + PW * pt + 32 * g, su[0]);
+                        if (SA_BOUNDS(128 * b + PW * pt + 32 * g + 32 <= tmem_cols(MODE), status))
+                            tc::tmem_ld32(tS + 128 * b + lanebase + PW * pt + 32 * g, su[0]);
                         if (DS) tc::tmem_ld32(tG + lanebase + PW * pt + 32 * g, gu[0]);
                         tc::tmem_wait_ld();
     #pragma unroll
@@ -720,7 +721,8 @@ __global__ void __launch_bounds__(nthreads(MODE), ctas_per_sm(MODE)) tc_band_swe
                             w.y = tc::pack_bf16(pv[8 * q + 2], pv[8 * q + 3]);
                             w.z = tc::pack_bf16(pv[8 * q + 4], pv[8 * q + 5]);
                             w.w = tc::pack_bf16(pv[8 * q + 6], pv[8 * q + 7]);
-                            *reinterpret_cast<uint4*>(dst + tc::sw128_off(lr, ((jc & 63) >> 3) + q)) = w;
+                            if (SA_BOUNDS(pb * 2 * TILE + (jc >> 6) * TILE + (int)tc::sw128_off(lr, ((jc & 63) >> 3) + q) + 16 <= 2 * 2 * TILE, status))
+                                *reinterpret_cast<uint4*>(dst + tc::sw128_off(lr, ((jc & 63) >> 3) + q)) = w;
                         }
                     }
                 }
@@ -783,7 +785,7 @@ __global__ void __launch_bounds__(nthreads(MODE), ctas_per_sm(MODE)) tc_band_swe
                         if (a.dustbin) tot += ex2(a.sd2 + rd2f + ce_d) * a.w.at(bh, L);
                         out = bb + a.sgn * mu * tot;
                     }
-                    a.out_vec.at(bh, r) = rokf ? out : 0.f;
+                    if (SA_BOUNDS(bh < BH && r >= 0, status)) a.out_vec.at(bh, r) = rokf ? out : 0.f;
                 }
             } else if (DS) {
                 pend = true;
@@ -833,7 +835,7 @@ __global__ void __launch_bounds__(nthreads(MODE), ctas_per_sm(MODE)) tc_band_swe
                     for (int q = 0; q < OW / 4; ++q)
                         reinterpret_cast<float4*>(accr)[q] =
                             make_float4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
-                } else if (r < L) {
+                } else if (r < L && SA_BOUNDS(bh < BH && r >= 0, status)) {
                     __nv_bfloat16* outp =
                         reinterpret_cast<__nv_bfloat16*>(a.out_mat) + ((size_t)bh * L + r) * 64 + OW * pt;
 #pragma unroll
@@ -865,7 +867,7 @@ __global__ void __launch_bounds__(nthreads(MODE), ctas_per_sm(MODE)) tc_band_swe
                         float tot = 0.f;
 #pragma unroll
                         for (int k = 0; k < NPART; ++k) tot += rr[k * 128 + lr];
-                        a.out_vec.at(bh, r) = rokf ? tot : 0.f;
+                        if (SA_BOUNDS(bh < BH && r >= 0, status)) a.out_vec.at(bh, r) = rokf ? tot : 0.f;
                     }
                 }
             }

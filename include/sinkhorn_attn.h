@@ -21,6 +21,12 @@
  *   dustbin row and one dustbin column (plus their corner) carrying the
  *   constant score dustbin_score, with unit mass like every other row/column.
  *
+ * Debug build: compiled with -DSA_DEBUG (libsinkhorn_attn_debug.so) every
+ * kernel checks the indices of its guarded accesses (global rows and columns,
+ * ring and buffer slots, tensor-memory columns, shared-memory offsets) before
+ * making them; a failed check skips the access and records SA_ERR_BOUNDS in
+ * the status word (read by sinkhorn_attn_poll).  Nothing traps.
+ *
  * Conventions shared by every entry point
  *   - The caller owns every buffer.  The library allocates no device or host
  *     memory in any call and keeps no mutable global state, so concurrent
@@ -58,7 +64,8 @@ typedef enum {
     SA_ERR_CUDA = -4,         /* a CUDA runtime call or kernel launch failed */
     SA_ERR_NONFINITE = -5,    /* device found a NaN/Inf (only with check_finite) */
     SA_ERR_TIMEOUT = -6,      /* a bounded device-side wait gave up */
-    SA_ERR_EXCHANGE = -7      /* a sharded call's halo exchange callback failed */
+    SA_ERR_EXCHANGE = -7,     /* a sharded call's halo exchange callback failed */
+    SA_ERR_BOUNDS = -8        /* debug build only: a device-side bounds check failed */
 } sa_status;
 
 typedef enum { SA_F32 = 0, SA_BF16 = 1 } sa_dtype;

@@ -143,7 +143,7 @@ def test_empty_problem_is_a_noop():
 
 
 def test_strerror_covers_every_status():
-    for s in range(0, -7, -1):
+    for s in range(0, -9, -1):
         assert sa.strerror(s) and "unknown" not in sa.strerror(s)
     assert "unknown" in sa.strerror(42)
 
@@ -233,3 +233,12 @@ def test_binding_does_none_of_the_methods_arithmetic():
     # the score scale and the certificate's eta / R* live in the C library
     src = open(os.path.join(ROOT, "banded_log_domain_b200", "__init__.py")).read()
     assert "score_scale" not in src and "math.sqrt" not in src and "import math" not in src
+
+
+def test_debug_library_exports_the_same_entry_points():
+    # the bounds-checked build (-DSA_DEBUG) is the same C ABI
+    assert os.path.exists(sa.DEBUG_LIB_PATH)
+    lib = ctypes.CDLL(sa.DEBUG_LIB_PATH)
+    for n in declared():
+        assert hasattr(lib, n), n
+    assert sa.strerror(-8) and "bounds" in sa.strerror(-8)

@@ -53,6 +53,11 @@ SMALL = [
     # after the next tile's first chunk
     (8192, 64, 0.9, 3, 2, "bf16", (6000, 8192), False),
     (8192, 100, 1.0, 2, 1, "bf16", "holes", False),
+    # every chunk count modulo the four epilogue parts (a chunk's readers then
+    # fall on different parts): 2W + 128 over 128 = 4, 6, 7
+    (4096, 192, 1.0, 3, 2, "bf16", "holes", False),
+    (4096, 320, 0.8, 2, 2, "bf16", None, False),
+    (4096, 384, 1.0, 2, 1, "bf16", (3000, 4096), False),
 ]
 
 

@@ -1,0 +1,100 @@
+"""The method's cost model on the device (gist.science/de, technical summary
+section 2.1): O((T+R) L W) time and O(L) extra memory.
+
+* Time: forward + backward device time, fitted linearly against L at fixed W
+  (R^2 > 0.99) and against W at fixed L.  The kernels tile rows in blocks of 128
+  and columns in chunks of 128, so the work of a row block follows its chunk
+  count ceil((2W + 128) / 128), a step function of W; the W sweep uses W with
+  2W + 128 a multiple of 128, where the count is exact.  Even chunk counts run
+  a few percent less efficiently than odd ones (the four epilogue parts then
+  see a shorter MMA lookahead), so the W fit is held to R^2 > 0.98 (measured
+  0.986-0.990) and the time must rise strictly with W.
+* Memory: the device memory a forward + backward allocates beyond its inputs
+  (outputs, dual state and both workspaces, allocated through PyTorch by the
+  binding) grows linearly in L and does not depend on W: nothing of size L*W
+  is ever stored.
+"""
+import numpy as np
+import pytest
+import torch
+
+pytestmark = pytest.mark.gpu
+
+
+def _inputs(H, L, seed=0):
+    g = torch.Generator(device="cuda").manual_seed(seed)
+    mk = lambda: torch.randn(1, H, L, 64, generator=g, device="cuda").to(torch.bfloat16)
+    return mk(), mk(), mk(), mk()
+
+
+def _step_ms(q, k, v, dO, W, reps=3):
+    import banded_log_domain_b200 as sa
+
+    kw = dict(W=W, eps=1.0, R=2)
+    o, st = sa.sinkhorn_attn_fwd(q, k, v, T=6, **kw)
+    sa.sinkhorn_attn_bwd(q, k, v, o, dO, st, **kw)  # warm-up
+    times = []
+    for _ in range(reps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        e0.record()
+        o, st = sa.sinkhorn_attn_fwd(q, k, v, T=6, **kw)
+        sa.sinkhorn_attn_bwd(q, k, v, o, dO, st, **kw)
+        e1.record()
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1))
+    return float(np.median(times))
+
+
+def _r2(x, y):
+    x, y = np.asarray(x, float), np.asarray(y, float)
+    A = np.vstack([x, np.ones_like(x)]).T
+    coef, *_ = np.linalg.lstsq(A, y, rcond=None)
+    res = y - A @ coef
+    return 1.0 - (res @ res) / ((y - y.mean()) @ (y - y.mean())), coef
+
+
+def test_device_time_is_linear_in_L_and_W():
+    H = 16
+    Ls = [16384, 32768, 49152, 65536]
+    q, k, v, dO = _inputs(H, max(Ls))
+    tL = [_step_ms(*(t[:, :, :L].contiguous() for t in (q, k, v, dO)), W=128) for L in Ls]
+    r2L, cL = _r2(Ls, tL)
+    assert cL[0] > 0 and r2L > 0.99, (tL, r2L)
+    L = 32768
+    Ws = [64, 128, 192, 256, 320]
+    qs = [t[:, :, :L].contiguous() for t in (q, k, v, dO)]
+    tW = [_step_ms(*qs, W=W) for W in Ws]
+    r2W, cW = _r2(Ws, tW)
+    assert cW[0] > 0 and r2W > 0.98, (tW, r2W)
+    assert all(b > a for a, b in zip(tW, tW[1:])), tW
+
+
+def test_extra_memory_is_linear_in_L_and_independent_of_W():
+    import banded_log_domain_b200 as sa
+
+    H = 8
+
+    def extra(L, W):
+        q, k, v, dO = _inputs(H, L, seed=1)
+        torch.cuda.synchronize()
+        base = torch.cuda.memory_allocated()
+        torch.cuda.reset_peak_memory_stats()
+        kw = dict(W=W, eps=1.0, R=2)
+        o, st = sa.sinkhorn_attn_fwd(q, k, v, T=3, **kw)
+        g = sa.sinkhorn_attn_bwd(q, k, v, o, dO, st, **kw)
+        torch.cuda.synchronize()
+        peak = torch.cuda.max_memory_allocated() - base
+        del o, st, g
+        return peak
+
+    Ls = [8192, 16384, 32768]
+    for W in (32, 256):
+        m = [extra(L, W) for L in Ls]
+        # linear in L: doubling L doubles the extra memory (within allocator rounding)
+        assert abs(m[1] / m[0] - 2.0) < 0.02 and abs(m[2] / m[1] - 2.0) < 0.02, m
+    assert extra(16384, 32) == extra(16384, 256)
+    # and it is O(L) with a small constant: outputs (4 d-vectors per token) plus
+    # the dual state and workspaces (tens of floats per token), far below L*W
+    per_token = extra(16384, 256) / (H * 16384)
+    assert per_token < 4 * 64 * 2 + 100 * 4, per_token
