@@ -64,8 +64,8 @@ using simt::SweepArgs;
 constexpr int LSE = simt::LSE, WSUM = simt::WSUM;
 
 constexpr int NEPI = 16;                 // epilogue warps: quadrant w % 4, part w / 4
-constexpr int W_LOAD = NEPI, W_MMA = NEPI + 1;
-constexpr int NTHREADS = (NEPI + 2) * 32;
+constexpr int W_LOAD = NEPI, W_MMA = NEPI + 1, W_FIN = NEPI + 2;
+constexpr int NTHREADS = (NEPI + 3) * 32;
 constexpr int NRING = 8;                 // K-chunk ring slots
 constexpr int NRED = 8;                  // ring of per-tile partial row sums
 constexpr int TILE = 16384;              // 128 tokens x 64 bf16, 128-byte swizzle
@@ -83,7 +83,7 @@ constexpr int OFF_CV = OFF_K + NRING * TILE;          // NRING x 128 column dual
 constexpr int OFF_WV = OFF_CV + NRING * 128 * 4;      // NRING x 128 weights (WSUM)
 constexpr int OFF_SCR = OFF_WV + NRING * 128 * 4;     // per warp: 128 shifted column duals
 constexpr int OFF_RED = OFF_SCR + NEPI * 128 * 4;     // NRED x 4 parts x 128 partial sums
-constexpr int OFF_CNT = OFF_RED + NRED * 4 * 128 * 4; // NRED x 4 arrival counters
+constexpr int OFF_CNT = OFF_RED + NRED * 4 * 128 * 4; // (unused)
 // Per-tile row data, copied by the loader ahead of the epilogue (a ring of NRI
 // tiles): the rows' working duals (shift sources or row duals), and the WSUM
 // base and multiplier.
@@ -97,7 +97,8 @@ constexpr int OFF_RI = OFF_CNT + NRED * 4 * 4;
 constexpr int OFF_BAR = (OFF_RI + NRI * (int)sizeof(RowInfo) + 7) / 8 * 8;
 enum { B_AFULL = 0, B_AEMPTY = 2, B_FULL = 4, B_EMPTY = B_FULL + NRING, B_SFULL = B_EMPTY + NRING,
        B_SEMPTY = B_SFULL + 4, B_RFULL = B_SEMPTY + 4, B_REMPTY = B_RFULL + NRI,
-       B_DRAIN = B_REMPTY + NRI, NBAR = B_DRAIN + 1 };
+       B_QFULL = B_REMPTY + NRI, B_QEMPTY = B_QFULL + NRED, B_DRAIN = B_QEMPTY + NRED,
+       NBAR = B_DRAIN + 1 };
 constexpr int SMEM_BYTES = OFF_BAR + NBAR * 8 + 16 + 1024;
 static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
 
@@ -228,7 +229,6 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_rowsum_sweep(const SweepArgs a
     float* cvring = reinterpret_cast<float*>(sm + OFF_CV);
     float* wring = reinterpret_cast<float*>(sm + OFF_WV);
     float* red = reinterpret_cast<float*>(sm + OFF_RED);
-    int* cnt = reinterpret_cast<int*>(sm + OFF_CNT);
     RowInfo* rinfo = reinterpret_cast<RowInfo*>(sm + OFF_RI);
     Ctl ctl{bar, abort_flag, status};
 
@@ -263,13 +263,16 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_rowsum_sweep(const SweepArgs a
         }
         for (int i = 0; i < NRI; ++i) {
             tc::mbar_init(bar + B_RFULL + i, 32);     // the loader lanes' copies
-            tc::mbar_init(bar + B_REMPTY + i, NEPI);  // every epilogue warp has read it
+            tc::mbar_init(bar + B_REMPTY + i, NEPI + 1);  // every epilogue warp and the finisher
+        }
+        for (int i = 0; i < NRED; ++i) {
+            tc::mbar_init(bar + B_QFULL + i, NEPI);   // every epilogue warp's partial row sums
+            tc::mbar_init(bar + B_QEMPTY + i, 1);     // the finisher has read them
         }
         tc::mbar_init(bar + B_DRAIN, 1);
         *abort_flag = 0;
         tc::fence_mbar_init();
     }
-    for (int i = threadIdx.x; i < NRED * 4; i += NTHREADS) cnt[i] = 0;
     if (warp == 0) {
         tc::tmem_alloc(tbase, 512);
         tc::tmem_relinquish();
@@ -423,6 +426,54 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_rowsum_sweep(const SweepArgs a
         if (tc::elect_one()) tc::tc_commit(bar + B_DRAIN);
         __syncwarp();
         tc::mbar_wait(bar + B_DRAIN, 0, kWaitBudget);
+    } else if (warp == W_FIN) {
+        // ------------------------------------------------------------ finisher
+        // Each tile's outputs from the four parts' partial row sums; lane l
+        // writes rows 32k + l.  The shift of a quadrant is formed as the
+        // epilogue forms it (the smallest working dual of its valid rows,
+        // per-row shifts past a spread of 64).
+        Cursor cur = cur0;
+        for (int it = 0; it < ntl; ++it, cur.next(nblk, H)) {
+            const int bh = cur.b * H + cur.h, r0 = cur.rb * 128, slot = it % NRED;
+            if (!ctl.wait(B_RFULL + it % NRI, (it / NRI) & 1)) break;
+            if (!ctl.wait(B_QFULL + slot, (it / NRED) & 1)) break;
+            const RowInfo& ri = rinfo[it % NRI];
+            const float* rs = red + slot * 512;
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const int lr = 32 * k + lane, r = r0 + lr;
+                const float rwv = ri.rw[lr];
+                const bool valid = r < L && rwv != -INFINITY;
+                const float sr = valid ? rwv : 0.f;
+                float mn = valid ? sr : INFINITY, mx = valid ? sr : -INFINITY;
+                asm("redux.sync.min.f32 %0, %0, 0xffffffff;" : "+f"(mn));
+                asm("redux.sync.max.f32 %0, %0, 0xffffffff;" : "+f"(mx));
+                const float sq = mn == INFINITY ? 0.f : mn;
+                const bool fb = mn != INFINITY && mx - mn > kFallbackSpread;
+                const float seff = (fb && valid) ? sr : sq;
+                const float tot = (rs[lr] + rs[128 + lr]) + (rs[256 + lr] + rs[384 + lr]);
+                if (r < L && SA_BOUNDS(bh < BH, status)) {
+                    float out = 0.f, outw = -INFINITY;
+                    if (valid) {
+                        if (MODE == LSE) {
+                            outw = seff - lg2(tot);
+                            out = outw * kLn2;
+                        } else {
+                            const float bb = ri.base[lr];
+                            const float mu = a.mult.p ? ri.mult[lr] : 1.f;
+                            out = bb + a.sgn * mu * (tot * ex2(sr - seff));
+                        }
+                    }
+                    a.out_vec.at(bh, r) = out;
+                    if (MODE == LSE && a.outw.p) a.outw.at(bh, r) = outw;
+                }
+            }
+            __syncwarp();
+            if (lane == 0) {
+                tc::mbar_arrive(bar + B_QEMPTY + slot);
+                tc::mbar_arrive(bar + B_REMPTY + it % NRI);
+            }
+        }
     } else {
         // ------------------------------------------------------------ epilogue
         const int qd = warp & 3, pt = warp >> 2;
@@ -442,7 +493,6 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_rowsum_sweep(const SweepArgs a
             ids.advance(succ, nch);
             Cursor nx = cur;
             nx.next(nblk, H);
-            const bool next_succ = reuse && it + 1 < ntl && nx.b * H + nx.h == bh && nx.rb == cur.rb + 1;
             // this thread's row and the warp's shift (the smallest working dual of
             // the quadrant's valid rows; per-row shifts past a spread of 64)
             const int rw0 = r0 + qd * 32, r = rw0 + lane;
@@ -451,27 +501,26 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_rowsum_sweep(const SweepArgs a
             const float rwv = ri.rw[qd * 32 + lane];
             const bool valid = r < L && rwv != -INFINITY;
             const float sr = valid ? rwv : 0.f;
-            const float bb = MODE == WSUM ? ri.base[qd * 32 + lane] : 0.f;
-            const float mu = (MODE == WSUM && a.mult.p) ? ri.mult[qd * 32 + lane] : 1.f;  // none: 1
             __syncwarp();
             if (lane == 0) tc::mbar_arrive(bar + B_REMPTY + it % NRI);
             float mn = valid ? sr : INFINITY, mx = valid ? sr : -INFINITY;
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) {
-                mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
-                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-            }
+            asm("redux.sync.min.f32 %0, %0, 0xffffffff;" : "+f"(mn));
+            asm("redux.sync.max.f32 %0, %0, 0xffffffff;" : "+f"(mx));
             const float sq = mn == INFINITY ? 0.f : mn;
             const bool fb = mn != INFINITY && mx - mn > kFallbackSpread;
             const float seff = (fb && valid) ? sr : sq;  // this row's shift
             const float delta = seff - sq;
             uint64_t acc[4] = {0, 0, 0, 0};
-            for (int c = 0; c < nch; ++c, ++g) {
-                // chunk g of tile it goes to part (g + rot * it) % 4, in that
+            // this part's chunks of the tile: c = c0, c0 + 4, ...
+            const int g_t = g;
+            g += nch;
+            for (int c = (pt - (g_t + rot * it)) & 3; c < nch; c += 4) {
+                const int gg = g_t + c;
+                // chunk gg of tile it goes to part (gg + rot * it) % 4, in that
                 // part's own TMEM buffer, whose phases its one part consumes in
                 // order
-                if (((g + rot * it) & 3) != pt) continue;
                 const int id = ids.base + c, s = id % NRING, b = pt;
+                (void)gg;
                 if (!ctl.wait(B_SFULL + b, nu & 1)) { ok = false; break; }
                 ++nu;
                 if (!ctl.wait(B_FULL + s, (id / NRING) & 1)) { ok = false; break; }
@@ -514,39 +563,18 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_rowsum_sweep(const SweepArgs a
             }
             if (!ok) break;
             // ---------------------------------------------------------- end of tile
+            // this part's partial row sums, for the finisher
             float a0, a1, a2, a3, a4, a5, a6, a7;
             tc::upk2(acc[0], a0, a1);
             tc::upk2(acc[1], a2, a3);
             tc::upk2(acc[2], a4, a5);
             tc::upk2(acc[3], a6, a7);
             const int slot = it % NRED;
-            float* rs = red + slot * 512;
-            if (SA_BOUNDS(slot < NRED && pt < 4, status)) rs[pt * 128 + qd * 32 + lane] = ((a0 + a1) + (a2 + a3)) + ((a4 + a5) + (a6 + a7));
+            if (it >= NRED && !ctl.wait(B_QEMPTY + slot, ((it / NRED) - 1) & 1)) { ok = false; break; }
+            if (SA_BOUNDS(slot < NRED && pt < 4, status))
+                red[slot * 512 + pt * 128 + qd * 32 + lane] = ((a0 + a1) + (a2 + a3)) + ((a4 + a5) + (a6 + a7));
             __syncwarp();
-            __threadfence_block();
-            int old = 0;
-            if (lane == 0) old = atomicAdd(cnt + slot * 4 + qd, 1);
-            old = __shfl_sync(0xffffffffu, old, 0);
-            if ((old & 3) == 3) {  // the last of the quadrant's four parts: write its rows
-                __threadfence_block();
-                const float tot = (rs[qd * 32 + lane] + rs[128 + qd * 32 + lane]) +
-                                  (rs[256 + qd * 32 + lane] + rs[384 + qd * 32 + lane]);
-                if (r < L) {
-                    float out = 0.f, outw = -INFINITY;
-                    if (valid) {
-                        if (MODE == LSE) {
-                            outw = seff - lg2(tot);
-                            out = outw * kLn2;
-                        } else {
-                            out = bb + a.sgn * mu * (tot * ex2(sr - seff));
-                        }
-                    }
-                    if (SA_BOUNDS(bh < BH && r >= 0, status)) {
-                        a.out_vec.at(bh, r) = out;
-                        if (MODE == LSE && a.outw.p) a.outw.at(bh, r) = outw;
-                    }
-                }
-            }
+            if (lane == 0) tc::mbar_arrive(bar + B_QFULL + slot);
             cur = nx;
         }
     }
