@@ -88,6 +88,11 @@ struct SweepArgs {
     Vec cdw;                // column side
     Vec rdw;                // row side (LSE: the shift source; WSUM: the row dual)
     MVec outw;              // LSE: the new dual's working copy (or p null)
+    // and the column side's dual as a score-MMA operand row, bf16 [BH][..][L][16]
+    // (element (bh, t) at augc + bh * aug_s + 16 t), and the LSE output's row
+    const void* augc;
+    void* augo;
+    long long aug_s;
 };
 
 // ---------------------------------------------------------------------------

@@ -103,9 +103,14 @@ bool mask_ok(const void* x) { return !x || on_current_device(x); }
 
 // The row-sum sweeps on the tensor cores (bf16 storage without a dustbin) read
 // the duals as a working copy of the state: [BH][2R+2][L] float32, log2(e)
-// times each dual on valid tokens and -inf on masked ones.
+// times each dual on valid tokens and -inf on masked ones; then the same duals
+// as score-MMA operands, [BH][2R+2][L][16] bf16: slots 0-2 hold a three-way
+// bf16 split of dual / c (c the score scale, so the dual is in the units of
+// <q, k>), -1e30 on masked tokens, slots 3-15 zero.
 bool uses_work_state(const sa_params* p) { return p->dtype == SA_BF16 && !p->dustbin; }
-size_t work_state_bytes(const Dims& d) { return align_up((size_t)d.BH * (2 * d.R + 2) * d.L * sizeof(float)); }
+size_t work_floats_bytes(const Dims& d) { return align_up((size_t)d.BH * (2 * d.R + 2) * d.L * sizeof(float)); }
+size_t work_aug_bytes(const Dims& d) { return align_up((size_t)d.BH * (2 * d.R + 2) * d.L * 16 * 2); }
+size_t work_state_bytes(const Dims& d) { return work_floats_bytes(d) + work_aug_bytes(d); }
 
 // Forward workspace: the status header, then the working copy of the state
 // (tensor-core path only).
@@ -205,18 +210,23 @@ __global__ void k_vmul(const float* x, const float* y, float s, float* out, long
 }
 
 // Working copy of state rows [r_lo, r_hi) of every problem: w = log2(e) * dual
-// on valid tokens, -inf on masked ones (state [BH][2R+2][ld], work [BH][2R+2][L]).
+// on valid tokens, -inf on masked ones (state [BH][2R+2][ld], work [BH][2R+2][L]),
+// and the operand rows aug [BH][2R+2][L][16] (see tcr::put_aug).
 __global__ void k_work(const float* state, int nrows, int ld, int L, int H, int BH,
-                       const uint8_t* mask, int r_lo, int r_hi, float* work) {
+                       const uint8_t* mask, int r_lo, int r_hi, float inv_c, float* work,
+                       __nv_bfloat16* aug, int* status) {
     const long long g = (long long)blockIdx.x * blockDim.x + threadIdx.x;
     const int nr = r_hi - r_lo;
     if (g >= (long long)BH * nr * L) return;
     const int t = (int)(g % L);
     const long long rest = g / L;
     const int row = r_lo + (int)(rest % nr), bh = (int)(rest / nr);
+    if (!SA_BOUNDS(bh < BH && row < nrows, status)) return;
     const bool ok = mask == nullptr || mask[(size_t)(bh / H) * L + t];
     const float v = state[((size_t)bh * nrows + row) * ld + t];
-    work[((size_t)bh * nrows + row) * L + t] = ok ? v * kLog2e : -INFINITY;
+    const size_t o = ((size_t)bh * nrows + row) * L + t;
+    work[o] = ok ? v * kLog2e : -INFINITY;
+    tcr::put_aug(aug + o * 16, ok, v * inv_c);
 }
 
 // dv_dust[h][e] = sum_b part[(b*H + h)][e]
@@ -517,6 +527,20 @@ bool make_map_aug(CUtensorMap* m, const void* ptr, int L, int BH) {
            CUDA_SUCCESS;
 }
 
+// [BH][L][16] bf16 operand rows whose problems lie `bh_stride` elements apart
+bool make_map_aug_strided(CUtensorMap* m, const void* ptr, int L, int BH, long long bh_stride) {
+    auto fn = encode_tiled();
+    if (!fn || !ptr) return false;
+    cuuint64_t dims[3] = {16, (cuuint64_t)L, (cuuint64_t)BH};
+    cuuint64_t strides[2] = {16 * 2, (cuuint64_t)bh_stride * 2};
+    cuuint32_t box[3] = {16, 128, 1};
+    cuuint32_t es[3] = {1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box,
+              es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_32B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+           CUDA_SUCCESS;
+}
+
 template <int MODE, bool ONLINE, int NT>
 cudaError_t launch_tc(const simt::SweepArgs& a, int BH, cudaStream_t st, Tracer& tr,
                       int* status) {
@@ -572,7 +596,11 @@ cudaError_t launch_rowsum(const simt::SweepArgs& a, int BH, cudaStream_t st, Tra
                           int* status) {
     tcr::Maps maps;
     std::memset(&maps, 0, sizeof(maps));
-    if (!make_map(&maps.A, a.A, a.L, BH) || !make_map(&maps.B, a.Bo, a.L, BH))
+    void* ones = nullptr;
+    if (cudaGetSymbolAddress(&ones, tcr::g_aug_ones) != cudaSuccess || !ones) return cudaErrorInvalidValue;
+    if (!make_map(&maps.A, a.A, a.L, BH) || !make_map(&maps.B, a.Bo, a.L, BH) ||
+        !make_map_aug_strided(&maps.BA, a.augc, a.L, BH, a.aug_s) ||
+        !make_map_aug_strided(&maps.AO, ones, 128, 1, 128 * 16))
         return cudaErrorInvalidValue;
     const long long ntiles = (long long)((a.L + 127) / 128) * BH;
     const dim3 grid((unsigned)std::min<long long>(ntiles, (long long)sm_count()));
@@ -647,19 +675,27 @@ struct Ctx {
     const sa_shard* shard = nullptr;  // sequence-sharded call, else null
     // state row r (0..2R+1) as a Vec
     Vec srow(int r) const { return vec(state + (size_t)r * d.ld, sst); }
-    // its working copy (tensor-core row-sum sweeps), or a null Vec
+    // its working copy and operand row (tensor-core row-sum sweeps), or null
     float* work = nullptr;
+    __nv_bfloat16* waug = nullptr;
     Vec wrow(int r) const {
         return work ? vec(work + (size_t)r * d.L, (long long)(2 * d.R + 2) * d.L) : Vec{nullptr, 0};
     }
     MVec mwrow(int r) const { Vec v = wrow(r); return MVec{const_cast<float*>(v.p), v.s}; }
+    __nv_bfloat16* augrow(int r) const { return waug ? waug + (size_t)r * d.L * 16 : nullptr; }
+    long long aug_stride() const { return (long long)(2 * d.R + 2) * d.L * 16; }
+    void set_work(char* base) {
+        work = (float*)base;
+        waug = (__nv_bfloat16*)(base + work_floats_bytes(d));
+    }
     // rebuilds working rows [lo, hi) from the state
     sa_status refresh_work(const uint8_t* mask, int lo, int hi) const {
         if (!work) return SA_OK;
         const long long n = (long long)d.BH * (hi - lo) * d.L;
         tr.begin(SA_KERNEL_AUX);
         k_work<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(state, 2 * d.R + 2, d.ld, d.L, d.H,
-                                                             d.BH, mask, lo, hi, work);
+                                                             d.BH, mask, lo, hi, 1.0f / c, work,
+                                                             waug, status);
         tr.end();
         return cudaGetLastError() == cudaSuccess ? SA_OK : SA_ERR_CUDA;
     }
@@ -724,6 +760,9 @@ sa_status fwd_impl(const Ctx& x, const T* q, const T* k, const T* v, const uint8
         a.cdw = x.wrow(2 * rin + 1);
         a.rdw = x.wrow(2 * rin);
         a.outw = x.mwrow(2 * rout);
+        a.augc = x.augrow(2 * rin + 1);
+        a.augo = x.augrow(2 * rout);
+        a.aug_s = x.aug_stride();
         a.online = (it == 0);
         a.out_vec = mvec(state + (size_t)(2 * rout) * d.ld, x.sst);
         SA_CUDA((launch_sweep<T, simt::LSE>(a, d.BH, x.st, x.tr, x.status)));
@@ -741,6 +780,9 @@ sa_status fwd_impl(const Ctx& x, const T* q, const T* k, const T* v, const uint8
         a.cdw = x.wrow(2 * rout);
         a.rdw = x.wrow(2 * rin + 1);
         a.outw = x.mwrow(2 * rout + 1);
+        a.augc = x.augrow(2 * rout);
+        a.augo = x.augrow(2 * rout + 1);
+        a.aug_s = x.aug_stride();
         a.online = 0;
         a.out_vec = mvec(state + (size_t)(2 * rout + 1) * d.ld, x.sst);
         SA_CUDA((launch_sweep<T, simt::LSE>(a, d.BH, x.st, x.tr, x.status)));
@@ -821,6 +863,7 @@ sa_status bwd_impl(const Ctx& x, const T* q, const T* k, const T* v, const uint8
         a.A = q; a.Bo = k;
         a.rd = uR; a.cd = vR;
         a.rdw = x.wrow(2 * R); a.cdw = x.wrow(2 * R + 1);
+        a.augc = x.augrow(2 * R + 1); a.aug_s = x.aug_stride();
         a.w = vec(vb(R), vs);
         a.base = vec(A_, vs);
         a.sgn = -1.f;
@@ -838,11 +881,13 @@ sa_status bwd_impl(const Ctx& x, const T* q, const T* k, const T* v, const uint8
         if (direct) {
             a.rd = V(r - 1); a.cd = U(r);
             a.rdw = x.wrow(2 * (r - 1) + 1); a.cdw = x.wrow(2 * r);
+            a.augc = x.augrow(2 * r); a.aug_s = x.aug_stride();
             a.w = vec(ub(r), vs);
         } else {
             SA_AUX(x.tr, k_vmul<<<egrid, eb, 0, x.st>>>(eu(r), ub(r), 1.f, W_(l.w, 0), nvec));
             a.rd = vR; a.cd = uR;
             a.rdw = x.wrow(2 * R + 1); a.cdw = x.wrow(2 * R);
+            a.augc = x.augrow(2 * R); a.aug_s = x.aug_stride();
             a.w = vec(W_(l.w, 0), vs);
             a.mult = vec(ev(r - 1), vs);
         }
@@ -857,11 +902,13 @@ sa_status bwd_impl(const Ctx& x, const T* q, const T* k, const T* v, const uint8
         if (direct) {
             b.rd = U(r - 1); b.cd = V(r - 1);
             b.rdw = x.wrow(2 * (r - 1)); b.cdw = x.wrow(2 * (r - 1) + 1);
+            b.augc = x.augrow(2 * (r - 1) + 1); b.aug_s = x.aug_stride();
             b.w = vec(vb(r - 1), vs);
         } else {
             SA_AUX(x.tr, k_vmul<<<egrid, eb, 0, x.st>>>(ev(r - 1), vb(r - 1), 1.f, W_(l.w, 0), nvec));
             b.rd = uR; b.cd = vR;
             b.rdw = x.wrow(2 * R); b.cdw = x.wrow(2 * R + 1);
+            b.augc = x.augrow(2 * R + 1); b.aug_s = x.aug_stride();
             b.w = vec(W_(l.w, 0), vs);
             b.mult = vec(eu(r - 1), vs);
         }
@@ -1059,7 +1106,7 @@ sa_status fwd_call(const sa_params* p, const sa_shard* shard, const void* q, con
     x.tr.p = p;
     x.tr.st = x.st;
     x.shard = shard;
-    if (uses_work_state(p)) x.work = (float*)((char*)ws + fwd_layout(d, p).work);
+    if (uses_work_state(p)) x.set_work((char*)ws + fwd_layout(d, p).work);
     const float* vd = p->dustbin ? v_dust : nullptr;
     if (p->dtype == SA_F32)
         s = fwd_impl<float>(x, (const float*)q, (const float*)k, (const float*)v, mask, vd,
@@ -1109,7 +1156,7 @@ sa_status bwd_call(const sa_params* p, const sa_shard* shard, const void* q, con
     x.tr.p = p;
     x.tr.st = x.st;
     x.shard = shard;
-    if (uses_work_state(p)) x.work = (float*)((char*)ws + bwd_layout(d, p).work);
+    if (uses_work_state(p)) x.set_work((char*)ws + bwd_layout(d, p).work);
     const float* vd = p->dustbin ? v_dust : nullptr;
     float* dvd = p->dustbin ? dv_dust : nullptr;
     float* dsc = p->dustbin ? d_dust_score : nullptr;
@@ -1505,7 +1552,7 @@ sa_status sinkhorn_attn_bwd_static_ws(const sa_params* p, const void* q, const v
     x.status = (int*)ws;
     x.tr.p = p;
     x.tr.st = st;
-    if (uses_work_state(p)) x.work = (float*)((char*)ws + bwd_layout(d, p).work);
+    if (uses_work_state(p)) x.set_work((char*)ws + bwd_layout(d, p).work);
     const float* vd = p->dustbin ? v_dust : nullptr;
     float* dvd = p->dustbin ? dv_dust : nullptr;
     float* dsc = p->dustbin ? d_dust_score : nullptr;

@@ -13,7 +13,7 @@
 // block of 128) tiles.  A tile's columns are the chunks r0 - W + 128 c,
 // c < nch = ceil((2W + 128) / 128), on one grid for the whole problem, so that
 // the next row block of the same problem needs only one new chunk: the K-side
-// chunks (TMA tiles with their column duals) sit in a ring of NRING slots and
+// chunks (TMA tiles with their column-dual operands) sit in a ring of NRING slots and
 // a chunk stays until every tile that reads it has (reuse; streaming when W is
 // so large that a tile's chunks do not fit the ring).  A slot's EMPTY barrier
 // expects 4 arrivals (one per quadrant warp) from each of up to nch uses and
@@ -23,25 +23,28 @@
 // part p) processes the 32 rows of quadrant q of the chunks assigned to part
 // p, from buffer p: a whole 128-column chunk per warp, so the MMA runs up to
 // four chunks ahead; the assignment rotates the band-edge chunks over the
-// parts.  The four parts' partial row sums of a tile meet in
-// shared memory; the last part of a quadrant to finish the tile writes its 32
-// outputs (a counter per quadrant, no waiting).
+// parts.  The four parts' partial row sums of a tile meet in shared memory,
+// where a finisher warp adds them and writes the tile's outputs.
 //
-// Operand traffic.  Q and K tiles come by TMA; the O(L) vectors by 4-byte
-// cp.async into the same ring slots (completion counted on the slot's
-// mbarrier), so the loader never waits for a global load.  The duals are read
-// as working copies (log2(e) times the dual, -inf on masked tokens), which
-// each LSE sweep writes next to its natural-unit output for the sweep after it:
-// no mask or scaling on the loader's path.  Columns outside [0, L) are
-// zero-filled and excluded by the band-edge test.
+// Operand traffic.  Q and K tiles come by TMA, and with each K chunk the
+// column duals as a 16-wide bf16 operand row per token (a three-way bf16 split
+// of dual / c in slots 0-2, c the score scale): a fifth MMA of the chunk, with a
+// constant row-block operand [1, 1, 1, 0, ...], adds the column dual to every
+// score in TMEM, so the epilogue reads no column vector at all.  The split
+// keeps 24 significant bits of the dual; the sum is formed in the fp32
+// accumulator.  Masked columns carry -1e30, which drives their terms to 0.
+// The per-row data (the rows' working duals, the WSUM base and multiplier)
+// and the WSUM weights come by 4-byte cp.async, counted on mbarriers, so the
+// loader never waits for a global load.  The duals are read as working copies
+// (log2(e) times the dual, -inf on masked tokens, and the operand rows), which
+// each LSE sweep writes next to its natural-unit output for the sweep after
+// it.  Columns outside [0, L) are zero-filled and excluded by the band-edge
+// test.
 //
 // Exponent shift.  Every term is a plan entry of a plan with unit columns (or
-// rows) and so is at most 1 when shifted by the row's previous dual rd_i.  A
-// warp uses one shift for its 32 rows, the smallest rd_i of the valid rows, so
-// that the per-entry argument is one FMA, c2 * s + (cd_j + shift), with the
-// column part formed once per chunk; all arguments stay <= 0.  When the rows'
-// duals spread over more than 64 (log2 units) the warp falls back to per-row
-// shifts (one more addition per entry).
+// rows) and so is at most 1 when shifted by the row's previous dual rd_i, so
+// each row uses its own shift: the per-entry argument is one FMA,
+// c2 * (s + cd_j / c) + rd_i, with all arguments <= 0 up to rounding.
 //
 // Exponentials: 2^x on the MUFU unit (ex2.approx), and for KP of every 32
 // entries of a group that lies inside the band on the FMA pipe: range
@@ -69,8 +72,9 @@ constexpr int NTHREADS = (NEPI + 3) * 32;
 constexpr int NRING = 8;                 // K-chunk ring slots
 constexpr int NRED = 8;                  // ring of per-tile partial row sums
 constexpr int TILE = 16384;              // 128 tokens x 64 bf16, 128-byte swizzle
+constexpr int AUGB = 4096;               // 128 tokens x 16 bf16 operand rows, 32-byte swizzle
 constexpr long long kWaitBudget = 4000000000LL;  // clock cycles (about 2 s)
-constexpr float kFallbackSpread = 64.f;  // log2 units
+constexpr float kMaskedDual = -1e30f;    // an operand row's dual on a masked token
 
 // nch chunks of one tile fit the ring with two to spare: chunks are reused
 __host__ __device__ constexpr int nchunks(int W) { return (2 * W + 128 + 127) / 128; }
@@ -79,11 +83,10 @@ __host__ __device__ constexpr bool reuse_ok(int W) { return nchunks(W) + 2 <= NR
 // shared memory (offsets from a 1024-aligned base)
 constexpr int OFF_A = 0;                              // 2 row-block tiles (tile parity)
 constexpr int OFF_K = OFF_A + 2 * TILE;               // NRING chunk tiles
-constexpr int OFF_CV = OFF_K + NRING * TILE;          // NRING x 128 column duals (log2)
-constexpr int OFF_WV = OFF_CV + NRING * 128 * 4;      // NRING x 128 weights (WSUM)
-constexpr int OFF_SCR = OFF_WV + NRING * 128 * 4;     // per warp: 128 shifted column duals
-constexpr int OFF_RED = OFF_SCR + NEPI * 128 * 4;     // NRED x 4 parts x 128 partial sums
-constexpr int OFF_CNT = OFF_RED + NRED * 4 * 128 * 4; // (unused)
+constexpr int OFF_AUG = OFF_K + NRING * TILE;         // NRING chunk operand rows
+constexpr int OFF_ONES = OFF_AUG + NRING * AUGB;      // the row-block operand [1, 1, 1, 0, ...]
+constexpr int OFF_WV = OFF_ONES + AUGB;               // NRING x 128 weights (WSUM)
+constexpr int OFF_RED = OFF_WV + NRING * 128 * 4;     // NRED x 4 parts x 128 partial sums
 // Per-tile row data, copied by the loader ahead of the epilogue (a ring of NRI
 // tiles): the rows' working duals (shift sources or row duals), and the WSUM
 // base and multiplier.
@@ -93,18 +96,56 @@ struct RowInfo {
     float base[128];
     float mult[128];
 };
-constexpr int OFF_RI = OFF_CNT + NRED * 4 * 4;
+constexpr int OFF_RI = OFF_RED + NRED * 4 * 128 * 4;
 constexpr int OFF_BAR = (OFF_RI + NRI * (int)sizeof(RowInfo) + 7) / 8 * 8;
 enum { B_AFULL = 0, B_AEMPTY = 2, B_FULL = 4, B_EMPTY = B_FULL + NRING, B_SFULL = B_EMPTY + NRING,
        B_SEMPTY = B_SFULL + 4, B_RFULL = B_SEMPTY + 4, B_REMPTY = B_RFULL + NRI,
-       B_QFULL = B_REMPTY + NRI, B_QEMPTY = B_QFULL + NRED, B_DRAIN = B_QEMPTY + NRED,
-       NBAR = B_DRAIN + 1 };
+       B_QFULL = B_REMPTY + NRI, B_QEMPTY = B_QFULL + NRED, B_ONES = B_QEMPTY + NRED,
+       B_DRAIN = B_ONES + 1, NBAR = B_DRAIN + 1 };
 constexpr int SMEM_BYTES = OFF_BAR + NBAR * 8 + 16 + 1024;
 static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
+static_assert(OFF_AUG % 1024 == 0 && OFF_ONES % 1024 == 0, "operand tiles keep the swizzle atoms aligned");
 
+// TMA maps: row blocks (A), K chunks (B), the chunks' operand rows (BA) and
+// the constant row-block operand (AO, a 128 x 16 tile)
 struct Maps {
-    CUtensorMap A, B;
+    CUtensorMap A, B, BA, AO;
 };
+
+// The constant row-block operand: 128 rows of [1, 1, 1, 0, ..., 0] (bf16 1.0 =
+// 0x3F80), whose product with a chunk's operand rows adds slots 0-2 of each
+// column's row, the three parts of its dual, to every score of the column.
+struct OnesTile {
+    uint16_t v[128 * 16];
+};
+constexpr OnesTile make_ones_tile() {
+    OnesTile t{};
+    for (int r = 0; r < 128; ++r)
+        for (int k = 0; k < 3; ++k) t.v[r * 16 + k] = 0x3F80;
+    return t;
+}
+__device__ __align__(256) const OnesTile g_aug_ones = make_ones_tile();
+
+// Writes a token's operand row: y = dual / c as hi + mid + lo, each the bf16
+// rounding of what the parts before it leave (so the three carry the 24
+// significant bits of y), in slots 0-2; slots 3-15 zero.  A masked token
+// (ok false) gets kMaskedDual in slot 0.
+__device__ __forceinline__ void put_aug(__nv_bfloat16* dst, bool ok, float y) {
+    uint32_t w0 = 0, w1 = 0;
+    if (ok) {
+        const __nv_bfloat16 hi = __float2bfloat16_rn(y);
+        const float r1 = y - __bfloat162float(hi);
+        const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
+        const __nv_bfloat16 lo = __float2bfloat16_rn(r1 - __bfloat162float(mid));
+        w0 = (uint32_t)__bfloat16_as_ushort(hi) | ((uint32_t)__bfloat16_as_ushort(mid) << 16);
+        w1 = (uint32_t)__bfloat16_as_ushort(lo);
+    } else {
+        w0 = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(kMaskedDual));
+    }
+    uint4* o = reinterpret_cast<uint4*>(dst);
+    o[0] = make_uint4(w0, w1, 0u, 0u);
+    o[1] = make_uint4(0u, 0u, 0u, 0u);
+}
 
 struct Ctl {
     uint64_t* bar;
@@ -166,26 +207,16 @@ __device__ __forceinline__ void exp2_poly2(float x0, float x1, float& e0, float&
     e1 = __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23));
 }
 
-// One warp's 32 rows x 32 columns, staged: all arguments, then all
-// exponentials, then the sums.  EDGE keeps only local columns lo..hi.
-template <int MODE, int KP, bool EDGE, bool FB>
-__device__ __forceinline__ void group(const uint32_t (&u)[32], const float* cs, const float* wv,
-                                      float c2, float delta, int lo, int hi, uint64_t (&acc)[4]) {
-    const uint64_t c2p = tc::pk2(c2, c2), dp = tc::pk2(delta, delta);
-    const float4* c4 = reinterpret_cast<const float4*>(cs);
+// One warp's 32 rows x 32 columns, staged: all arguments c2 * S' + rd (S' the
+// score with the column dual folded in), then all exponentials, then the sums.
+// EDGE keeps only local columns lo..hi.
+template <int MODE, int KP, bool EDGE>
+__device__ __forceinline__ void group(const uint32_t (&u)[32], const float* wv, uint64_t c2p,
+                                      uint64_t srp, int lo, int hi, uint64_t (&acc)[4]) {
     uint64_t xp[16];
 #pragma unroll
-    for (int q = 0; q < 8; ++q) {
-        const float4 cv = c4[q];
-        xp[2 * q] = tc::fma2(tc::pk2(__uint_as_float(u[4 * q]), __uint_as_float(u[4 * q + 1])), c2p,
-                             tc::pk2(cv.x, cv.y));
-        xp[2 * q + 1] = tc::fma2(tc::pk2(__uint_as_float(u[4 * q + 2]), __uint_as_float(u[4 * q + 3])), c2p,
-                                 tc::pk2(cv.z, cv.w));
-        if (FB) {
-            xp[2 * q] = tc::add2(xp[2 * q], dp);
-            xp[2 * q + 1] = tc::add2(xp[2 * q + 1], dp);
-        }
-    }
+    for (int j = 0; j < 16; ++j)
+        xp[j] = tc::fma2(tc::pk2(__uint_as_float(u[2 * j]), __uint_as_float(u[2 * j + 1])), c2p, srp);
     float e[32];
 #pragma unroll
     for (int j = 0; j < 16; ++j) {
@@ -226,7 +257,6 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_rowsum_sweep(const SweepArgs a
     uint64_t* bar = reinterpret_cast<uint64_t*>(sm + OFF_BAR);
     uint32_t* tbase = reinterpret_cast<uint32_t*>(sm + OFF_BAR + NBAR * 8);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tbase + 1);
-    float* cvring = reinterpret_cast<float*>(sm + OFF_CV);
     float* wring = reinterpret_cast<float*>(sm + OFF_WV);
     float* red = reinterpret_cast<float*>(sm + OFF_RED);
     RowInfo* rinfo = reinterpret_cast<RowInfo*>(sm + OFF_RI);
@@ -254,7 +284,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_rowsum_sweep(const SweepArgs a
             tc::mbar_init(bar + B_AEMPTY + i, 1);
         }
         for (int s = 0; s < NRING; ++s) {
-            tc::mbar_init(bar + B_FULL + s, 33);      // the TMA bytes + 32 column-vector lanes
+            // the TMA bytes (+ the 32 weight lanes)
+            tc::mbar_init(bar + B_FULL + s, MODE == WSUM ? 33 : 1);
             tc::mbar_init(bar + B_EMPTY + s, 1 + 4 * nch);  // the last MMA + 4 warps x nch uses
         }
         for (int b = 0; b < 4; ++b) {
@@ -269,6 +300,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_rowsum_sweep(const SweepArgs a
             tc::mbar_init(bar + B_QFULL + i, NEPI);   // every epilogue warp's partial row sums
             tc::mbar_init(bar + B_QEMPTY + i, 1);     // the finisher has read them
         }
+        tc::mbar_init(bar + B_ONES, 1);
         tc::mbar_init(bar + B_DRAIN, 1);
         *abort_flag = 0;
         tc::fence_mbar_init();
@@ -287,6 +319,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_rowsum_sweep(const SweepArgs a
         if (lane == 0) {
             tc::prefetch_tmap(&maps.A);
             tc::prefetch_tmap(&maps.B);
+            tc::prefetch_tmap(&maps.BA);
+            tc::prefetch_tmap(&maps.AO);
+            tc::mbar_expect_tx(bar + B_ONES, AUGB);
+            tc::tma_load_3d(sm + OFF_ONES, &maps.AO, bar + B_ONES, 0, 0, 0);
         }
         ChunkIds ids;
         int issued = 0, a_issued = 0, pbh = -1, prb = -1;
@@ -334,8 +370,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_rowsum_sweep(const SweepArgs a
                 if (id >= NRING && !ctl.wait(B_EMPTY + s, ((id / NRING) - 1) & 1)) { ok = false; break; }
                 const int col0 = r0 - W + 128 * c;
                 if (lane == 0 && SA_BOUNDS(s < NRING && col0 >= -W - 128 && col0 < L + W + 128, status)) {
-                    tc::mbar_expect_tx(bar + B_FULL + s, TILE);
+                    tc::mbar_expect_tx(bar + B_FULL + s, TILE + AUGB);
                     tc::tma_load_3d(sm + OFF_K + s * TILE, &maps.B, bar + B_FULL + s, 0, col0, bh);
+                    tc::tma_load_3d(sm + OFF_AUG + s * AUGB, &maps.BA, bar + B_FULL + s, 0, col0, bh);
                     // The slot is released once every tile that reads the chunk has
                     // (each use arrives 4 times, the last use's MMA once): the uses
                     // are this tile and the successors that follow it, at most c of
@@ -354,39 +391,43 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_rowsum_sweep(const SweepArgs a
                     if (uses < nch) tc::mbar_arrive_cnt(bar + B_EMPTY + s, 4 * (nch - uses));
                 }
                 issued = id + 1;
-                // working column duals and WSUM weights; zero off [0, L)
+                if (MODE == WSUM) {  // the weights, zero off [0, L)
 #pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const int col = col0 + 32 * k + lane;
-                    const bool in = col >= 0 && col < L;
-                    tc::cp_async4(&cvring[s * 128 + 32 * k + lane],
-                                  a.cdw.p + (long long)bh * a.cdw.s + (in ? col : 0), in);
-                    if (MODE == WSUM)
+                    for (int k = 0; k < 4; ++k) {
+                        const int col = col0 + 32 * k + lane;
+                        const bool in = col >= 0 && col < L;
                         tc::cp_async4(&wring[s * 128 + 32 * k + lane],
                                       a.w.p + (long long)bh * a.w.s + (in ? col : 0), in);
+                    }
+                    tc::cp_async_arrive(bar + B_FULL + s);
                 }
-                tc::cp_async_arrive(bar + B_FULL + s);
             }
         }
         asm volatile("cp.async.wait_all;" ::: "memory");  // nothing in flight at exit
-        if (lane == 0 && *abort_flag) {  // let issued loads land before teardown
-            for (int x = max(0, a_issued - 2); x < a_issued; ++x)
-                tc::mbar_wait(bar + B_AFULL + (x & 1), (x >> 1) & 1, kWaitBudget);
-            for (int x = max(0, issued - NRING); x < issued; ++x)
-                tc::mbar_wait(bar + B_FULL + x % NRING, (x / NRING) & 1, kWaitBudget);
+        if (lane == 0) {  // let issued loads land before teardown
+            tc::mbar_wait(bar + B_ONES, 0, kWaitBudget);
+            if (*abort_flag) {
+                for (int x = max(0, a_issued - 2); x < a_issued; ++x)
+                    tc::mbar_wait(bar + B_AFULL + (x & 1), (x >> 1) & 1, kWaitBudget);
+                for (int x = max(0, issued - NRING); x < issued; ++x)
+                    tc::mbar_wait(bar + B_FULL + x % NRING, (x / NRING) & 1, kWaitBudget);
+            }
         }
         __syncwarp();
     } else if (warp == W_MMA) {
         // ------------------------------------------------------------ MMA issuer
         // The whole warp runs the loop (uniform control flow and values); one
-        // elected lane issues the MMAs and commits.
+        // elected lane issues the MMAs and commits.  A chunk's scores are four
+        // K16 steps of Q K^T and a fifth that adds the column duals.
         const uint32_t id_s = tc::idesc_bf16(128, 128, false, false);
         const uint64_t dA0 = tc::sdesc_sw128(tc::smem_u32(sm + OFF_A), 16, 1024);
         const uint64_t dK0 = tc::sdesc_sw128(tc::smem_u32(sm + OFF_K), 16, 1024);
+        const uint64_t dOnes = tc::sdesc_sw32(tc::smem_u32(sm + OFF_ONES));
+        const uint64_t dAug0 = tc::sdesc_sw32(tc::smem_u32(sm + OFF_AUG));
         ChunkIds ids;
         int g = 0, pbh = -1, prb = -1;
         int nb[4] = {0, 0, 0, 0};  // uses of each TMEM buffer so far
-        bool ok = true;
+        bool ok = ctl.wait(B_ONES, 0);
         Cursor cur = cur0;
         for (int it = 0; ok && it < ntl; ++it) {
             const int bh = cur.b * H + cur.h;
@@ -413,6 +454,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_rowsum_sweep(const SweepArgs a
                     for (int k = 0; k < 4; ++k)
                         tc::mma_bf16(tS + 128 * b, tc::sdesc_add(dA, 32 * k), tc::sdesc_add(dB, 32 * k),
                                      id_s, k > 0);
+                    tc::mma_bf16(tS + 128 * b, dOnes, tc::sdesc_add(dAug0, s * AUGB), id_s, 1u);
                     tc::tc_commit(bar + B_SFULL + b);
                     if (!next_succ || c == 0) tc::tc_commit(bar + B_EMPTY + s);  // its last reader
                 }
@@ -429,9 +471,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_rowsum_sweep(const SweepArgs a
     } else if (warp == W_FIN) {
         // ------------------------------------------------------------ finisher
         // Each tile's outputs from the four parts' partial row sums; lane l
-        // writes rows 32k + l.  The shift of a quadrant is formed as the
-        // epilogue forms it (the smallest working dual of its valid rows,
-        // per-row shifts past a spread of 64).
+        // writes rows 32k + l.  An LSE sweep also writes its output's working
+        // copy and operand row for the sweep after it.
+        const float inv_c2 = 1.f / a.c2;
         Cursor cur = cur0;
         for (int it = 0; it < ntl; ++it, cur.next(nblk, H)) {
             const int bh = cur.b * H + cur.h, r0 = cur.rb * 128, slot = it % NRED;
@@ -444,28 +486,24 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_rowsum_sweep(const SweepArgs a
                 const int lr = 32 * k + lane, r = r0 + lr;
                 const float rwv = ri.rw[lr];
                 const bool valid = r < L && rwv != -INFINITY;
-                const float sr = valid ? rwv : 0.f;
-                float mn = valid ? sr : INFINITY, mx = valid ? sr : -INFINITY;
-                asm("redux.sync.min.f32 %0, %0, 0xffffffff;" : "+f"(mn));
-                asm("redux.sync.max.f32 %0, %0, 0xffffffff;" : "+f"(mx));
-                const float sq = mn == INFINITY ? 0.f : mn;
-                const bool fb = mn != INFINITY && mx - mn > kFallbackSpread;
-                const float seff = (fb && valid) ? sr : sq;
                 const float tot = (rs[lr] + rs[128 + lr]) + (rs[256 + lr] + rs[384 + lr]);
                 if (r < L && SA_BOUNDS(bh < BH, status)) {
                     float out = 0.f, outw = -INFINITY;
                     if (valid) {
                         if (MODE == LSE) {
-                            outw = seff - lg2(tot);
+                            outw = rwv - lg2(tot);
                             out = outw * kLn2;
                         } else {
                             const float bb = ri.base[lr];
                             const float mu = a.mult.p ? ri.mult[lr] : 1.f;
-                            out = bb + a.sgn * mu * (tot * ex2(sr - seff));
+                            out = bb + a.sgn * mu * tot;
                         }
                     }
                     a.out_vec.at(bh, r) = out;
                     if (MODE == LSE && a.outw.p) a.outw.at(bh, r) = outw;
+                    if (MODE == LSE && a.augo)
+                        put_aug(reinterpret_cast<__nv_bfloat16*>(a.augo) + (long long)bh * a.aug_s + 16LL * r,
+                                valid, outw * inv_c2);
                 }
             }
             __syncwarp();
@@ -478,8 +516,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_rowsum_sweep(const SweepArgs a
         // ------------------------------------------------------------ epilogue
         const int qd = warp & 3, pt = warp >> 2;
         const uint32_t lanebase = (uint32_t)(qd * 32) << 16;
-        float* scr = reinterpret_cast<float*>(sm + OFF_SCR) + warp * 128;
-        const float c2 = a.c2;
+        const uint64_t c2p = tc::pk2(a.c2, a.c2);
         ChunkIds ids;
         int g = 0, pbh = -1, prb = -1;
         int nu = 0;  // chunks this part has processed (uses of its TMEM buffer)
@@ -493,43 +530,28 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_rowsum_sweep(const SweepArgs a
             ids.advance(succ, nch);
             Cursor nx = cur;
             nx.next(nblk, H);
-            // this thread's row and the warp's shift (the smallest working dual of
-            // the quadrant's valid rows; per-row shifts past a spread of 64)
+            // this thread's row and its shift (its working dual; -inf on an
+            // invalid row, whose sum is not used)
             const int rw0 = r0 + qd * 32, r = rw0 + lane;
             if (!ctl.wait(B_RFULL + it % NRI, (it / NRI) & 1)) { ok = false; break; }
-            const RowInfo& ri = rinfo[it % NRI];
-            const float rwv = ri.rw[qd * 32 + lane];
-            const bool valid = r < L && rwv != -INFINITY;
-            const float sr = valid ? rwv : 0.f;
+            const float rwv = rinfo[it % NRI].rw[qd * 32 + lane];
             __syncwarp();
             if (lane == 0) tc::mbar_arrive(bar + B_REMPTY + it % NRI);
-            float mn = valid ? sr : INFINITY, mx = valid ? sr : -INFINITY;
-            asm("redux.sync.min.f32 %0, %0, 0xffffffff;" : "+f"(mn));
-            asm("redux.sync.max.f32 %0, %0, 0xffffffff;" : "+f"(mx));
-            const float sq = mn == INFINITY ? 0.f : mn;
-            const bool fb = mn != INFINITY && mx - mn > kFallbackSpread;
-            const float seff = (fb && valid) ? sr : sq;  // this row's shift
-            const float delta = seff - sq;
+            const float sr = r < L ? rwv : -INFINITY;
+            const uint64_t srp = tc::pk2(sr, sr);
             uint64_t acc[4] = {0, 0, 0, 0};
-            // this part's chunks of the tile: c = c0, c0 + 4, ...
+            // this part's chunks of the tile: c = c0, c0 + 4, ...; chunk g_t + c
+            // goes to part (g_t + c + rot * it) % 4, in that part's own TMEM
+            // buffer, whose phases its one part consumes in order
             const int g_t = g;
             g += nch;
             for (int c = (pt - (g_t + rot * it)) & 3; c < nch; c += 4) {
-                const int gg = g_t + c;
-                // chunk gg of tile it goes to part (gg + rot * it) % 4, in that
-                // part's own TMEM buffer, whose phases its one part consumes in
-                // order
                 const int id = ids.base + c, s = id % NRING, b = pt;
-                (void)gg;
                 if (!ctl.wait(B_SFULL + b, nu & 1)) { ok = false; break; }
                 ++nu;
-                if (!ctl.wait(B_FULL + s, (id / NRING) & 1)) { ok = false; break; }
+                if (MODE == WSUM && !ctl.wait(B_FULL + s, (id / NRING) & 1)) { ok = false; break; }
                 tc::tc_fence_after();
                 const int col0 = r0 - W + 128 * c;
-                // this warp's copy of the chunk's column duals with its shift added
-#pragma unroll
-                for (int k = 0; k < 4; ++k) scr[32 * k + lane] = cvring[s * 128 + 32 * k + lane] + sq;
-                __syncwarp();
                 const float* wv = wring + s * 128;
 #pragma unroll 1
                 for (int gr = 0; gr < 4; ++gr) {
@@ -541,17 +563,11 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_rowsum_sweep(const SweepArgs a
                     if (SA_BOUNDS(128 * b + 32 * gr + 32 <= 512, status))
                         tc::tmem_ld32(tS + 128 * b + lanebase + 32 * gr, u);
                     tc::tmem_wait_ld();
-                    const float* cs = scr + 32 * gr;
                     const float* ws = wv + 32 * gr;
                     // this row's band and [0, L), as local columns of the group
                     const int lo = max(r - W, 0) - cg, hi = min(r + W, L - 1) - cg;
-                    if (fb) {
-                        if (all_in) group<MODE, KP, false, true>(u, cs, ws, c2, delta, lo, hi, acc);
-                        else group<MODE, KP, true, true>(u, cs, ws, c2, delta, lo, hi, acc);
-                    } else {
-                        if (all_in) group<MODE, KP, false, false>(u, cs, ws, c2, 0.f, lo, hi, acc);
-                        else group<MODE, KP, true, false>(u, cs, ws, c2, 0.f, lo, hi, acc);
-                    }
+                    if (all_in) group<MODE, KP, false>(u, ws, c2p, srp, lo, hi, acc);
+                    else group<MODE, KP, true>(u, ws, c2p, srp, lo, hi, acc);
                 }
                 // every TMEM read and shared-memory read of the chunk is done
                 tc::tc_fence_before();
