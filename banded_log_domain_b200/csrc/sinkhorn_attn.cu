@@ -585,8 +585,14 @@ int sm_count() {
 
 // Exponentials of every 32 entries of a row-sum sweep's in-band group that run
 // on the FMA pipe (the rest on the MUFU unit).
-#ifndef SA_ROWSUM_KP
-#define SA_ROWSUM_KP 0
+// Exponentials per 32 on the FMA pipe (the rest on MUFU) in the row-sum sweeps'
+// in-band groups: measured on long32k, 8 of 32 takes 1-4 % off an LSE sweep
+// (W 256-320) and slows WSUM, whose epilogue has more FMA work of its own.
+#ifndef SA_ROWSUM_KP_LSE
+#define SA_ROWSUM_KP_LSE 8
+#endif
+#ifndef SA_ROWSUM_KP_WSUM
+#define SA_ROWSUM_KP_WSUM 0
 #endif
 
 // The row-sum sweeps (shifted LSE, WSUM) on the tensor cores: persistent, one
@@ -604,7 +610,7 @@ cudaError_t launch_rowsum(const simt::SweepArgs& a, int BH, cudaStream_t st, Tra
         return cudaErrorInvalidValue;
     const long long ntiles = (long long)((a.L + 127) / 128) * BH;
     const dim3 grid((unsigned)std::min<long long>(ntiles, (long long)sm_count()));
-    auto kern = tcr::tc_rowsum_sweep<MODE, SA_ROWSUM_KP>;
+    auto kern = tcr::tc_rowsum_sweep<MODE, MODE == simt::LSE ? SA_ROWSUM_KP_LSE : SA_ROWSUM_KP_WSUM>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          tcr::SMEM_BYTES);
     if (e != cudaSuccess) return e;

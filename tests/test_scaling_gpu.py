@@ -91,10 +91,16 @@ def test_extra_memory_is_linear_in_L_and_independent_of_W():
     Ls = [8192, 16384, 32768]
     for W in (32, 256):
         m = [extra(L, W) for L in Ls]
-        # linear in L: doubling L doubles the extra memory (within allocator rounding)
-        assert abs(m[1] / m[0] - 2.0) < 0.02 and abs(m[2] / m[1] - 2.0) < 0.02, m
+        # affine in L: the increment from 2L to 4L is twice the one from L to 2L
+        # (to 1 %), and the intercept is within the caching allocator's rounding
+        # (its blocks are 2 MiB)
+        d1, d2 = m[1] - m[0], m[2] - m[1]
+        assert abs(d2 / d1 - 2.0) < 0.01, m
+        assert abs(m[0] - d1) <= 4 << 20, m
+    # independent of W: no band-sized buffer anywhere
     assert extra(16384, 32) == extra(16384, 256)
-    # and it is O(L) with a small constant: outputs (4 d-vectors per token) plus
-    # the dual state and workspaces (tens of floats per token), far below L*W
+    # and O(L) with a small constant: the outputs (4 d-vectors of bf16 per token)
+    # plus the dual state, its working copies (a float and a 16-slot bf16 operand
+    # row per dual) and the backward's vectors, below 1 KiB per token and head
     per_token = extra(16384, 256) / (H * 16384)
-    assert per_token < 4 * 64 * 2 + 100 * 4, per_token
+    assert per_token < 4 * 64 * 2 + 128 * 4, per_token
