@@ -806,6 +806,7 @@ sa_status fwd_impl(const Ctx& x, const T* q, const T* k, const T* v, const uint8
     b.Xd = v_dust;
     b.rd = x.srow(2 * d.R);
     b.cd = x.srow(2 * d.R + 1);
+    b.cdw = x.wrow(2 * d.R + 1);
     b.out_mat = o;
     SA_CUDA((launch_sweep<T, simt::PV>(b, d.BH, x.st, x.tr, x.status)));
     return SA_OK;
@@ -856,6 +857,7 @@ sa_status bwd_impl(const Ctx& x, const T* q, const T* k, const T* v, const uint8
         a.A = k; a.Bo = q; a.X = dO; a.Y = v;
         a.Yd = v_dust;
         a.rd = vR; a.cd = uR;
+        a.cdw = x.wrow(2 * R);
         a.out_mat = dv;
         a.out_vec = mvec(vb(R), vs);
         a.dvd_part = dvd;
@@ -1008,6 +1010,7 @@ sa_status bwd_impl(const Ctx& x, const T* q, const T* k, const T* v, const uint8
             if (side == 0) {
                 a.A = q; a.Bo = k; a.A2 = dO; a.B2 = v; a.X = k;
                 a.rd = uR; a.cd = vR;
+                a.cdw = x.wrow(2 * R + 1);
                 a.out_mat = dq;
                 for (int t = 0; t < kn; ++t) {
                     a.rv[t] = rq[k0 + t]; a.cv[t] = rk[k0 + t];
@@ -1017,6 +1020,7 @@ sa_status bwd_impl(const Ctx& x, const T* q, const T* k, const T* v, const uint8
             } else {
                 a.A = k; a.Bo = q; a.A2 = v; a.B2 = dO; a.X = q;
                 a.rd = vR; a.cd = uR;
+                a.cdw = x.wrow(2 * R);
                 a.out_mat = dk;
                 for (int t = 0; t < kn; ++t) {
                     a.rv[t] = rk[k0 + t]; a.cv[t] = rq[k0 + t];

@@ -126,9 +126,9 @@ __device__ __forceinline__ float* colvec(uint8_t* sm, int mode, int nt, int s, i
 }
 
 // Exponent arguments (log2 units) of one thread's 32 columns:
-// x_j = c2 * s_j + (ce_j + rd2), -inf off the band when `partial`.
+// x_j = c2 * s_j + (ce_j + rd2), -inf off the band or past L when `partial`.
 __device__ __forceinline__ void group_args(const float (&sv)[32], const float* ce, float rd2,
-                                           float c2, bool partial, int r, int cg, int W,
+                                           float c2, bool partial, int r, int cg, int W, int L,
                                            float (&x)[32]) {
     const uint64_t c2p = tc::pk2(c2, c2), rdp = tc::pk2(rd2, rd2);
     const float4* c4 = reinterpret_cast<const float4*>(ce);
@@ -145,7 +145,7 @@ __device__ __forceinline__ void group_args(const float (&sv)[32], const float* c
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
             const int d = r - (cg + j);
-            if ((unsigned)(d + W) > (unsigned)(2 * W)) x[j] = -INFINITY;
+            if ((unsigned)(d + W) > (unsigned)(2 * W) || cg + j >= L) x[j] = -INFINITY;
         }
     }
 }
@@ -172,6 +172,8 @@ __global__ void __launch_bounds__(nthreads(MODE), ctas_per_sm(MODE)) tc_band_swe
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tbase + 1);
     float* red = reinterpret_cast<float*>(sm + off_red(MODE, NT));
     constexpr bool AUG = aug(MODE, NT);
+    // the column dual is the chunk's only column vector
+    constexpr bool CPA = MODE == LSE || MODE == PV || (MODE == DS1 && AUG);
     Ctl ctl{bar, abort_flag, status};
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -279,7 +281,23 @@ __global__ void __launch_bounds__(nthreads(MODE), ctas_per_sm(MODE)) tc_band_swe
                                         bar + B_FULL + s, 0, c0, bh);
                     if (MODE == PV) tc::tma_load_3d(st + TILE, &maps.X, bar + B_FULL + s, 0, c0, bh);
                 }
-                // column vectors: -inf / 0 outside [cbeg, cend) and on masked columns.
+                // Column vectors.  The modes whose only one is the column dual copy it
+                // from its working copy (log2(e) times the dual, -inf on masked
+                // tokens) by 4-byte cp.async, counted on the stage's mbarrier, so the
+                // loader never waits for a global load; columns past L are
+                // zero-filled and excluded by the epilogue's band test.
+                if (CPA && a.cdw.p) {
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const int col = c0 + 32 * k + lane;
+                        const bool in = col < L;
+                        tc::cp_async4(colvec(sm, MODE, NT, s, 0) + 32 * k + lane,
+                                      a.cdw.p + (long long)bh * a.cdw.s + (in ? col : 0), in);
+                    }
+                    tc::cp_async_arrive(bar + B_FULL + s);
+                    continue;
+                }
+                // Otherwise: -inf / 0 outside [cbeg, cend) and on masked columns.
                 // Every load of the chunk (4 columns per lane, each vector, the mask)
                 // is issued before any value is used or stored.
                 {
@@ -333,6 +351,7 @@ __global__ void __launch_bounds__(nthreads(MODE), ctas_per_sm(MODE)) tc_band_swe
                 tc::mbar_arrive(bar + B_FULL + s);
             }
         }
+        asm volatile("cp.async.wait_all;" ::: "memory");  // nothing in flight at exit
         // after an abort, let the tile loads already issued land before teardown
         if (lane == 0 && *abort_flag) {
             for (int x = max(0, a_issued - NAB); x < a_issued; ++x)
@@ -523,20 +542,9 @@ __global__ void __launch_bounds__(nthreads(MODE), ctas_per_sm(MODE)) tc_band_swe
             const int bh = tl.bh, r0 = tl.r0, cbeg = tl.cbeg, nch = tl.nch;
             const int r = r0 + lr;              // global row
             const int rw0 = r0 + qd * 32;       // first row of this warp
-            // PV with a row dot: this thread's slice of the Y row; WSUM: the output's
-            // base and multiplier.  Loaded now, used after the chunk loop.
-            uint4 yq[MODE == PV ? OWY / 8 : 1];
+            // WSUM: the output's base and multiplier, loaded now, used after the
+            // chunk loop
             float bb = 0.f, mu = 1.f;
-            if (MODE == PV) {
-#pragma unroll
-                for (int q = 0; q < (MODE == PV ? OWY / 8 : 1); ++q) yq[q] = make_uint4(0, 0, 0, 0);
-                if (a.Y && r < L) {
-                    const uint4* yp = reinterpret_cast<const uint4*>(
-                        reinterpret_cast<const __nv_bfloat16*>(a.Y) + ((size_t)bh * L + r) * 64 + OWY * pt);
-#pragma unroll
-                    for (int q = 0; q < (MODE == PV ? OWY / 8 : 1); ++q) yq[q] = yp[q];
-                }
-            }
             if (MODE == WSUM && r < L) {
                 bb = a.base.p ? a.base.at(bh, r) : 0.f;
                 mu = a.mult.p ? a.mult.at(bh, r) : 1.f;
@@ -596,8 +604,8 @@ __global__ void __launch_bounds__(nthreads(MODE), ctas_per_sm(MODE)) tc_band_swe
                     }
                     // band test for this warp's 32 rows x these 32 columns (warp-uniform)
                     const int cg = c0 + PW * pt + 32 * g;
-                    const bool all_in = (cg >= rw0 + 31 - W) && (cg + 31 <= rw0 + W);
-                    const bool all_out = (cg + 31 < rw0 - W) || (cg > rw0 + 31 + W);
+                    const bool all_in = (cg >= rw0 + 31 - W) && (cg + 31 <= rw0 + W) && cg + 31 < L;
+                    const bool all_out = (cg + 31 < rw0 - W) || (cg > rw0 + 31 + W) || cg >= L;
                     const float* ce = cvs + 32 * g;
                     if (MODE == LSE || MODE == WSUM || MODE == PV) {
                         if (all_out) {
@@ -607,7 +615,7 @@ __global__ void __launch_bounds__(nthreads(MODE), ctas_per_sm(MODE)) tc_band_swe
                             }
                         } else {
                             float x[32];
-                            group_args(sv, ce, rd2, c2, !all_in, r, cg, W, x);
+                            group_args(sv, ce, rd2, c2, !all_in, r, cg, W, L, x);
                             if (MODE == LSE && ONLINE) {
                                 float mloc = -INFINITY;
     #pragma unroll
@@ -649,13 +657,13 @@ __global__ void __launch_bounds__(nthreads(MODE), ctas_per_sm(MODE)) tc_band_swe
                     } else if (MODE == DS1 && AUG) {
                         // dS = P * M, M = G + sum_k rv_k[row] cv_k[col] from the contraction
                         float x[32];
-                        group_args(sv, ce, rd2, c2, !all_in, r, cg, W, x);
+                        group_args(sv, ce, rd2, c2, !all_in, r, cg, W, L, x);
     #pragma unroll
                         for (int j = 0; j < 32; ++j) pv[j] = ex2(x[j]) * gv[j];
                     } else if (MODE == DS1) {
                         // dS = P * M,  M = G + sum_k rv_k[row] cv_k[col]
                         float x[32];
-                        group_args(sv, ce, rd2, c2, !all_in, r, cg, W, x);
+                        group_args(sv, ce, rd2, c2, !all_in, r, cg, W, L, x);
     #pragma unroll
                         for (int q = 0; q < 8; ++q) {
                             uint64_t m01 = tc::pk2(gv[4 * q], gv[4 * q + 1]);
@@ -798,6 +806,19 @@ __global__ void __launch_bounds__(nthreads(MODE), ctas_per_sm(MODE)) tc_band_swe
                 // of its lanes, then frees the buffer for tile it + 2
                 constexpr int OW = 64 / NPART;
                 const int ob = it & 1;
+                // PV with a row dot: this thread's slice of the Y row, loaded while
+                // the tile's last P X contraction completes
+                uint4 yq[MODE == PV ? OWY / 8 : 1];
+                if (MODE == PV) {
+#pragma unroll
+                    for (int q = 0; q < (MODE == PV ? OWY / 8 : 1); ++q) yq[q] = make_uint4(0, 0, 0, 0);
+                    if (a.Y && r < L) {
+                        const uint4* yp = reinterpret_cast<const uint4*>(
+                            reinterpret_cast<const __nv_bfloat16*>(a.Y) + ((size_t)bh * L + r) * 64 + OWY * pt);
+#pragma unroll
+                        for (int q = 0; q < (MODE == PV ? OWY / 8 : 1); ++q) yq[q] = yp[q];
+                    }
+                }
                 if (!ctl.wait(B_OFULL + ob, (it >> 1) & 1)) { ok = false; break; }
                 float o[OW];
                 {
