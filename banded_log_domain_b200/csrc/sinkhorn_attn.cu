@@ -551,6 +551,12 @@ cudaError_t launch_tc(const simt::SweepArgs& a, int BH, cudaStream_t st, Tracer&
     if (MODE == simt::PV) ok = ok && make_map(&maps.X, a.X, a.L, BH);
     if (tcs::aug(MODE, NT))
         ok = ok && make_map_aug(&maps.AR, a.aug_row, a.L, BH) && make_map_aug(&maps.AC, a.aug_col, a.L, BH);
+    if (tcs::augs(MODE)) {  // the constant row-block operand and the column duals' rows
+        void* ones = nullptr;
+        ok = ok && cudaGetSymbolAddress(&ones, tcr::g_aug_ones) == cudaSuccess && ones &&
+             make_map_aug_strided(&maps.AR, ones, 128, 1, 128 * 16) &&
+             make_map_aug_strided(&maps.AC, a.augc, a.L, BH, a.aug_s);
+    }
     if (!ok) return cudaErrorInvalidValue;
     // persistent: one CTA per SM (two for LSE and WSUM), each a contiguous tile range
     static int nsm = 0;
@@ -807,6 +813,8 @@ sa_status fwd_impl(const Ctx& x, const T* q, const T* k, const T* v, const uint8
     b.rd = x.srow(2 * d.R);
     b.cd = x.srow(2 * d.R + 1);
     b.cdw = x.wrow(2 * d.R + 1);
+    b.augc = x.augrow(2 * d.R + 1);
+    b.aug_s = x.aug_stride();
     b.out_mat = o;
     SA_CUDA((launch_sweep<T, simt::PV>(b, d.BH, x.st, x.tr, x.status)));
     return SA_OK;
@@ -858,6 +866,8 @@ sa_status bwd_impl(const Ctx& x, const T* q, const T* k, const T* v, const uint8
         a.Yd = v_dust;
         a.rd = vR; a.cd = uR;
         a.cdw = x.wrow(2 * R);
+        a.augc = x.augrow(2 * R);
+        a.aug_s = x.aug_stride();
         a.out_mat = dv;
         a.out_vec = mvec(vb(R), vs);
         a.dvd_part = dvd;

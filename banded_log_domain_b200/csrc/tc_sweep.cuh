@@ -4,9 +4,9 @@
 // the band contractions on the 5th-generation tensor cores:
 //   S  = A_blk B_chunk^T   128 x 128 x 64, bf16 in, fp32 accumulation in TMEM
 //   G  = A2_blk B2_chunk^T (dS sweeps only)
-//   O += P X_chunk         128 x 64 x 128, P (or dS) rounded to bf16 and staged
-//                          in shared memory in the 128-byte-swizzled K-major
-//                          layout, X read MN-major straight from its TMA tile.
+//   O += P X_chunk         128 x 64 x 128, P (or dS) rounded to bf16 and stored
+//                          in TMEM (two bf16 per column, the contraction's A
+//                          operand), X read MN-major straight from its TMA tile.
 // One CTA owns a block of 128 rows (TMEM lanes) of one (batch, head) problem
 // and walks the band's column chunks [r0 - W, r0 + 127 + W] in steps of 128.
 //
@@ -50,7 +50,10 @@ struct Maps {
 
 __host__ __device__ constexpr bool is_ds(int m) { return m == DS1 || m == DSD; }
 __host__ __device__ constexpr bool has_x(int m) { return m == PV || is_ds(m); }
-__host__ __device__ constexpr int nst(int m) { return is_ds(m) ? 3 : (m == PV ? 3 : 4); }
+// operand stages: five for PV and DS1 (their P tiles live in TMEM, which leaves
+// the shared memory to the stages), four for the others
+constexpr int NST_MAX = 5;
+__host__ __device__ constexpr int nst(int m) { return (m == PV || m == DS1) ? 5 : 4; }
 __host__ __device__ constexpr int nsb(int m) { return is_ds(m) ? 1 : 2; }
 // DS1 with at most five modifier terms adds the modifier to G on the tensor
 // core: one more K16 step of the dO V^T contraction whose operands, prepared
@@ -60,6 +63,12 @@ __host__ __device__ constexpr int nsb(int m) { return is_ds(m) ? 1 : 2; }
 //   sum_k rv_k cv_k ~ sum_k rv_hi cv_hi + rv_hi cv_lo + rv_lo cv_hi
 // to about 2^-16 of each product, far below the bf16 rounding of dS.
 __host__ __device__ constexpr bool aug(int m, int nt) { return m == DS1 && nt > 0 && 3 * nt <= 16; }
+// PV adds the column dual to its scores the same way, in one more K16 step of
+// the score contraction: a constant row-block operand [1, 1, 1, 0, ...] against
+// the chunk's operand rows, which hold a three-way bf16 split of dual / c (c the
+// score scale; -1e30 on masked tokens), so its epilogue reads no column vector.
+__host__ __device__ constexpr bool augs(int m) { return m == PV; }
+__host__ __device__ constexpr bool has_aug(int m, int nt) { return aug(m, nt) || augs(m); }
 // column vectors staged per operand stage
 __host__ __device__ constexpr int ncv(int m, int nt) {
     return m == WSUM ? 2 : (m == DS1 ? (aug(m, nt) ? 1 : 1 + nt) : (m == DSD ? 2 * MAXT : 1));
@@ -79,8 +88,7 @@ __host__ __device__ constexpr int ctas_per_sm(int m) { return (m == LSE || m == 
 __host__ __device__ constexpr int off_a(int m, int i) { return TILE * i; }
 __host__ __device__ constexpr int off_a2(int m) { return TILE; }
 __host__ __device__ constexpr int off_stage(int m) { return 2 * TILE; }
-__host__ __device__ constexpr int off_p(int m) { return off_stage(m) + nst(m) * stage_bytes(m); }
-__host__ __device__ constexpr int off_cv(int m) { return off_p(m) + (has_x(m) ? 2 * 2 * TILE : 0); }
+__host__ __device__ constexpr int off_cv(int m) { return off_stage(m) + nst(m) * stage_bytes(m); }
 // the modifier's K16 operand tiles (aug): the row block's, then one per operand
 // stage, 4 KB each (128 rows x 32 bytes), 1024-aligned
 constexpr int AUG_BYTES = 4096;
@@ -88,15 +96,16 @@ __host__ __device__ constexpr int off_aug(int m, int nt) {
     return (off_cv(m) + nst(m) * ncv(m, nt) * 128 * 4 + 1023) / 1024 * 1024;
 }
 __host__ __device__ constexpr int off_red(int m, int nt) {
-    return aug(m, nt) ? off_aug(m, nt) + (1 + nst(m)) * AUG_BYTES : off_cv(m) + nst(m) * ncv(m, nt) * 128 * 4;
+    return has_aug(m, nt) ? off_aug(m, nt) + (1 + nst(m)) * AUG_BYTES : off_cv(m) + nst(m) * ncv(m, nt) * 128 * 4;
 }
 __host__ __device__ constexpr int off_bar(int m, int nt) { return off_red(m, nt) + 2 * 4 * 128 * 4; }
 __host__ __device__ constexpr int smem_bytes(int m, int nt) { return off_bar(m, nt) + 64 * 8 + 64 + 1024; }
 
 // barrier slots (pairs indexed by tile parity, chunk parity or buffer)
-enum { B_AFULL = 0, B_AEMPTY = 2, B_FULL = 4, B_EMPTY = 8, B_SFULL = 12, B_SEMPTY = 14,
-       B_PFULL = 16, B_PEMPTY = 18, B_OFULL = 20, B_OEMPTY = 22, B_DRAIN = 24, B_EPI = 25,
-       NBAR = 26 };
+enum { B_AFULL = 0, B_AEMPTY = 2, B_FULL = 4, B_EMPTY = B_FULL + NST_MAX, B_SFULL = B_EMPTY + NST_MAX,
+       B_SEMPTY = B_SFULL + 2, B_PFULL = B_SEMPTY + 2, B_PEMPTY = B_PFULL + 2, B_OFULL = B_PEMPTY + 2,
+       B_OEMPTY = B_OFULL + 2, B_DRAIN = B_OEMPTY + 2, B_EPI = B_DRAIN + 1, NBAR = B_EPI + 1 };
+static_assert(NBAR <= 64, "barrier area");
 
 struct Ctl {
     uint64_t* bar;
@@ -150,6 +159,23 @@ __device__ __forceinline__ void group_args(const float (&sv)[32], const float* c
     }
 }
 
+// The same with the column dual already in the score (s_j' = s_j + ce_j / c2):
+// x_j = c2 * s_j' + rd2.
+__device__ __forceinline__ void group_args_s(const float (&sv)[32], float rd2, float c2, bool partial,
+                                             int r, int cg, int W, int L, float (&x)[32]) {
+    const uint64_t c2p = tc::pk2(c2, c2), rdp = tc::pk2(rd2, rd2);
+#pragma unroll
+    for (int q = 0; q < 16; ++q)
+        tc::upk2(tc::fma2(tc::pk2(sv[2 * q], sv[2 * q + 1]), c2p, rdp), x[2 * q], x[2 * q + 1]);
+    if (partial) {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+            const int d = r - (cg + j);
+            if ((unsigned)(d + W) > (unsigned)(2 * W) || cg + j >= L) x[j] = -INFINITY;
+        }
+    }
+}
+
 // ---------------------------------------------------------------------------
 // NT: number of modifier (DS1) or staircase (DSD) terms, 2R; 0 for the other modes.
 // Persistent: each CTA walks a contiguous range of (problem, row block) tiles;
@@ -171,9 +197,12 @@ __global__ void __launch_bounds__(nthreads(MODE), ctas_per_sm(MODE)) tc_band_swe
     uint32_t* tbase = reinterpret_cast<uint32_t*>(sm + off_bar(MODE, NT) + 64 * 8);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tbase + 1);
     float* red = reinterpret_cast<float*>(sm + off_red(MODE, NT));
-    constexpr bool AUG = aug(MODE, NT);
+    constexpr bool AUG = aug(MODE, NT), AUGS = augs(MODE), HAUG = has_aug(MODE, NT);
+    static_assert(smem_bytes(MODE, NT) <= 227 * 1024 && smem_bytes(MODE, NT) * ctas_per_sm(MODE) <= 228 * 1024,
+                  "shared memory");
+    static_assert(NST <= NST_MAX, "stage barriers");
     // the column dual is the chunk's only column vector
-    constexpr bool CPA = MODE == LSE || MODE == PV || (MODE == DS1 && AUG);
+    constexpr bool CPA = MODE == LSE || (MODE == DS1 && AUG);
     Ctl ctl{bar, abort_flag, status};
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -223,7 +252,7 @@ __global__ void __launch_bounds__(nthreads(MODE), ctas_per_sm(MODE)) tc_band_swe
             tc::mbar_init(bar + B_OEMPTY + i, NEPI);
         }
         for (int s = 0; s < NST; ++s) {
-            tc::mbar_init(bar + B_FULL + s, 33);
+            tc::mbar_init(bar + B_FULL + s, AUGS ? 1 : 33);  // the TMA bytes (+ 32 lanes' vectors)
             tc::mbar_init(bar + B_EMPTY + s, NEPI + 1);
         }
         tc::mbar_init(bar + B_DRAIN, 1);
@@ -239,8 +268,9 @@ __global__ void __launch_bounds__(nthreads(MODE), ctas_per_sm(MODE)) tc_band_swe
     __syncthreads();
     tc::tc_fence_after();
     const uint32_t tm = *tbase;
-    // TMEM columns: S buffer b at 128*b (DS: S at 0, G at 128); O buffer ob at 256 + 64*ob
-    const uint32_t tS = tm, tG = tm + 128, tO = tm + 256;
+    // TMEM columns: S buffer b at 128*b (DS: S at 0, G at 128); O buffer ob at
+    // 256 + 64*ob; P (or dS) buffer pb, 128 bf16 per row, at 384 + 64*pb
+    const uint32_t tS = tm, tG = tm + 128, tO = tm + 256, tP = tm + 384;
 
     if (warp == W_LOAD) {
         // ------------------------------------------------------------ loader
@@ -257,10 +287,14 @@ __global__ void __launch_bounds__(nthreads(MODE), ctas_per_sm(MODE)) tc_band_swe
             if (lane == 0) {
                 if (it >= NAB && !ctl.wait(B_AEMPTY + ab, ((it / NAB) - 1) & 1)) ok = false;
                 if (ok) {
-                    tc::mbar_expect_tx(bar + B_AFULL + ab, TILE * (DS ? 2 : 1) + (AUG ? AUG_BYTES : 0));
+                    // the row-block operand rows: per tile (DS1), or the constant one
+                    // once, with the first tile (PV)
+                    const bool ld_ar = AUG || (AUGS && it == 0);
+                    tc::mbar_expect_tx(bar + B_AFULL + ab, TILE * (DS ? 2 : 1) + (ld_ar ? AUG_BYTES : 0));
                     tc::tma_load_3d(sm + off_a(MODE, ab), &maps.A, bar + B_AFULL + ab, 0, tl.r0, tl.bh);
                     if (DS) tc::tma_load_3d(sm + off_a2(MODE), &maps.A2, bar + B_AFULL + ab, 0, tl.r0, tl.bh);
                     if (AUG) tc::tma_load_3d(sm + off_aug(MODE, NT), &maps.AR, bar + B_AFULL + ab, 0, tl.r0, tl.bh);
+                    if (AUGS && it == 0) tc::tma_load_3d(sm + off_aug(MODE, NT), &maps.AR, bar + B_AFULL + ab, 0, 0, 0);
                     a_issued = it + 1;
                 }
             }
@@ -273,14 +307,15 @@ __global__ void __launch_bounds__(nthreads(MODE), ctas_per_sm(MODE)) tc_band_swe
                 const uint8_t* mk = tl.mk;
                 uint8_t* st = sm + off_stage(MODE) + s * stage_bytes(MODE);
                 if (lane == 0) {
-                    tc::mbar_expect_tx(bar + B_FULL + s, stage_bytes(MODE) + (AUG ? AUG_BYTES : 0));
+                    tc::mbar_expect_tx(bar + B_FULL + s, stage_bytes(MODE) + (HAUG ? AUG_BYTES : 0));
                     tc::tma_load_3d(st, &maps.B, bar + B_FULL + s, 0, c0, bh);
                     if (DS) tc::tma_load_3d(st + TILE, &maps.B2, bar + B_FULL + s, 0, c0, bh);
-                    if (AUG)
+                    if (HAUG)
                         tc::tma_load_3d(sm + off_aug(MODE, NT) + AUG_BYTES * (1 + s), &maps.AC,
                                         bar + B_FULL + s, 0, c0, bh);
                     if (MODE == PV) tc::tma_load_3d(st + TILE, &maps.X, bar + B_FULL + s, 0, c0, bh);
                 }
+                if (AUGS) continue;  // no column vector
                 // Column vectors.  The modes whose only one is the column dual copy it
                 // from its working copy (log2(e) times the dual, -inf on masked
                 // tokens) by 4-byte cp.async, counted on the stage's mbarrier, so the
@@ -372,7 +407,6 @@ __global__ void __launch_bounds__(nthreads(MODE), ctas_per_sm(MODE)) tc_band_swe
             const uint64_t dA2 = tc::sdesc_sw128(tc::smem_u32(sm + off_a2(MODE)), 16, 1024);
             const uint64_t dStK = tc::sdesc_sw128(tc::smem_u32(sm + off_stage(MODE)), 16, 1024);
             const uint64_t dStMN = tc::sdesc_sw128(tc::smem_u32(sm + off_stage(MODE)), TILE, 1024);
-            const uint64_t dP = tc::sdesc_sw128(tc::smem_u32(sm + off_p(MODE)), 16, 1024);
             const uint64_t dAug = tc::sdesc_sw32(tc::smem_u32(sm + off_aug(MODE, NT)));
             // O += P X of chunk c (global chunk g) of tile it (nch chunks)
             auto issue_pv = [&](int g, int it, int c, int nch) -> bool {
@@ -382,12 +416,11 @@ __global__ void __launch_bounds__(nthreads(MODE), ctas_per_sm(MODE)) tc_band_swe
                 if (!ctl.wait(B_PFULL + pb, (g >> 1) & 1)) return false;
                 tc::tc_fence_after();
                 const uint64_t dX = tc::sdesc_add(dStMN, s * stage_bytes(MODE) + (MODE == PV ? TILE : 0));
-                const uint64_t dPb = tc::sdesc_add(dP, pb * 2 * TILE);
                 if (tc::elect_one()) {
 #pragma unroll
-                    for (int k = 0; k < 8; ++k) {
-                        tc::mma_bf16(tO + 64 * ob, tc::sdesc_add(dPb, (k >> 2) * TILE + (k & 3) * 32),
-                                     tc::sdesc_add(dX, k * 2048), id_o, (c > 0 || k > 0) ? 1u : 0u);
+                    for (int k = 0; k < 8; ++k) {  // A = P from TMEM, 16 chunk columns per step
+                        tc::mma_bf16_ts(tO + 64 * ob, tP + 64 * pb + 8 * k, tc::sdesc_add(dX, k * 2048), id_o,
+                                        (c > 0 || k > 0) ? 1u : 0u);
                     }
                     tc::tc_commit(bar + B_PEMPTY + pb);
                     tc::tc_commit(bar + B_EMPTY + s);
@@ -416,6 +449,8 @@ __global__ void __launch_bounds__(nthreads(MODE), ctas_per_sm(MODE)) tc_band_swe
                         for (int k = 0; k < 4; ++k)
                             tc::mma_bf16(tS + 128 * b, tc::sdesc_add(dA, 32 * k), tc::sdesc_add(dB, 32 * k),
                                          id_s, k > 0);
+                        if (AUGS)  // + the column duals
+                            tc::mma_bf16(tS + 128 * b, dAug, tc::sdesc_add(dAug, AUG_BYTES * (1 + s)), id_s, 1u);
                         if (DS) {
 #pragma unroll
                             for (int k = 0; k < 4; ++k)
@@ -449,7 +484,6 @@ __global__ void __launch_bounds__(nthreads(MODE), ctas_per_sm(MODE)) tc_band_swe
         const int qd = warp & 3, pt = warp >> 2;  // part pt: columns PW*pt..PW*pt+PW-1 of a chunk
         const int lr = qd * 32 + lane;            // local row
         const uint32_t lanebase = (uint32_t)(qd * 32) << 16;
-        uint8_t* Pb = sm + off_p(MODE);
         const float c2 = a.c2;
         constexpr int OWY = 64 / NPART;
         int gc = 0;
@@ -615,7 +649,8 @@ __global__ void __launch_bounds__(nthreads(MODE), ctas_per_sm(MODE)) tc_band_swe
                             }
                         } else {
                             float x[32];
-                            group_args(sv, ce, rd2, c2, !all_in, r, cg, W, L, x);
+                            if (AUGS) group_args_s(sv, rd2, c2, !all_in, r, cg, W, L, x);
+                            else group_args(sv, ce, rd2, c2, !all_in, r, cg, W, L, x);
                             if (MODE == LSE && ONLINE) {
                                 float mloc = -INFINITY;
     #pragma unroll
@@ -720,22 +755,20 @@ __global__ void __launch_bounds__(nthreads(MODE), ctas_per_sm(MODE)) tc_band_swe
                         }
                     }
                     if (HASX) {
+                        // the group's 32 columns as 16 bf16 pairs, at TMEM column
+                        // (chunk column) / 2 of the P buffer
                         const int jc = PW * pt + 32 * g;  // first column of the group within the chunk
-                        uint8_t* dst = Pb + pb * 2 * TILE + (jc >> 6) * TILE;
+                        uint32_t w[16];
     #pragma unroll
-                        for (int q = 0; q < 4; ++q) {
-                            uint4 w;
-                            w.x = tc::pack_bf16(pv[8 * q + 0], pv[8 * q + 1]);
-                            w.y = tc::pack_bf16(pv[8 * q + 2], pv[8 * q + 3]);
-                            w.z = tc::pack_bf16(pv[8 * q + 4], pv[8 * q + 5]);
-                            w.w = tc::pack_bf16(pv[8 * q + 6], pv[8 * q + 7]);
-                            if (SA_BOUNDS(pb * 2 * TILE + (jc >> 6) * TILE + (int)tc::sw128_off(lr, ((jc & 63) >> 3) + q) + 16 <= 2 * 2 * TILE, status))
-                                *reinterpret_cast<uint4*>(dst + tc::sw128_off(lr, ((jc & 63) >> 3) + q)) = w;
-                        }
+                        for (int q = 0; q < 16; ++q) w[q] = tc::pack_bf16(pv[2 * q], pv[2 * q + 1]);
+                        if (SA_BOUNDS(384 + 64 * pb + jc / 2 + 16 <= tmem_cols(MODE), status))
+                            tc::tmem_st16(tP + 64 * pb + lanebase + jc / 2, w);
                     }
                 }
                 if (HASX) {
-                    tc::fence_async_smem();
+                    // the stores have landed before the MMA that reads them is issued
+                    tc::tmem_wait_st();
+                    tc::tc_fence_before();
                     __syncwarp();
                     if (lane == 0) tc::mbar_arrive(bar + B_PFULL + pb);
                 }
