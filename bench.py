@@ -76,7 +76,11 @@ CONTRACTIONS = {"lse_sweep": 1, "pv": 2, "wsum": 1, "ds": 3}
 # DRAM bytes (read + write) per launch from one ncu capture (profiles/), keyed by
 # (workload, kernel kind), with the SHA-256 of the kernel source the capture was
 # taken from: a changed source reports traffic as null until it is captured again.
-MEASURED_TRAFFIC = {}
+MEASURED_TRAFFIC = {
+    # profiles/tc_rowsum_sweep_long32k.md: 164.82 MB read + 13.13 MB written
+    ("long32k", "lse_sweep"): (177.95e6, "banded_log_domain_b200/csrc/tc_rowsum.cuh",
+                               "292bb96804b5a375b12e033d68de11f81811411f889321dd8b00fd213dce88c1"),
+}
 
 
 def measured_traffic(workload, kind):
