@@ -119,11 +119,15 @@ sa_status sinkhorn_attn_state_size(const sa_params* p, size_t* n_floats);
 
 /* Workspace bytes needed by sinkhorn_attn_fwd and sinkhorn_attn_bwd (either
  * pointer may be NULL).  Both are O(B*H*L) and include a 256-byte status
- * header at offset 0.  The backward's grows with R (a few float32 vectors of
- * B*H*(L+dustbin) per tail step); it holds four bf16 [B][H][L][16] arrays
- * (the modifier's operands of the bf16 dS contraction, 128 bytes per token),
- * and for R > 4 a float32 [B][H][L][d] sum of the dQ / dK sweeps over blocks of
- * at most 8 modifier terms. */
+ * header at offset 0.  With bf16 storage and no dustbin (the tensor-core
+ * path) both hold a working copy of the dual state: per dual, log2(e) times
+ * its value as float32 and a bf16 [16] operand row per token (the dual divided
+ * by the score scale, split in three bf16 parts), 36 bytes per token and dual.
+ * The backward's grows with R (a few float32 vectors of B*H*(L+dustbin) per
+ * tail step); it holds four bf16 [B][H][L][16] arrays (the modifier's
+ * operands of the bf16 dS contraction, 128 bytes per token), and for R > 4 a
+ * float32 [B][H][L][d] sum of the dQ / dK sweeps over blocks of at most 8
+ * modifier terms. */
 sa_status sinkhorn_attn_workspace_size(const sa_params* p, size_t* fwd_bytes, size_t* bwd_bytes);
 
 /*
