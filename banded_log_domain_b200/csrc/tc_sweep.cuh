@@ -10,12 +10,14 @@
 // One CTA owns a block of 128 rows (TMEM lanes) of one (batch, head) problem
 // and walks the band's column chunks [r0 - W, r0 + 127 + W] in steps of 128.
 //
-// Warp roles (320 threads):
-//   warps 0-7  epilogue: warp w reads TMEM lanes 32*(w%4)..+31 (its rows) and
-//              columns 64*(w/4)..+63 of each chunk;
-//   warp 8     loader: TMA tiles (lane 0) and the chunk's column vectors
-//              (all lanes) into a ring of NST stages;
-//   warp 9     MMA issuer (lane 0).
+// Warp roles:
+//   NEPI epilogue warps (16 for PV, 8 for the others): warp w reads TMEM lanes
+//              32*(w%4)..+31 (its rows) and a 128/(NEPI/4)-column part of each
+//              chunk;
+//   a loader:  TMA tiles (lane 0) and the chunk's column vectors (all lanes)
+//              into a ring of NST stages;
+//   a score-MMA issuer, and for PV and dS a second issuer for P X (one
+//              elected lane each).
 // Pipelines are mbarriers; every wait is bounded and a timeout records
 // SA_ERR_TIMEOUT in the status word and unwinds.
 //
@@ -40,7 +42,6 @@ constexpr int LSE = simt::LSE, WSUM = simt::WSUM, PV = simt::PV, DS1 = simt::DS1
 // 8 for the others (each warp 64 columns; LSE and WSUM run two CTAs per SM, the
 // dS modes need the registers); then the loader warp and the MMA warp.
 __host__ __device__ constexpr int nepi(int m) { return m == simt::PV ? 16 : 8; }
-__host__ __device__ constexpr int nthreads(int m) { return (nepi(m) + 2) * 32; }
 constexpr int TILE = 16384;  // one 128 x 64 bf16 tile
 constexpr long long kWaitBudget = 4000000000LL;  // clock cycles (about 2 s)
 
@@ -50,6 +51,9 @@ struct Maps {
 
 __host__ __device__ constexpr bool is_ds(int m) { return m == DS1 || m == DSD; }
 __host__ __device__ constexpr bool has_x(int m) { return m == PV || is_ds(m); }
+// the epilogue warps, the loader, the score-MMA issuer, and for the modes with
+// a P X contraction a second issuer for it
+__host__ __device__ constexpr int nthreads(int m) { return (nepi(m) + (has_x(m) ? 3 : 2)) * 32; }
 // operand stages: five for PV and DS1 (their P tiles live in TMEM, which leaves
 // the shared memory to the stages), four for the others
 constexpr int NST_MAX = 5;
@@ -192,7 +196,7 @@ __global__ void __launch_bounds__(nthreads(MODE), ctas_per_sm(MODE)) tc_band_swe
     constexpr int NST = nst(MODE), NSB = nsb(MODE), NAB = nab(MODE);
     constexpr bool DS = is_ds(MODE), HASX = has_x(MODE);
     constexpr int NEPI = nepi(MODE), NPART = NEPI / 4, PW = 128 / NPART, NG = PW / 32;
-    constexpr int W_LOAD = NEPI, W_MMA = NEPI + 1;
+    constexpr int W_LOAD = NEPI, W_MMA = NEPI + 1, W_MMA2 = NEPI + 2;
     uint64_t* bar = reinterpret_cast<uint64_t*>(sm + off_bar(MODE, NT));
     uint32_t* tbase = reinterpret_cast<uint32_t*>(sm + off_bar(MODE, NT) + 64 * 8);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tbase + 1);
@@ -255,7 +259,7 @@ __global__ void __launch_bounds__(nthreads(MODE), ctas_per_sm(MODE)) tc_band_swe
             tc::mbar_init(bar + B_FULL + s, AUGS ? 1 : 33);  // the TMA bytes (+ 32 lanes' vectors)
             tc::mbar_init(bar + B_EMPTY + s, NEPI + 1);
         }
-        tc::mbar_init(bar + B_DRAIN, 1);
+        tc::mbar_init(bar + B_DRAIN, HASX ? 2 : 1);  // every MMA issuer
         tc::mbar_init(bar + B_EPI, NEPI);
         *abort_flag = 0;
         tc::fence_mbar_init();
@@ -395,10 +399,13 @@ __global__ void __launch_bounds__(nthreads(MODE), ctas_per_sm(MODE)) tc_band_swe
                 tc::mbar_wait(bar + B_FULL + x % NST, (x / NST) & 1, kWaitBudget);
         }
         __syncwarp();
-    } else if (warp == W_MMA) {
-        // ------------------------------------------------------------ MMA issuer
+    } else if (warp == W_MMA || (HASX && warp == W_MMA2)) {
+        // ------------------------------------------------------------ MMA issuers
         // The whole warp runs the loop (uniform control flow and values); one
-        // elected lane issues the MMAs and commits.
+        // elected lane issues the MMAs and commits.  W_MMA issues the score
+        // contractions; for the modes with one, W_MMA2 issues P X, so that
+        // neither stream of MMA instructions waits behind the other's issue.
+        const bool pvw = HASX && warp == W_MMA2;
         {
             const uint32_t id_s = tc::idesc_bf16(128, 128, false, false);
             const uint32_t id_o = tc::idesc_bf16(128, 64, false, true);
@@ -431,48 +438,54 @@ __global__ void __launch_bounds__(nthreads(MODE), ctas_per_sm(MODE)) tc_band_swe
             };
             bool ok = true;
             int gc = 0;
-            int pg = -1, pit = 0, pc = 0, pn = 0;  // the chunk whose P X is still to issue
             Cursor cur = cur0;
-            for (int it = 0; ok && it < ntl; ++it, cur.next(nblk, a.H)) {
-                const Tile tl = tile(cur);
-                const int ab = it % NAB;
-                if (!ctl.wait(B_AFULL + ab, (it / NAB) & 1)) { ok = false; break; }
-                const uint64_t dA = tc::sdesc_add(dA0, off_a(MODE, ab));
-                for (int c = 0; c < tl.nch; ++c, ++gc) {
-                    const int s = gc % NST, b = gc % NSB;
-                    if (!ctl.wait(B_FULL + s, (gc / NST) & 1)) { ok = false; break; }
-                    if (gc >= NSB && !ctl.wait(B_SEMPTY + b, ((gc / NSB) - 1) & 1)) { ok = false; break; }
-                    tc::tc_fence_after();
-                    const uint64_t dB = tc::sdesc_add(dStK, s * stage_bytes(MODE));
-                    if (tc::elect_one()) {
-#pragma unroll
-                        for (int k = 0; k < 4; ++k)
-                            tc::mma_bf16(tS + 128 * b, tc::sdesc_add(dA, 32 * k), tc::sdesc_add(dB, 32 * k),
-                                         id_s, k > 0);
-                        if (AUGS)  // + the column duals
-                            tc::mma_bf16(tS + 128 * b, dAug, tc::sdesc_add(dAug, AUG_BYTES * (1 + s)), id_s, 1u);
-                        if (DS) {
-#pragma unroll
-                            for (int k = 0; k < 4; ++k)
-                                tc::mma_bf16(tG, tc::sdesc_add(dA2, 32 * k), tc::sdesc_add(dB, TILE + 32 * k),
-                                             id_s, k > 0);
-                            if (AUG)  // + the modifier, one more K16 step
-                                tc::mma_bf16(tG, dAug, tc::sdesc_add(dAug, AUG_BYTES * (1 + s)), id_s, 1u);
-                        }
-                        tc::tc_commit(bar + B_SFULL + b);
-                        if (!HASX) tc::tc_commit(bar + B_EMPTY + s);
-                    }
-                    __syncwarp();
-                    if (HASX) {
-                        if (pg >= 0 && !issue_pv(pg, pit, pc, pn)) { ok = false; break; }
-                        pg = gc; pit = it; pc = c; pn = tl.nch;
+            if (pvw) {
+                for (int it = 0; ok && it < ntl; ++it, cur.next(nblk, a.H)) {
+                    const Tile tl = tile(cur);
+                    for (int c = 0; c < tl.nch; ++c, ++gc) {
+                        // the stage's X tile has landed (its phase cannot move on before
+                        // this warp's commit releases the stage)
+                        if (!ctl.wait(B_FULL + gc % NST, (gc / NST) & 1)) { ok = false; break; }
+                        if (!issue_pv(gc, it, c, tl.nch)) { ok = false; break; }
                     }
                 }
-                if (!ok) break;
-                if (tc::elect_one()) tc::tc_commit(bar + B_AEMPTY + ab);  // every score MMA of the tile has read A
-                __syncwarp();
+            } else {
+                for (int it = 0; ok && it < ntl; ++it, cur.next(nblk, a.H)) {
+                    const Tile tl = tile(cur);
+                    const int ab = it % NAB;
+                    if (!ctl.wait(B_AFULL + ab, (it / NAB) & 1)) { ok = false; break; }
+                    const uint64_t dA = tc::sdesc_add(dA0, off_a(MODE, ab));
+                    for (int c = 0; c < tl.nch; ++c, ++gc) {
+                        const int s = gc % NST, b = gc % NSB;
+                        if (!ctl.wait(B_FULL + s, (gc / NST) & 1)) { ok = false; break; }
+                        if (gc >= NSB && !ctl.wait(B_SEMPTY + b, ((gc / NSB) - 1) & 1)) { ok = false; break; }
+                        tc::tc_fence_after();
+                        const uint64_t dB = tc::sdesc_add(dStK, s * stage_bytes(MODE));
+                        if (tc::elect_one()) {
+#pragma unroll
+                            for (int k = 0; k < 4; ++k)
+                                tc::mma_bf16(tS + 128 * b, tc::sdesc_add(dA, 32 * k), tc::sdesc_add(dB, 32 * k),
+                                             id_s, k > 0);
+                            if (AUGS)  // + the column duals
+                                tc::mma_bf16(tS + 128 * b, dAug, tc::sdesc_add(dAug, AUG_BYTES * (1 + s)), id_s, 1u);
+                            if (DS) {
+#pragma unroll
+                                for (int k = 0; k < 4; ++k)
+                                    tc::mma_bf16(tG, tc::sdesc_add(dA2, 32 * k), tc::sdesc_add(dB, TILE + 32 * k),
+                                                 id_s, k > 0);
+                                if (AUG)  // + the modifier, one more K16 step
+                                    tc::mma_bf16(tG, dAug, tc::sdesc_add(dAug, AUG_BYTES * (1 + s)), id_s, 1u);
+                            }
+                            tc::tc_commit(bar + B_SFULL + b);
+                            if (!HASX) tc::tc_commit(bar + B_EMPTY + s);
+                        }
+                        __syncwarp();
+                    }
+                    if (!ok) break;
+                    if (tc::elect_one()) tc::tc_commit(bar + B_AEMPTY + ab);  // every score MMA of the tile has read A
+                    __syncwarp();
+                }
             }
-            if (HASX && ok && pg >= 0) ok = issue_pv(pg, pit, pc, pn);
             // drain: every MMA issued above has completed once this arrives
             if (tc::elect_one()) tc::tc_commit(bar + B_DRAIN);
             __syncwarp();
