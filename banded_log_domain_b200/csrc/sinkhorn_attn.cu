@@ -541,6 +541,41 @@ bool make_map_aug_strided(CUtensorMap* m, const void* ptr, int L, int BH, long l
            CUDA_SUCCESS;
 }
 
+// SMs of the device (persistent grids take one or two CTAs per SM); read once
+// from the first device asked, since the library targets a single GPU model
+// (sm_100a)
+int sm_count() {
+    static int nsm = 0;
+    if (nsm == 0) {
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || nsm <= 0)
+            nsm = 148;
+    }
+    return nsm;
+}
+
+// Launches a persistent sweep with programmatic stream serialisation: its
+// CTAs may be placed while the previous kernel of the stream finishes, so their
+// set-up (barrier init, TMEM allocation) overlaps its tail; the sweeps wait for
+// that kernel (griddepcontrol.wait) before any global access, so the ordering
+// of their reads and writes is that of a plain launch.
+template <typename... Params, typename... Args>
+cudaError_t launch_pdl(void (*kern)(Params...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                       Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
 template <int MODE, bool ONLINE, int NT>
 cudaError_t launch_tc(const simt::SweepArgs& a, int BH, cudaStream_t st, Tracer& tr,
                       int* status) {
@@ -558,35 +593,18 @@ cudaError_t launch_tc(const simt::SweepArgs& a, int BH, cudaStream_t st, Tracer&
              make_map_aug_strided(&maps.AC, a.augc, a.L, BH, a.aug_s);
     }
     if (!ok) return cudaErrorInvalidValue;
-    // persistent: one CTA per SM (two for LSE and WSUM), each a contiguous tile range
-    static int nsm = 0;
-    if (nsm == 0) {
-        int dev = 0;
-        if (cudaGetDevice(&dev) != cudaSuccess ||
-            cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || nsm <= 0)
-            nsm = 148;
-    }
+    // persistent: one CTA per SM (two for the online LSE sweep), each a contiguous tile range
     const long long ntiles = (long long)((a.L + 127) / 128) * BH;
-    const dim3 grid((unsigned)std::min<long long>(ntiles, (long long)nsm * tcs::ctas_per_sm(MODE)));
+    const dim3 grid((unsigned)std::min<long long>(ntiles, (long long)sm_count() * tcs::ctas_per_sm(MODE)));
     const int smem = tcs::smem_bytes(MODE, NT);
     cudaError_t e = cudaFuncSetAttribute(tcs::tc_band_sweep<MODE, ONLINE, NT>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     tr.begin(kind_of(MODE));
-    tcs::tc_band_sweep<MODE, ONLINE, NT><<<grid, tcs::nthreads(MODE), smem, st>>>(a, maps, status, BH);
+    e = launch_pdl(tcs::tc_band_sweep<MODE, ONLINE, NT>, grid, dim3(tcs::nthreads(MODE)), smem, st, a, maps,
+                   status, BH);
     tr.end();
-    return cudaGetLastError();
-}
-
-int sm_count() {
-    static int nsm = 0;
-    if (nsm == 0) {
-        int dev = 0;
-        if (cudaGetDevice(&dev) != cudaSuccess ||
-            cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || nsm <= 0)
-            nsm = 148;
-    }
-    return nsm;
+    return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 // Exponentials of every 32 entries of a row-sum sweep's in-band group that run
@@ -621,9 +639,9 @@ cudaError_t launch_rowsum(const simt::SweepArgs& a, int BH, cudaStream_t st, Tra
                                          tcr::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     tr.begin(kind_of(MODE));
-    kern<<<grid, tcr::NTHREADS, tcr::SMEM_BYTES, st>>>(a, maps, status, BH);
+    e = launch_pdl(kern, grid, dim3(tcr::NTHREADS), tcr::SMEM_BYTES, st, a, maps, status, BH);
     tr.end();
-    return cudaGetLastError();
+    return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 template <typename T, int MODE>

@@ -190,6 +190,19 @@ __device__ __forceinline__ void fence_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// Programmatic dependent launch.  grid_dep_wait returns once the grids this
+// one depends on (the previous kernel of the stream, when it was launched with
+// programmatic stream serialisation) have completed and their memory writes
+// are visible; grid_dep_launch lets the next such kernel start launching once
+// every CTA of this grid has signalled (or exited).  Without the launch
+// attribute both return at once.
+__device__ __forceinline__ void grid_dep_wait() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void grid_dep_launch() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // One lane of the (converged) warp, the same one for the same mask: the
 // issuing thread of a tcgen05 operation.  The code around it stays
 // warp-uniform, which keeps descriptors and addresses in uniform registers;

@@ -313,6 +313,11 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_rowsum_sweep(const SweepArgs a
     __syncthreads();
     tc::tc_fence_after();
     const uint32_t tS = *tbase;  // score buffer b at columns 128 b
+    // The set-up above overlaps the previous kernel's tail; every global
+    // access comes after this wait.  Then the next sweep may begin launching:
+    // its CTAs take an SM only as this grid's leave it.
+    tc::grid_dep_wait();
+    tc::grid_dep_launch();
 
     if (warp == W_LOAD) {
         // ------------------------------------------------------------ loader

@@ -275,6 +275,10 @@ __global__ void __launch_bounds__(nthreads(MODE), ctas_per_sm(MODE)) tc_band_swe
     // TMEM columns: S buffer b at 128*b (DS: S at 0, G at 128); O buffer ob at
     // 256 + 64*ob; P (or dS) buffer pb, 128 bf16 per row, at 384 + 64*pb
     const uint32_t tS = tm, tG = tm + 128, tO = tm + 256, tP = tm + 384;
+    // The set-up above overlaps the previous kernel's tail; every global
+    // access comes after this wait.  Then the next kernel may begin launching.
+    tc::grid_dep_wait();
+    tc::grid_dep_launch();
 
     if (warp == W_LOAD) {
         // ------------------------------------------------------------ loader

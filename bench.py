@@ -14,7 +14,9 @@ independent, so there is no data-path collective) and the step time is the
 maximum over ranks.
 
 Extra keys: ``roofline`` for the dominant kernel (per-launch CUDA events
-recorded by the library around each launch, see sa_params.trace_*),
+recorded by the library around each launch, see sa_params.trace_*, in up to 10
+traced replicas of the step run after the timed ones, which carry no such
+events),
 ``cpu_baseline`` (the CPU oracle on a bounded sample, rank 0 at N=1), ``e2e``
 (the same step through the library's host-buffer call
 ``sinkhorn_attn_step_host``: pinned-host inputs copied in and the results copied
@@ -399,24 +401,35 @@ def main():
     launches = 0
     torch.cuda.synchronize()
     barrier(ws)
+    # the timed steps run without the library's per-launch trace events (which
+    # sit between the kernels); the per-kernel breakdown and the launch count
+    # come from traced replicas of the same step right after them
     for _ in range(args.steps):
         flush.zero_()
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
         e0.record(stream)
-        step()
+        step(trace=False)
         e1.record(stream)
         torch.cuda.synchronize()
         step_ms.append(e0.elapsed_time(e1))
+    torch.cuda.synchronize()
+    barrier(ws)
+    clk = clocks.stop()
+    n_traced = min(args.steps, 10)
+    for _ in range(n_traced):
+        flush.zero_()
+        step()
+        torch.cuda.synchronize()
         for tr in (tr_f, tr_b):
             launches += tr.count.value
             for kind, ms in tr.durations():
                 a = kern.setdefault(kind, [0.0, 0])
                 a[0] += ms
                 a[1] += 1
+    launches = launches * args.steps // max(n_traced, 1)
     torch.cuda.synchronize()
     barrier(ws)
-    clk = clocks.stop()
     total_ms = allreduce_max(sum(step_ms), ws)
     ms_per_step = total_ms / args.steps
     units = w.B * w.H * w.L
@@ -445,7 +458,7 @@ def main():
         roof = {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                 "frac": achieved / peak, "traffic": None, "kernel": dom_kind,
                 "peak_source": "FP32 FFMA: 148 SMs x 128 lanes x 2 FLOP x max SM clock",
-                "launches_per_step": dom_n / args.steps, "avg_launch_ms": avg_ms}
+                "launches_per_step": dom_n / n_traced, "avg_launch_ms": avg_ms}
     else:
         # the burst peak: each launch is well under a millisecond, inside a step of a
         # few milliseconds, not a seconds-long loop under the power cap
@@ -454,7 +467,7 @@ def main():
                 "frac": achieved / peak, "traffic": measured_traffic(w.name, dom_kind),
                 "kernel": dom_kind,
                 "peak_source": f"{peaks['source']} bf16 dense (burst)",
-                "launches_per_step": dom_n / args.steps, "avg_launch_ms": avg_ms,
+                "launches_per_step": dom_n / n_traced, "avg_launch_ms": avg_ms,
                 "exp_per_s": exp_rate, "exp_frac_of_mufu": (exp_rate / mufu_peak) if exp_rate else None,
                 "mufu_peak_per_s": mufu_peak}
     # the whole step against the method's roofline: (T + R + 9) band contractions at the
@@ -463,7 +476,7 @@ def main():
     step_flops = (w.T + w.R + 9) * unit_flops
     step_bytes = w.B * w.H * w.L * w.d * elt * 12 + 12 * 4 * w.B * w.H * (w.L + w.dustbin)
     t_roof = max(step_flops / (peaks["bf16_tflops"] * 1e12), step_bytes / (peaks["hbm_gbs"] * 1e9))
-    kernels = {kd: {"ms_per_step": a[0] / args.steps, "launches_per_step": a[1] / args.steps,
+    kernels = {kd: {"ms_per_step": a[0] / n_traced, "launches_per_step": a[1] / n_traced,
                     "share": a[0] / max(sum(b[0] for b in kern.values()), 1e-9)}
                for kd, a in kern.items()}
 
