@@ -161,6 +161,8 @@ BwdLayout bwd_layout(const Dims& d, const sa_params* p) {
 template <typename T>
 __global__ void k_rowdot(const T* X, const T* Y, const uint8_t* mask, int L, int H, int ld,
                          int BH, float* out) {
+    tc::grid_dep_wait();  // launched with programmatic stream serialisation
+    tc::grid_dep_launch();
     constexpr int VE = 16 / (int)sizeof(T), LPT = kD / VE;  // elements per load, lanes per token
     static_assert(32 % LPT == 0, "a token's lanes share a warp");
     const long long g = (long long)blockIdx.x * blockDim.x + threadIdx.x;
@@ -186,6 +188,8 @@ __global__ void k_rowdot(const T* X, const T* Y, const uint8_t* mask, int L, int
 // zero on masked tokens.  state: [BH][2R+2][ld].
 __global__ void k_orbit(const float* state, int R, int L, int H, int ld, int BH,
                         const uint8_t* mask, float* eu, float* ev, size_t vstride) {
+    tc::grid_dep_wait();  // launched with programmatic stream serialisation
+    tc::grid_dep_launch();
     const long long g = (long long)blockIdx.x * blockDim.x + threadIdx.x;
     if (g >= (long long)BH * ld) return;
     const int bh = (int)(g / ld), t = (int)(g % ld);
@@ -201,6 +205,8 @@ __global__ void k_orbit(const float* state, int R, int L, int H, int ld, int BH,
 
 // out = s * x * y elementwise over BH*ld (x or y null means 1).
 __global__ void k_vmul(const float* x, const float* y, float s, float* out, long long n) {
+    tc::grid_dep_wait();  // launched with programmatic stream serialisation
+    tc::grid_dep_launch();
     const long long g = (long long)blockIdx.x * blockDim.x + threadIdx.x;
     if (g >= n) return;
     float v = s;
@@ -215,6 +221,8 @@ __global__ void k_vmul(const float* x, const float* y, float s, float* out, long
 __global__ void k_work(const float* state, int nrows, int ld, int L, int H, int BH,
                        const uint8_t* mask, int r_lo, int r_hi, float inv_c, float* work,
                        __nv_bfloat16* aug, int* status) {
+    tc::grid_dep_wait();  // launched with programmatic stream serialisation
+    tc::grid_dep_launch();
     const long long g = (long long)blockIdx.x * blockDim.x + threadIdx.x;
     const int nr = r_hi - r_lo;
     if (g >= (long long)BH * nr * L) return;
@@ -345,6 +353,8 @@ __device__ __forceinline__ void put_aug_row(const Vec (&v)[4], int n, bool row, 
     o[1] = make_uint4(w[4], w[5], w[6], w[7]);
 }
 __global__ void k_aug(AugTerms tm, int L, int BH) {
+    tc::grid_dep_wait();  // launched with programmatic stream serialisation
+    tc::grid_dep_launch();
     const long long g = (long long)blockIdx.x * blockDim.x + threadIdx.x;
     if (g >= (long long)BH * L) return;
     const int bh = (int)(g / L), t = (int)(g % L);
@@ -723,11 +733,11 @@ struct Ctx {
         if (!work) return SA_OK;
         const long long n = (long long)d.BH * (hi - lo) * d.L;
         tr.begin(SA_KERNEL_AUX);
-        k_work<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(state, 2 * d.R + 2, d.ld, d.L, d.H,
-                                                             d.BH, mask, lo, hi, 1.0f / c, work,
-                                                             waug, status);
+        const cudaError_t e = launch_pdl(k_work, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, st, state,
+                                         2 * d.R + 2, d.ld, d.L, d.H, d.BH, mask, lo, hi, 1.0f / c, work,
+                                         waug, status);
         tr.end();
-        return cudaGetLastError() == cudaSuccess ? SA_OK : SA_ERR_CUDA;
+        return (e == cudaSuccess && cudaGetLastError() == cudaSuccess) ? SA_OK : SA_ERR_CUDA;
     }
     // sharded calls: the neighbours' values into the halo entries of a vector
     // just produced (rows of d.L entries, row_stride apart)
@@ -863,10 +873,10 @@ sa_status bwd_impl(const Ctx& x, const T* q, const T* k, const T* v, const uint8
     // a = rowdot(dO, O); orbit factors
     {
         const long long thr = nvec * (kD / (16 / (long long)sizeof(T)));
-        SA_AUX(x.tr, k_rowdot<T><<<(unsigned)((thr + 255) / 256), 256, 0, x.st>>>(
-                         dO, o, mask, d.L, d.H, d.ld, d.BH, A_));
-        SA_AUX(x.tr, k_orbit<<<egrid, eb, 0, x.st>>>(x.state, R, d.L, d.H, d.ld, d.BH, mask,
-                                                     W_(l.eu, 0), W_(l.ev, 0), vstride));
+        SA_AUX(x.tr, SA_CUDA(launch_pdl(k_rowdot<T>, dim3((unsigned)((thr + 255) / 256)), dim3(256), 0,
+                                        x.st, dO, o, mask, d.L, d.H, d.ld, d.BH, A_)));
+        SA_AUX(x.tr, SA_CUDA(launch_pdl(k_orbit, dim3(egrid), dim3(eb), 0, x.st, x.state, R, d.L, d.H,
+                                        d.ld, d.BH, mask, W_(l.eu, 0), W_(l.ev, 0), vstride)));
     }
     const Vec uR = x.srow(2 * R), vR = x.srow(2 * R + 1);
     auto U = [&](int r) { return x.srow(2 * r); };
@@ -920,7 +930,8 @@ sa_status bwd_impl(const Ctx& x, const T* q, const T* k, const T* v, const uint8
             a.augc = x.augrow(2 * r); a.aug_s = x.aug_stride();
             a.w = vec(ub(r), vs);
         } else {
-            SA_AUX(x.tr, k_vmul<<<egrid, eb, 0, x.st>>>(eu(r), ub(r), 1.f, W_(l.w, 0), nvec));
+            SA_AUX(x.tr, SA_CUDA(launch_pdl(k_vmul, dim3(egrid), dim3(eb), 0, x.st,
+                                 eu(r), ub(r), 1.f, W_(l.w, 0), nvec)));
             a.rd = vR; a.cd = uR;
             a.rdw = x.wrow(2 * R + 1); a.cdw = x.wrow(2 * R);
             a.augc = x.augrow(2 * R); a.aug_s = x.aug_stride();
@@ -941,7 +952,8 @@ sa_status bwd_impl(const Ctx& x, const T* q, const T* k, const T* v, const uint8
             b.augc = x.augrow(2 * (r - 1) + 1); b.aug_s = x.aug_stride();
             b.w = vec(vb(r - 1), vs);
         } else {
-            SA_AUX(x.tr, k_vmul<<<egrid, eb, 0, x.st>>>(ev(r - 1), vb(r - 1), 1.f, W_(l.w, 0), nvec));
+            SA_AUX(x.tr, SA_CUDA(launch_pdl(k_vmul, dim3(egrid), dim3(eb), 0, x.st,
+                                 ev(r - 1), vb(r - 1), 1.f, W_(l.w, 0), nvec)));
             b.rd = uR; b.cd = vR;
             b.rdw = x.wrow(2 * R); b.cdw = x.wrow(2 * R + 1);
             b.augc = x.augrow(2 * R + 1); b.aug_s = x.aug_stride();
@@ -965,15 +977,18 @@ sa_status bwd_impl(const Ctx& x, const T* q, const T* k, const T* v, const uint8
     auto slot_k = [&](int i) { return (float*)(ws + l.cv + (size_t)i * l.vec); };
     if (R > 0) {  // R = 0: every dual is a constant and dS = P * G (no terms)
         // k = 0
-        SA_AUX(x.tr, k_vmul<<<egrid, eb, 0, x.st>>>(vb(R), nullptr, -1.f, slot_k(0), nvec));
+        SA_AUX(x.tr, SA_CUDA(launch_pdl(k_vmul, dim3(egrid), dim3(eb), 0, x.st,
+                             vb(R), nullptr, -1.f, slot_k(0), nvec)));
         rq[nt] = none; rk[nt] = vec(slot_k(0), vs);
         eq[nt] = uR; ek[nt] = vR; cq[nt] = none; ck[nt] = vec(slot_k(0), vs); gk[nt] = 1.f;
         ++nt;
         for (int r = 1; r <= R; ++r) {
             if (direct) {
-                SA_AUX(x.tr, k_vmul<<<egrid, eb, 0, x.st>>>(ub(r), nullptr, -1.f, slot_q(nt), nvec));
+                SA_AUX(x.tr, SA_CUDA(launch_pdl(k_vmul, dim3(egrid), dim3(eb), 0, x.st,
+                                     ub(r), nullptr, -1.f, slot_q(nt), nvec)));
             } else {
-                SA_AUX(x.tr, k_vmul<<<egrid, eb, 0, x.st>>>(eu(r), ub(r), -1.f, slot_q(nt), nvec));
+                SA_AUX(x.tr, SA_CUDA(launch_pdl(k_vmul, dim3(egrid), dim3(eb), 0, x.st,
+                                     eu(r), ub(r), -1.f, slot_q(nt), nvec)));
             }
             rq[nt] = vec(slot_q(nt), vs); rk[nt] = vec(ev(r - 1), vs);
             eq[nt] = U(r); ek[nt] = V(r - 1); cq[nt] = vec(slot_q(nt), vs); ck[nt] = none;
@@ -982,12 +997,15 @@ sa_status bwd_impl(const Ctx& x, const T* q, const T* k, const T* v, const uint8
         }
         for (int r = 1; r < R; ++r) {
             if (direct) {
-                SA_AUX(x.tr, k_vmul<<<egrid, eb, 0, x.st>>>(vb(r), nullptr, -1.f, slot_k(nt), nvec));
+                SA_AUX(x.tr, SA_CUDA(launch_pdl(k_vmul, dim3(egrid), dim3(eb), 0, x.st,
+                                     vb(r), nullptr, -1.f, slot_k(nt), nvec)));
                 eq[nt] = U(r); ek[nt] = V(r); cq[nt] = none; ck[nt] = vec(slot_k(nt), vs);
                 gk[nt] = 0.f;
             } else {
-                SA_AUX(x.tr, k_vmul<<<egrid, eb, 0, x.st>>>(eu(r), nullptr, -1.f, slot_q(nt), nvec));
-                SA_AUX(x.tr, k_vmul<<<egrid, eb, 0, x.st>>>(ev(r), vb(r), 1.f, slot_k(nt), nvec));
+                SA_AUX(x.tr, SA_CUDA(launch_pdl(k_vmul, dim3(egrid), dim3(eb), 0, x.st,
+                                     eu(r), nullptr, -1.f, slot_q(nt), nvec)));
+                SA_AUX(x.tr, SA_CUDA(launch_pdl(k_vmul, dim3(egrid), dim3(eb), 0, x.st,
+                                     ev(r), vb(r), 1.f, slot_k(nt), nvec)));
                 rq[nt] = vec(slot_q(nt), vs); rk[nt] = vec(slot_k(nt), vs);
             }
             ++nt;
@@ -1015,7 +1033,7 @@ sa_status bwd_impl(const Ctx& x, const T* q, const T* k, const T* v, const uint8
         }
         tm.n = first;
         for (int i = 0; i < 4; ++i) tm.out[i] = augs[i] = (__nv_bfloat16*)(ws + l.aug + i * one);
-        SA_AUX(x.tr, k_aug<<<(unsigned)((n + 255) / 256), 256, 0, x.st>>>(tm, d.L, d.BH));
+        SA_AUX(x.tr, SA_CUDA(launch_pdl(k_aug, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, x.st, tm, d.L, d.BH)));
     }
     for (int side = 0; side < 2; ++side) {
         for (int tb = 0; tb < nblk_t; ++tb) {
