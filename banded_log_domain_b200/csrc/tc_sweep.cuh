@@ -38,9 +38,12 @@ using simt::SweepArgs;
 using simt::MAXT;
 constexpr int LSE = simt::LSE, WSUM = simt::WSUM, PV = simt::PV, DS1 = simt::DS1,
               DSD = simt::DSD;
+// The modes this kernel runs: the first (online) dual update of a solve, PV and
+// the two dS sweeps; the shifted dual updates and the vector-cotangent sweeps
+// run in tc_rowsum.cuh.
 // Epilogue warps: 16 for PV (one CTA per SM, each warp 32 columns of a chunk),
-// 8 for the others (each warp 64 columns; LSE and WSUM run two CTAs per SM, the
-// dS modes need the registers); then the loader warp and the MMA warp.
+// 8 for the others (each warp 64 columns; the online LSE sweep runs two CTAs per
+// SM, the dS modes need the registers); then the loader and the MMA issuers.
 __host__ __device__ constexpr int nepi(int m) { return m == simt::PV ? 16 : 8; }
 constexpr int TILE = 16384;  // one 128 x 64 bf16 tile
 constexpr long long kWaitBudget = 4000000000LL;  // clock cycles (about 2 s)
@@ -75,7 +78,7 @@ __host__ __device__ constexpr bool augs(int m) { return m == PV; }
 __host__ __device__ constexpr bool has_aug(int m, int nt) { return aug(m, nt) || augs(m); }
 // column vectors staged per operand stage
 __host__ __device__ constexpr int ncv(int m, int nt) {
-    return m == WSUM ? 2 : (m == DS1 ? (aug(m, nt) ? 1 : 1 + nt) : (m == DSD ? 2 * MAXT : 1));
+    return m == DS1 ? (aug(m, nt) ? 1 : 1 + nt) : (m == DSD ? 2 * MAXT : 1);
 }
 __host__ __device__ constexpr int stage_bytes(int m) {
     return TILE * (1 + (is_ds(m) ? 1 : 0) + (m == PV ? 1 : 0));
@@ -85,8 +88,8 @@ __host__ __device__ constexpr int tmem_cols(int m) { return has_x(m) ? 512 : 256
 // row-block operand buffers: two (tile parity) of A for the modes without a second
 // score operand; one of A and A2 for the dS modes (their shared memory is full)
 __host__ __device__ constexpr int nab(int m) { return is_ds(m) ? 1 : 2; }
-// CTAs per SM (LSE and WSUM fit twice)
-__host__ __device__ constexpr int ctas_per_sm(int m) { return (m == LSE || m == WSUM) ? 2 : 1; }
+// CTAs per SM (the online LSE sweep fits twice)
+__host__ __device__ constexpr int ctas_per_sm(int m) { return m == LSE ? 2 : 1; }
 
 // shared-memory carve-up (offsets from a 1024-aligned base)
 __host__ __device__ constexpr int off_a(int m, int i) { return TILE * i; }
@@ -201,6 +204,8 @@ __global__ void __launch_bounds__(nthreads(MODE), ctas_per_sm(MODE)) tc_band_swe
     uint32_t* tbase = reinterpret_cast<uint32_t*>(sm + off_bar(MODE, NT) + 64 * 8);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tbase + 1);
     float* red = reinterpret_cast<float*>(sm + off_red(MODE, NT));
+    static_assert((MODE == LSE && ONLINE) || MODE == PV || MODE == DS1 || MODE == DSD,
+                  "the shifted dual updates and WSUM run in tc_rowsum.cuh");
     constexpr bool AUG = aug(MODE, NT), AUGS = augs(MODE), HAUG = has_aug(MODE, NT);
     static_assert(smem_bytes(MODE, NT) <= 227 * 1024 && smem_bytes(MODE, NT) * ctas_per_sm(MODE) <= 228 * 1024,
                   "shared memory");
@@ -344,7 +349,7 @@ __global__ void __launch_bounds__(nthreads(MODE), ctas_per_sm(MODE)) tc_band_swe
                 // Every load of the chunk (4 columns per lane, each vector, the mask)
                 // is issued before any value is used or stored.
                 {
-                    constexpr int NV = MODE == WSUM ? 2 : (MODE == DS1 ? 1 + NT : (MODE == DSD ? 2 * NT : 1));
+                    constexpr int NV = MODE == DS1 ? 1 + NT : (MODE == DSD ? 2 * NT : 1);
                     float val[4][NV > 0 ? NV : 1];
                     bool inr[4], mok[4];
     #pragma unroll
@@ -357,7 +362,6 @@ __global__ void __launch_bounds__(nthreads(MODE), ctas_per_sm(MODE)) tc_band_swe
                         if (inr[k]) {
                             if (mk) mok[k] = mk[col] != 0;
                             if (MODE != DSD) val[k][0] = a.cd.at(bh, col);
-                            if (MODE == WSUM) val[k][1] = a.w.at(bh, col);
                             if (MODE == DS1 && !AUG) {
     #pragma unroll
                                 for (int e = 0; e < NT; ++e) val[k][1 + e] = a.cv[e].p ? a.cv[e].at(bh, col) : 1.f;
@@ -377,7 +381,6 @@ __global__ void __launch_bounds__(nthreads(MODE), ctas_per_sm(MODE)) tc_band_swe
                         const bool ok = inr[k] && mok[k];
                         colvec(sm, MODE, NT, s, 0)[t] =
                             (MODE == DSD) ? 0.f : (ok ? val[k][0] * kLog2e : -INFINITY);
-                        if (MODE == WSUM) colvec(sm, MODE, NT, s, 1)[t] = ok ? val[k][1] : 0.f;
                         if (MODE == DS1 && !AUG) {
     #pragma unroll
                             for (int e = 0; e < NT; ++e) colvec(sm, MODE, NT, s, 1 + e)[t] = ok ? val[k][1 + e] : 0.f;
@@ -516,8 +519,7 @@ __global__ void __launch_bounds__(nthreads(MODE), ctas_per_sm(MODE)) tc_band_swe
             rok = r < L && (tl.mk == nullptr || tl.mk[r] != 0);
             rd2 = 0.f;
             if (r < L) {
-                if (MODE == LSE) rd2 = ONLINE ? 0.f : a.rd.at(tl.bh, r) * kLog2e;
-                else if (MODE != DSD) rd2 = a.rd.at(tl.bh, r) * kLog2e;
+                if (MODE != LSE && MODE != DSD) rd2 = a.rd.at(tl.bh, r) * kLog2e;
             }
 #pragma unroll
             for (int k = 0; k < NT; ++k) {
@@ -593,15 +595,7 @@ __global__ void __launch_bounds__(nthreads(MODE), ctas_per_sm(MODE)) tc_band_swe
             const int bh = tl.bh, r0 = tl.r0, cbeg = tl.cbeg, nch = tl.nch;
             const int r = r0 + lr;              // global row
             const int rw0 = r0 + qd * 32;       // first row of this warp
-            // WSUM: the output's base and multiplier, loaded now, used after the
-            // chunk loop
-            float bb = 0.f, mu = 1.f;
-            if (MODE == WSUM && r < L) {
-                bb = a.base.p ? a.base.at(bh, r) : 0.f;
-                mu = a.mult.p ? a.mult.at(bh, r) : 1.f;
-            }
-            float m = -INFINITY, acc = 0.f;   // LSE online max / running sum; WSUM sum
-            uint64_t accp[4] = {0, 0, 0, 0};  // packed partial sums (LSE with shift, WSUM)
+            float m = -INFINITY, acc = 0.f;   // LSE online max / running sum
 
             for (int c = 0; c < nch; ++c, ++gc) {
                 const int s = gc % NST, b = gc % NSB, pb = gc & 1;
@@ -658,7 +652,7 @@ __global__ void __launch_bounds__(nthreads(MODE), ctas_per_sm(MODE)) tc_band_swe
                     const bool all_in = (cg >= rw0 + 31 - W) && (cg + 31 <= rw0 + W) && cg + 31 < L;
                     const bool all_out = (cg + 31 < rw0 - W) || (cg > rw0 + 31 + W) || cg >= L;
                     const float* ce = cvs + 32 * g;
-                    if (MODE == LSE || MODE == WSUM || MODE == PV) {
+                    if (MODE == LSE || MODE == PV) {
                         if (all_out) {
                             if (MODE == PV) {
     #pragma unroll
@@ -668,7 +662,7 @@ __global__ void __launch_bounds__(nthreads(MODE), ctas_per_sm(MODE)) tc_band_swe
                             float x[32];
                             if (AUGS) group_args_s(sv, rd2, c2, !all_in, r, cg, W, L, x);
                             else group_args(sv, ce, rd2, c2, !all_in, r, cg, W, L, x);
-                            if (MODE == LSE && ONLINE) {
+                            if (MODE == LSE) {
                                 float mloc = -INFINITY;
     #pragma unroll
                                 for (int j = 0; j < 32; ++j) mloc = fmaxf(mloc, x[j]);
@@ -679,24 +673,6 @@ __global__ void __launch_bounds__(nthreads(MODE), ctas_per_sm(MODE)) tc_band_swe
                                 if (m != -INFINITY) {
     #pragma unroll
                                     for (int j = 0; j < 32; ++j) acc += ex2(x[j] - m);
-                                }
-                            } else if (MODE == LSE) {
-    #pragma unroll
-                                for (int q = 0; q < 16; ++q)
-                                    accp[q & 3] = tc::add2(accp[q & 3],
-                                                           tc::pk2(ex2(x[2 * q]), ex2(x[2 * q + 1])));
-                            } else if (MODE == WSUM) {
-                                const float4* w4 = reinterpret_cast<const float4*>(
-                                    colvec(sm, MODE, NT, s, 1) + PW * pt + 32 * g);
-    #pragma unroll
-                                for (int q = 0; q < 8; ++q) {
-                                    const float4 wv = w4[q];
-                                    accp[(2 * q) & 3] =
-                                        tc::fma2(tc::pk2(ex2(x[4 * q]), ex2(x[4 * q + 1])),
-                                                 tc::pk2(wv.x, wv.y), accp[(2 * q) & 3]);
-                                    accp[(2 * q + 1) & 3] =
-                                        tc::fma2(tc::pk2(ex2(x[4 * q + 2]), ex2(x[4 * q + 3])),
-                                                 tc::pk2(wv.z, wv.w), accp[(2 * q + 1) & 3]);
                                 }
                             } else {  // PV
     #pragma unroll
@@ -808,41 +784,19 @@ __global__ void __launch_bounds__(nthreads(MODE), ctas_per_sm(MODE)) tc_band_swe
             }
 
             // ---------------------------------------------------------- finish
-            if ((MODE == LSE && !ONLINE) || MODE == WSUM) {
-                float a0, a1, a2, a3, a4, a5, a6, a7;
-                tc::upk2(accp[0], a0, a1);
-                tc::upk2(accp[1], a2, a3);
-                tc::upk2(accp[2], a4, a5);
-                tc::upk2(accp[3], a6, a7);
-                acc = ((a0 + a1) + (a2 + a3)) + ((a4 + a5) + (a6 + a7));
-            }
             const float ce_d = a.dustbin ? a.cd.at(bh, L) * kLog2e : 0.f;
             float* rr = red + (it & 1) * 512;  // double-buffered by tile parity
-            if (MODE == LSE || MODE == WSUM) {
+            if (MODE == LSE) {
                 // combine the two column halves of each row
-                if (MODE == LSE && !ONLINE) m = 0.f;  // the sum is relative to the shift
                 rr[pt * 256 + lr] = m;
                 rr[pt * 256 + 128 + lr] = acc;
                 if (!ctl.epi_sync(eph)) { ok = false; break; }
                 if (pt == 0 && r < L && !*abort_flag) {
                     float m1 = rr[lr], s1 = rr[128 + lr];
                     const float m2 = rr[256 + lr], s2 = rr[384 + lr];
-                    float out = 0.f;
-                    if (MODE == LSE) {
-                        if (ONLINE) {
-                            lse_merge(m1, s1, m2, s2);
-                            if (a.dustbin) lse_merge(m1, s1, a.sd2 + ce_d, 1.f);
-                            out = -(m1 + lg2(s1)) * kLn2;
-                        } else {
-                            float tot = s1 + s2;
-                            if (a.dustbin) tot += ex2(a.sd2 + ce_d + rd2f);
-                            out = (rd2f - lg2(tot)) * kLn2;
-                        }
-                    } else {
-                        float tot = s1 + s2;
-                        if (a.dustbin) tot += ex2(a.sd2 + rd2f + ce_d) * a.w.at(bh, L);
-                        out = bb + a.sgn * mu * tot;
-                    }
+                    lse_merge(m1, s1, m2, s2);
+                    if (a.dustbin) lse_merge(m1, s1, a.sd2 + ce_d, 1.f);
+                    const float out = -(m1 + lg2(s1)) * kLn2;
                     if (SA_BOUNDS(bh < BH && r >= 0, status)) a.out_vec.at(bh, r) = rokf ? out : 0.f;
                 }
             } else if (DS) {
