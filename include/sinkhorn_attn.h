@@ -43,7 +43,8 @@
  *     serialisation (each one's set-up may overlap the end of the kernel
  *     before it on the stream, and every kernel waits for that kernel to
  *     complete before it touches global memory), so the ordering against the
- *     caller's own work on the stream is that of ordinary launches.  Conditions found on the device (a non-finite dual or output when
+ *     caller's own work on the stream is that of ordinary launches.
+ *     Conditions found on the device (a non-finite dual or output when
  *     check_finite is set) are recorded in a status word at the start of the
  *     workspace and returned by sinkhorn_attn_poll().
  *   - Masked tokens (mask_i == 0) have exactly zero duals, O, dQ, dK and dV.
