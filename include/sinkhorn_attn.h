@@ -39,10 +39,11 @@
  *     are rejected (make the tensors' device current before the call).
  *   - Work is enqueued asynchronously on `stream` (a cudaStream_t; NULL means
  *     the legacy default stream).  Argument and launch errors are returned at
- *     once.  The library's kernels are launched with programmatic stream
- *     serialisation (each one's set-up may overlap the end of the kernel
- *     before it on the stream, and every kernel waits for that kernel to
- *     complete before it touches global memory), so the ordering against the
+ *     once.  The tensor-core sweeps and the O(L) kernels between them are
+ *     launched with programmatic stream serialisation (a kernel's set-up may
+ *     overlap the end of the kernel before it on the stream, and it waits for
+ *     that kernel to complete before it touches global memory); the other
+ *     kernels are ordinary launches.  Either way the ordering against the
  *     caller's own work on the stream is that of ordinary launches.
  *     Conditions found on the device (a non-finite dual or output when
  *     check_finite is set) are recorded in a status word at the start of the
